@@ -1,0 +1,196 @@
+"""CPU oracle for the Fathom key scan -- TEST INFRASTRUCTURE, not the product.
+
+A ctypes wrapper over ``fathom_oracle.c``: a plain, slow, single-threaded fp64
+statement of the scan (bit-plane packing, reverse water-filling allocation,
+plane-prefix scores, brute-force top-k), written from the Fathom pages
+("Fathom Makes KV-Cache Scans Query-Adaptive for Long-Context Decoding",
+method paragraphs 2-3; arXiv 2609.17652 abstract).  Only ``tests/``,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference leg
+import it.  It imports nothing from the CUDA library and the library imports
+nothing from it.
+
+Every function is pinned in ``tests/test_oracle_pins.py``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fathom_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+_u32p = np.ctypeslib.ndpointer(dtype=np.uint32, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain -O2, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c99",
+                               "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        lib.oracle_plane_words.restype = _i64
+        lib.oracle_plane_words.argtypes = [_i64]
+        lib.oracle_pack_planes.restype = None
+        lib.oracle_pack_planes.argtypes = [_u8p, _i64, _int, _int, _u32p]
+        lib.oracle_prefix_values.restype = None
+        lib.oracle_prefix_values.argtypes = [_u32p, _i64, _int, _int, _int, _u8p]
+        lib.oracle_importance.restype = ctypes.c_double
+        lib.oracle_importance.argtypes = [ctypes.c_double, ctypes.c_double]
+        lib.oracle_allocate.restype = None
+        lib.oracle_allocate.argtypes = [_f64p, _f64p, _int, _int, _u8p]
+        lib.oracle_dequant_prefix.restype = ctypes.c_double
+        lib.oracle_dequant_prefix.argtypes = [ctypes.c_double, ctypes.c_double, _int, ctypes.c_uint]
+        lib.oracle_scores_from_codes.restype = None
+        lib.oracle_scores_from_codes.argtypes = [_u8p, _i64, _int, _f32p, _f32p, _f64p, _u8p, _f64p]
+        lib.oracle_scores_at.restype = None
+        lib.oracle_scores_at.argtypes = [_u8p, _i64, _int, _f32p, _f32p, _f64p, _u8p, _i64p,
+                                         _i64, _f64p]
+        lib.oracle_scores_from_planes.restype = None
+        lib.oracle_scores_from_planes.argtypes = [_u32p, _i64, _int, _f32p, _f32p, _f64p, _u8p,
+                                                  _f64p]
+        lib.oracle_topk.restype = None
+        lib.oracle_topk.argtypes = [_f64p, _i64, _int, _i32p, _f64p]
+        _lib = lib
+        return lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(np.asarray(a), dtype=dtype)
+
+
+def plane_words(n: int) -> int:
+    return int(_load().oracle_plane_words(n))
+
+
+def pack_planes(codes) -> np.ndarray:
+    """[h_kv, n, d/2] nibble codes -> [h_kv, d, 4, W] uint32 plane words."""
+    codes = _c(codes, np.uint8)
+    h_kv, n, half = codes.shape
+    d = 2 * half
+    out = np.zeros((h_kv, d, 4, plane_words(n)), dtype=np.uint32)
+    _load().oracle_pack_planes(codes, n, d, h_kv, out)
+    return out
+
+
+def prefix_values(planes, n: int, t: int) -> np.ndarray:
+    """Value of the first t planes of every (KV head, token, channel): [h_kv, n, d]."""
+    planes = _c(planes, np.uint32)
+    h_kv, d = planes.shape[0], planes.shape[1]
+    out = np.zeros((h_kv, n, d), dtype=np.uint8)
+    _load().oracle_prefix_values(planes, n, d, h_kv, t, out)
+    return out
+
+
+def importance(q: float, sigma: float) -> float:
+    return float(_load().oracle_importance(float(q), float(sigma)))
+
+
+def allocate(q, sigma, budget: int) -> np.ndarray:
+    """One query head: bits per channel, uint8 [d]."""
+    q = _c(q, np.float64)
+    sigma = _c(sigma, np.float64)
+    t = np.zeros(q.shape[0], dtype=np.uint8)
+    _load().oracle_allocate(q, sigma, q.shape[0], int(budget), t)
+    return t
+
+
+def allocate_heads(q, sigma, budget: int) -> np.ndarray:
+    """All query heads: q [h_q, d], sigma [h_kv, d] (head h reads KV head h // G)."""
+    q = np.asarray(q, dtype=np.float64)
+    sigma = np.asarray(sigma, dtype=np.float64)
+    G = q.shape[0] // sigma.shape[0]
+    return np.stack([allocate(q[h], sigma[h // G], budget) for h in range(q.shape[0])])
+
+
+def dequant_prefix(m: float, s: float, t: int, v: int) -> float:
+    return float(_load().oracle_dequant_prefix(float(m), float(s), int(t), int(v)))
+
+
+def scores_from_codes(codes_g, qmin_g, qscale_g, q_h, t_h) -> np.ndarray:
+    codes_g = _c(codes_g, np.uint8)
+    n, half = codes_g.shape
+    out = np.zeros(n, dtype=np.float64)
+    _load().oracle_scores_from_codes(codes_g, n, 2 * half, _c(qmin_g, np.float32),
+                                     _c(qscale_g, np.float32), _c(q_h, np.float64),
+                                     _c(t_h, np.uint8), out)
+    return out
+
+
+def scores_at(codes_g, qmin_g, qscale_g, q_h, t_h, idx) -> np.ndarray:
+    codes_g = _c(codes_g, np.uint8)
+    n, half = codes_g.shape
+    idx = _c(idx, np.int64)
+    out = np.zeros(idx.shape[0], dtype=np.float64)
+    _load().oracle_scores_at(codes_g, n, 2 * half, _c(qmin_g, np.float32),
+                             _c(qscale_g, np.float32), _c(q_h, np.float64), _c(t_h, np.uint8),
+                             idx, idx.shape[0], out)
+    return out
+
+
+def scores_from_planes(planes_g, n: int, qmin_g, qscale_g, q_h, t_h) -> np.ndarray:
+    planes_g = _c(planes_g, np.uint32)
+    d = planes_g.shape[0]
+    out = np.zeros(n, dtype=np.float64)
+    _load().oracle_scores_from_planes(planes_g, n, d, _c(qmin_g, np.float32),
+                                      _c(qscale_g, np.float32), _c(q_h, np.float64),
+                                      _c(t_h, np.uint8), out)
+    return out
+
+
+def topk(scores, k: int):
+    """(index int32 [k], score float64 [k]) by score desc, index asc; pads with -1/-inf."""
+    scores = _c(scores, np.float64)
+    idx = np.zeros(k, dtype=np.int32)
+    val = np.zeros(k, dtype=np.float64)
+    _load().oracle_topk(scores, scores.shape[0], int(k), idx, val)
+    return idx, val
+
+
+def scan_step(codes, qmin, qscale, q, sigma, budget: int, k: int, heads=None):
+    """One decode step for the listed query heads (default: all).
+
+    Returns dict(alloc=[h_q, d] uint8, idx={h: int32[k]}, score={h: float64[k]},
+    scores={h: float64[n]}).
+    """
+    codes = np.asarray(codes)
+    q = np.asarray(q, dtype=np.float64)
+    h_q = q.shape[0]
+    h_kv = codes.shape[0]
+    G = h_q // h_kv
+    alloc = allocate_heads(q, sigma, budget)
+    heads = range(h_q) if heads is None else heads
+    res = dict(alloc=alloc, idx={}, score={}, scores={})
+    for h in heads:
+        g = h // G
+        s = scores_from_codes(codes[g], qmin[g], qscale[g], q[h], alloc[h])
+        i, v = topk(s, k)
+        res["idx"][h] = i
+        res["score"][h] = v
+        res["scores"][h] = s
+    return res
