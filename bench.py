@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of one Fathom decode step: allocation + bit-plane scan + top-k.
+
+Workload (default): the 1M-token decode step -- n = 1,048,576 keys, 8 KV heads
+x d = 128 channels stored as 4-bit channel-major bit planes (512 MiB), 32 bf16
+query heads (GQA 4), budget B = 92 bits per key, top-k = 2048 per query head.
+Inputs are seeded synthetic (synthkv); the planes are packed once, before
+timing, and stay resident in HBM.
+
+One step = fathom_allocate + fathom_scan_topk (plan, sample scan, threshold,
+filtering scan, merge).  Device time per step comes from CUDA events on the
+launching stream; L2 is flushed (256 MiB write) between steps, outside the
+events.  The dominant kernel (the filtering scan) is timed alone with events
+recorded around it by the library's profiling hook.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Under torchrun each rank scores its own session (seed + rank): weak scaling,
+no collective on the data path; the step time is the max over ranks.
+--impl reference times the CPU oracle (the reference arm of this workload) on
+a bounded sample of the same step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Gkeys/s scanned+top-k at 1M ctx, B=92 bits; achieved HBM GB/s vs B200 peak"
+UNIT = "Gkeys/s"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", default="decode_1m")
+    ap.add_argument("--budget", type=int, default=92)
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_desc(cfg, budget, k):
+    return ("%s: n=%d keys, %d KV heads x d=%d (4-bit channel-major bit planes), %d %s query "
+            "heads (GQA %d), B=%d bits/key, top-k=%d" % (
+                cfg["name"], cfg["n"], cfg["h_kv"], cfg["d"], cfg["h_q"], cfg["q_dtype"],
+                cfg["h_q"] // cfg["h_kv"], budget, k))
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+_libcuda = None
+
+
+def event_ms(a, b) -> float:
+    """Elapsed ms between two torch CUDA events recorded by any runtime (the
+    library records the scan-kernel events itself, which torch's own
+    elapsed_time refuses), through the driver's cuEventElapsedTime."""
+    import ctypes
+    global _libcuda
+    if _libcuda is None:
+        _libcuda = ctypes.CDLL("libcuda.so.1")
+        _libcuda.cuEventElapsedTime.restype = ctypes.c_int
+        _libcuda.cuEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p,
+                                                ctypes.c_void_p]
+    ms = ctypes.c_float(0.0)
+    rc = _libcuda.cuEventElapsedTime(ctypes.byref(ms), ctypes.c_void_p(a.cuda_event),
+                                     ctypes.c_void_p(b.cuda_event))
+    if rc != 0:
+        raise RuntimeError("cuEventElapsedTime failed: %d" % rc)
+    return float(ms.value)
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def get_cfg(name):
+    import synthkv
+    cfg = dict(synthkv.CONFIGS[name])
+    cfg["name"] = name
+    return cfg
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(case_np, budget, k, heads):
+    """Oracle allocation + scores + top-k for the listed query heads; returns seconds."""
+    import oracle
+    codes, qmin, qscale, q, sigma = case_np
+    G = q.shape[0] // codes.shape[0]
+    t0 = time.perf_counter()
+    for h in heads:
+        g = h // G
+        t = oracle.allocate(q[h], sigma[g], budget)
+        s = oracle.scores_from_codes(codes[g], qmin[g], qscale[g], q[h], t)
+        oracle.topk(s, k)
+    return time.perf_counter() - t0
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle on a bounded sample of the same step."""
+    import torch
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return
+    cfg = get_cfg(args.config)
+    k = args.k or cfg["k"]
+    import oracle
+    import synthkv
+    oracle.build()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    case = synthkv.make_case(cfg["seed"], cfg["n"], cfg["h_kv"], cfg["h_q"], cfg["d"],
+                             cfg["q_dtype"], device=dev, keep_keys=False)
+    cn = (case.codes.cpu().numpy(), case.qmin.cpu().numpy(), case.qscale.cpu().numpy(),
+          case.q.cpu().numpy().astype(np.float64), case.sigma.cpu().numpy())
+    heads_per_step = 1
+    for i in range(args.warmup):
+        oracle_sample(cn, args.budget, k, [i % cfg["h_q"]])
+    secs = [oracle_sample(cn, args.budget, k, [(args.warmup + i) % cfg["h_q"]])
+            for i in range(args.steps)]
+    t = float(np.mean(secs))
+    value = heads_per_step * cfg["n"] / t / 1e9
+    sample = ("one query head per step (allocation, fp64 scores of all %d keys, brute-force "
+              "top-%d), single thread" % (cfg["n"], k))
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, synthkv)",
+        "config": {"workload": workload_desc(cfg, args.budget, k), "n": cfg["n"],
+                   "budget_bits": args.budget, "k": k, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+# ---------------------------------------------------------------- native --
+
+def run_native(args):
+    import torch
+    world, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl native needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    import bit_plane_kv_scan_b200 as F
+    from bit_plane_kv_scan_b200 import build as fbuild
+    import synthkv
+    fbuild.build()
+
+    cfg = get_cfg(args.config)
+    k = args.k or cfg["k"]
+    B = args.budget
+    n, h_kv, h_q, d = cfg["n"], cfg["h_kv"], cfg["h_q"], cfg["d"]
+    case = synthkv.make_case(cfg["seed"] + rank, n, h_kv, h_q, d, cfg["q_dtype"], device=device,
+                             keep_keys=False)
+    planes = F.pack_planes(case.codes)
+    q = case.q_storage().contiguous()
+    sigma, qmin, qscale = case.sigma, case.qmin, case.qscale
+    alloc = torch.empty((h_q, d), dtype=torch.uint8, device=device)
+    out = (torch.empty((h_q, k), dtype=torch.int32, device=device),
+           torch.empty((h_q, k), dtype=torch.float32, device=device))
+    ws = F.Workspace(device)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        F.allocate(q, sigma, B, out=alloc)
+        F.scan_topk(planes, qmin, qscale, q, alloc, k, n, workspace=ws, out=out)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    sb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    se = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    for ev in kb + ke:  # torch creates an event's handle at its first record
+        ev.record(stream)
+    sampler = ClockSampler(physical_gpu_index(local))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(K):
+        flush.zero_()
+        F.profile_scan_kernel(kb[i], ke[i])
+        sb[i].record(stream)
+        step()
+        se[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    F.profile_scan_kernel(None, None)
+    step_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(sb, se)]))
+    kern_ms = float(np.mean([event_ms(a, b) for a, b in zip(kb, ke)]))
+    rep = F.read_report(ws)
+    t_step = reduce_max(step_ms, world, device)
+    t_kern = reduce_max(kern_ms, world, device)
+
+    # algorithmic bytes of the filtering scan: the union plane prefixes of
+    # every KV head (one plane row = W words), the per-head inputs it reads
+    # (q, alloc, m, s) and the candidates it writes (about 2k per head).
+    W = F.plane_words(n)
+    union_bytes = int(rep.union_planes) * W * 4
+    small_bytes = h_q * d * (q.element_size() + 1) + 2 * h_kv * d * 4
+    alg_bytes = union_bytes + small_bytes
+    peak, peak_kind = load_peaks()
+    achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers: q uploaded from
+    # pinned memory, top-k read back to pinned memory, inside the timed region
+    q_host = q.cpu().pin_memory()
+    q_dev = torch.empty_like(q)
+    idx_host = torch.empty((h_q, k), dtype=torch.int32, pin_memory=True)
+    sc_host = torch.empty((h_q, k), dtype=torch.float32, pin_memory=True)
+    eb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+
+    def e2e_step():
+        q_dev.copy_(q_host, non_blocking=True)
+        F.allocate(q_dev, sigma, B, out=alloc)
+        F.scan_topk(planes, qmin, qscale, q_dev, alloc, k, n, workspace=ws, out=out)
+        idx_host.copy_(out[0], non_blocking=True)
+        sc_host.copy_(out[1], non_blocking=True)
+
+    for _ in range(3):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(K):
+        flush.zero_()
+        eb[i].record(stream)
+        e2e_step()
+        ee[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in zip(eb, ee)])), world,
+                        device)
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = idx_host.numel() * 4 + sc_host.numel() * 4
+
+    keys_per_step = h_q * n * world
+    value = keys_per_step / (t_step * 1e-3) / 1e9
+    e2e_value = keys_per_step / (e2e_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        cn = (case.codes.cpu().numpy(), qmin.cpu().numpy(), qscale.cpu().numpy(),
+              case.q.cpu().numpy().astype(np.float64), sigma.cpu().numpy())
+        heads = list(range(8))
+        secs = oracle_sample(cn, B, k, heads)
+        cpu = {"value": len(heads) * n / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "query heads 0-7 (KV heads 0-1) of this step: allocation, fp64 scores "
+                         "of all %d keys, brute-force top-%d; single thread, %.1f s" % (n, k, secs)}
+
+    if rank == 0:
+        res = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded, synthkv: Qwen3-8B-shaped GQA keys with outlier "
+                    "channels, 4-bit min-max codes)",
+            "config": {"workload": workload_desc(cfg, B, k), "n": n, "h_kv": h_kv, "h_q": h_q,
+                       "d": d, "budget_bits": B, "k": k, "per_rank_sessions": 1,
+                       "l2": "flushed between steps (256 MiB write, outside the events)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind, "kernel": "scan_kernel<4,1> (filtering scan)",
+                         "kernel_ms": t_kern, "algorithmic_bytes": alg_bytes,
+                         "union_planes": int(rep.union_planes)},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 6 * K,
+            "tokens_per_s": n * world / (t_step * 1e-3),
+            "fallback_heads": int(rep.fallback_heads),
+            "max_candidates": int(rep.max_candidates),
+            "clocks": clocks,
+        }
+        if cpu is not None:
+            res["cpu_baseline"] = cpu
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_native(a)

@@ -1,0 +1,338 @@
+// Host side of the C ABI declared in include/fathom.h: argument checks,
+// workspace layout and the launch sequence.  Every check runs before any
+// launch; a failed check launches nothing and returns a status.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "fathom_internal.cuh"
+
+namespace fathom {
+cudaError_t launch_pack(const uint8_t *codes, int64_t n, int d, int h_kv, uint32_t *planes,
+                        cudaStream_t stream);
+cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
+                            int budget, uint8_t *alloc, cudaStream_t stream);
+cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream);
+}  // namespace fathom
+
+using namespace fathom;
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local cudaEvent_t g_prof_begin = nullptr;
+thread_local cudaEvent_t g_prof_end = nullptr;
+
+fathom_status fail(fathom_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+fathom_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(FATHOM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+fathom_status ok() {
+  g_err[0] = 0;
+  return FATHOM_OK;
+}
+
+// Pointer kinds.  A device pointer is device or managed memory; a host-mapped
+// pointer is pinned host memory the device can address.
+enum PtrKind { kPtrDevice, kPtrHostMapped, kPtrOther };
+
+PtrKind ptr_kind(const void *p) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return kPtrOther;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return kPtrDevice;
+  if (a.type == cudaMemoryTypeHost && a.devicePointer == p) return kPtrHostMapped;
+  return kPtrOther;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+#define REQUIRE(cond, ...)                                            \
+  do {                                                                \
+    if (!(cond)) return fail(FATHOM_ERR_INVALID_ARGUMENT, __VA_ARGS__); \
+  } while (0)
+#define REQUIRE_DEV(ptr, name)                                                           \
+  do {                                                                                   \
+    if ((ptr) == nullptr) return fail(FATHOM_ERR_INVALID_ARGUMENT, "%s is NULL", name);   \
+    if (ptr_kind(ptr) != kPtrDevice)                                                     \
+      return fail(FATHOM_ERR_INVALID_ARGUMENT, "%s is not a device pointer", name);      \
+  } while (0)
+
+fathom_status check_shape(int d, int h_q, int h_kv) {
+  if (d < 32 || d > FATHOM_MAX_D || d % 32 != 0)
+    return fail(FATHOM_ERR_UNSUPPORTED, "d=%d: need a multiple of 32 in [32, %d]", d, FATHOM_MAX_D);
+  if (h_kv < 1 || h_q < 1) return fail(FATHOM_ERR_INVALID_ARGUMENT, "h_q=%d h_kv=%d: need >= 1", h_q, h_kv);
+  if (h_q % h_kv != 0)
+    return fail(FATHOM_ERR_INVALID_ARGUMENT, "h_q=%d is not a multiple of h_kv=%d", h_q, h_kv);
+  return FATHOM_OK;
+}
+
+// Workspace layout of one scan launch set.
+struct WsLayout {
+  size_t off_counts, off_tau, off_plans, off_sample, off_cand, total;
+  size_t zero_bytes;  // prefix cleared before every scan
+  int64_t cap, m_max;
+  int sample_rank;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(int S, int64_t n_max, int d, int h_q, int h_kv, int k, uint32_t flags) {
+  WsLayout L;
+  const int64_t heads = (int64_t)S * h_q;
+  const int64_t groups = (int64_t)S * h_kv;
+  L.sample_rank = sample_rank_for(k);
+  int64_t cap = 8 * (int64_t)k;
+  if (cap < 512 * (int64_t)L.sample_rank) cap = 512 * (int64_t)L.sample_rank;
+  if (flags & FATHOM_FLAG_NO_SAMPLING) cap = cap > n_max ? cap : n_max;
+  L.cap = cap + kFallbackSlack;
+  L.m_max = sampling_on(n_max, L.sample_rank, flags) ? sampled_sectors(n_max) * 256 : 0;
+  size_t o = sizeof(WsStatus);
+  L.off_counts = o;
+  o = up256(o + 4 * heads);
+  L.off_tau = o;
+  o = up256(o + 4 * heads);
+  L.zero_bytes = o;
+  L.off_plans = o;
+  o = up256(o + (size_t)groups * plan_layout(d).bytes);
+  L.off_sample = o;
+  o = up256(o + (size_t)heads * L.m_max * 4);
+  L.off_cand = o;
+  o = up256(o + (size_t)heads * L.cap * 8);
+  L.total = o;
+  return L;
+}
+
+void fill_ws(ScanParams &p, const WsLayout &L, void *ws) {
+  unsigned char *b = static_cast<unsigned char *>(ws);
+  p.status = reinterpret_cast<WsStatus *>(b);
+  p.counts = reinterpret_cast<uint32_t *>(b + L.off_counts);
+  p.tau = reinterpret_cast<uint32_t *>(b + L.off_tau);
+  p.plans = b + L.off_plans;
+  p.sample = reinterpret_cast<uint32_t *>(b + L.off_sample);
+  p.cand = reinterpret_cast<unsigned long long *>(b + L.off_cand);
+  p.cap = L.cap;
+  p.m_max = L.m_max;
+  p.sample_rank = L.sample_rank;
+}
+
+fathom_status check_scan_common(int64_t n, int d, int h_q, int h_kv, int k, int q_dtype,
+                                int planes_location) {
+  fathom_status st = check_shape(d, h_q, h_kv);
+  if (st != FATHOM_OK) return st;
+  const int G = h_q / h_kv;
+  if (G != 1 && G != 2 && G != 4)
+    return fail(FATHOM_ERR_UNSUPPORTED, "query heads per KV head G=%d: need 1, 2 or 4", G);
+  REQUIRE(n >= 0 && n < ((int64_t)1 << 31), "n=%lld out of range [0, 2^31)", (long long)n);
+  REQUIRE(k >= 1 && k <= FATHOM_MAX_K, "k=%d out of range [1, %d]", k, FATHOM_MAX_K);
+  REQUIRE(q_dtype == FATHOM_F32 || q_dtype == FATHOM_BF16, "q_dtype=%d unknown", q_dtype);
+  REQUIRE(planes_location == FATHOM_PLANES_DEVICE || planes_location == FATHOM_PLANES_HOST_MAPPED,
+          "planes_location=%d unknown", planes_location);
+  return FATHOM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *fathom_last_error(void) { return g_err; }
+
+void fathom_profile_scan_kernel(void *begin, void *end) {
+  g_prof_begin = (cudaEvent_t)begin;
+  g_prof_end = (cudaEvent_t)end;
+}
+
+int64_t fathom_plane_words(int64_t n) { return n < 0 ? 0 : plane_words(n); }
+
+size_t fathom_planes_bytes(int64_t n, int d, int h_kv) {
+  if (n < 0 || d < 0 || h_kv < 0) return 0;
+  return (size_t)h_kv * d * 4 * plane_words(n) * 4;
+}
+
+fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int d, int h_kv, uint32_t *planes,
+                                 void *stream) {
+  fathom_status st = check_shape(d, h_kv, h_kv);
+  if (st != FATHOM_OK) return st;
+  REQUIRE(n >= 0 && n < ((int64_t)1 << 31), "n=%lld out of range [0, 2^31)", (long long)n);
+  if (n == 0) return ok();
+  REQUIRE_DEV(codes, "codes");
+  REQUIRE_DEV(planes, "planes");
+  REQUIRE(aligned(codes, 16) && aligned(planes, 16), "codes and planes must be 16-byte aligned");
+  cudaError_t e = launch_pack(codes, n, d, h_kv, planes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return ok();
+}
+
+fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, const float *sigma, int h_q,
+                              int h_kv, int d, int budget_bits, uint8_t *alloc, void *stream) {
+  fathom_status st = check_shape(d, h_q, h_kv);
+  if (st != FATHOM_OK) return st;
+  REQUIRE(q_dtype == FATHOM_F32 || q_dtype == FATHOM_BF16, "q_dtype=%d unknown", (int)q_dtype);
+  REQUIRE(budget_bits >= 0 && budget_bits <= 4 * d, "budget_bits=%d out of range [0, 4d=%d]",
+          budget_bits, 4 * d);
+  REQUIRE_DEV(q, "q");
+  REQUIRE_DEV(sigma, "sigma");
+  REQUIRE_DEV(alloc, "alloc");
+  cudaError_t e = launch_allocate(q, q_dtype == FATHOM_BF16, sigma, h_q, h_kv, d, budget_bits,
+                                  alloc, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "allocate launch");
+  return ok();
+}
+
+static fathom_status check_scan_args(const fathom_scan_args *a) {
+  REQUIRE(a != nullptr, "args is NULL");
+  fathom_status st = check_scan_common(a->n, a->d, a->h_q, a->h_kv, a->k, a->q_dtype,
+                                       a->planes_location);
+  if (st != FATHOM_OK) return st;
+  REQUIRE_DEV(a->qmin, "qmin");
+  REQUIRE_DEV(a->qscale, "qscale");
+  REQUIRE_DEV(a->q, "q");
+  REQUIRE_DEV(a->alloc, "alloc");
+  REQUIRE_DEV(a->out_idx, "out_idx");
+  REQUIRE_DEV(a->out_score, "out_score");
+  if (a->debug_scores) REQUIRE_DEV(a->debug_scores, "debug_scores");
+  if (a->n > 0) {
+    REQUIRE(a->planes != nullptr, "planes is NULL");
+    const PtrKind kind = ptr_kind(a->planes);
+    if (a->planes_location == FATHOM_PLANES_DEVICE)
+      REQUIRE(kind == kPtrDevice, "planes is not a device pointer (planes_location=DEVICE)");
+    else
+      REQUIRE(kind == kPtrHostMapped,
+              "planes is not pinned, mapped host memory (planes_location=HOST_MAPPED)");
+    REQUIRE(aligned(a->planes, 16), "planes must be 16-byte aligned");
+  }
+  return FATHOM_OK;
+}
+
+size_t fathom_scan_topk_workspace_size(const fathom_scan_args *a) {
+  if (a == nullptr || check_scan_common(a->n, a->d, a->h_q, a->h_kv, a->k, a->q_dtype,
+                                        a->planes_location) != FATHOM_OK)
+    return 0;
+  return ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags).total;
+}
+
+fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_bytes, void *stream) {
+  fathom_status st = check_scan_args(a);
+  if (st != FATHOM_OK) return st;
+  const WsLayout L = ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags);
+  REQUIRE_DEV(ws, "workspace");
+  REQUIRE(aligned(ws, 256), "workspace must be 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(FATHOM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes,
+                L.total);
+  ScanParams p;
+  memset(&p, 0, sizeof(p));
+  p.sessions = nullptr;
+  p.one.planes = a->planes;
+  p.one.qmin = a->qmin;
+  p.one.qscale = a->qscale;
+  p.one.q = a->q;
+  p.one.alloc = a->alloc;
+  p.one.n = a->n;
+  p.one.out_idx = a->out_idx;
+  p.one.out_score = a->out_score;
+  p.batched = 0;
+  p.S = 1;
+  p.d = a->d;
+  p.h_q = a->h_q;
+  p.h_kv = a->h_kv;
+  p.G = a->h_q / a->h_kv;
+  p.k = a->k;
+  p.q_bf16 = a->q_dtype == FATHOM_BF16;
+  p.flags = a->flags;
+  p.debug_scores = a->debug_scores;
+  fill_ws(p, L, ws);
+  p.prof_begin = g_prof_begin;
+  p.prof_end = g_prof_end;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  e = launch_scan_pipeline(p, sampling_on(a->n, L.sample_rank, a->flags), s);
+  if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+  return ok();
+}
+
+static fathom_status check_batched_args(const fathom_batched_args *a) {
+  REQUIRE(a != nullptr, "args is NULL");
+  REQUIRE(a->num_sessions >= 1 && a->num_sessions <= 1024, "num_sessions=%d out of range [1, 1024]",
+          a->num_sessions);
+  fathom_status st = check_scan_common(a->n_max, a->d, a->h_q, a->h_kv, a->k, a->q_dtype,
+                                       a->planes_location);
+  if (st != FATHOM_OK) return st;
+  REQUIRE_DEV(a->sessions, "sessions");
+  return FATHOM_OK;
+}
+
+size_t fathom_scan_topk_batched_workspace_size(const fathom_batched_args *a) {
+  if (a == nullptr || a->num_sessions < 1 || a->num_sessions > 1024 ||
+      check_scan_common(a->n_max, a->d, a->h_q, a->h_kv, a->k, a->q_dtype, a->planes_location) !=
+          FATHOM_OK)
+    return 0;
+  return ws_layout(a->num_sessions, a->n_max, a->d, a->h_q, a->h_kv, a->k, a->flags).total;
+}
+
+fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, size_t ws_bytes,
+                                       void *stream) {
+  fathom_status st = check_batched_args(a);
+  if (st != FATHOM_OK) return st;
+  const WsLayout L = ws_layout(a->num_sessions, a->n_max, a->d, a->h_q, a->h_kv, a->k, a->flags);
+  REQUIRE_DEV(ws, "workspace");
+  REQUIRE(aligned(ws, 256), "workspace must be 256-byte aligned");
+  if (ws_bytes < L.total)
+    return fail(FATHOM_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes,
+                L.total);
+  ScanParams p;
+  memset(&p, 0, sizeof(p));
+  p.sessions = a->sessions;
+  p.batched = 1;
+  p.S = a->num_sessions;
+  p.d = a->d;
+  p.h_q = a->h_q;
+  p.h_kv = a->h_kv;
+  p.G = a->h_q / a->h_kv;
+  p.k = a->k;
+  p.q_bf16 = a->q_dtype == FATHOM_BF16;
+  p.flags = a->flags;
+  p.debug_scores = nullptr;
+  fill_ws(p, L, ws);
+  p.prof_begin = g_prof_begin;
+  p.prof_end = g_prof_end;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  e = launch_scan_pipeline(p, L.m_max > 0, s);
+  if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+  return ok();
+}
+
+fathom_status fathom_scan_read_report(const void *ws, fathom_scan_report *report, void *stream) {
+  REQUIRE(report != nullptr, "report is NULL");
+  REQUIRE_DEV(ws, "workspace");
+  WsStatus hs;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(&hs, ws, sizeof(hs), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "report copy");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "report sync");
+  report->fallback_heads = hs.fallback_heads;
+  report->device_faults = hs.device_faults;
+  report->max_candidates = hs.max_candidates;
+  report->union_planes = hs.union_planes;
+  if (hs.device_faults) return fail(FATHOM_ERR_DEVICE_CHECK, "device checks recorded %u faults",
+                                    hs.device_faults);
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,890 @@
+// The Fathom query-adaptive key scan and its top-k, for sm_100a.
+//
+// What is computed ("Fathom Makes KV-Cache Scans Query-Adaptive for
+// Long-Context Decoding", method paragraphs 1-3; arXiv 2609.17652
+// abstract): for every query head h and key i,
+//   s_h(i) = sum_c q_c * deq_{t_c}(v_{t_c}(i, c)),
+// v_t the value of the first t bit planes of channel c and deq_t the centre
+// of the t-bit cell, followed by the k largest s_h per head.
+//
+// How (B200 design, not the pages' A100 one):
+//  * plan_kernel, one block per (session, KV head): the union prefix
+//    t*_c = max over the G query heads of t_c, and per channel the distinct
+//    prefix lengths ("features") with the heads that use each.  Per head the
+//    score is rewritten as
+//        s_h(i) = K_h + sum_{c: t_c > 0} W_c * x_{t_c}(i, c),
+//        W_c = 16 q_c s_c,  x_t = 1 + y_t / 16,
+//    y_t the code's top t bits left-aligned in 4 bits (y_t = 2^(4-t) v_t),
+//    K_h = sum_c q_c (m_c + s_c (2^(4-t_c) - 1) / 2) - sum_{c: t_c > 0} W_c.
+//    x_t is built exactly as an fp32 bit pattern (exponent 0, y_t in the
+//    top four fraction bits), so one byte permute and one FMA per
+//    (token, channel, feature) replace t_c conditional adds per head.
+//  * scan_kernel, persistent blocks of 128 threads over 4096-token tiles:
+//    the union plane rows of a tile are staged into shared memory with
+//    16-byte cp.async copies, three stages in flight; each thread owns one
+//    plane word (32 tokens) and keeps its 32 x G scores in registers
+//    (packed fp32x2 FMAs); it writes the tokens whose score clears the
+//    head's sampled threshold as (score, index) candidates.
+//  * A sample pass of the same kernel scores one 256-token sector in 64
+//    and threshold_kernel takes the r-th largest sampled score per head as
+//    that threshold (expected ~2k candidates per head, no dense score write).
+//  * merge_kernel, one block per head: exact radix select of the k-th
+//    largest (score, -index) composite among the candidates, then a sort.
+//    When a threshold turns out invalid (fewer than k candidates, or more
+//    than the buffer holds) the block recomputes that head exactly with a
+//    streaming single-block scan.
+#include <float.h>
+
+#include "fathom_internal.cuh"
+
+namespace fathom {
+
+// ------------------------------------------------------------ utilities --
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t rotr(uint32_t x, int s) { return __funnelshift_r(x, x, s); }
+
+// Block-wide inclusive scan of one int per thread (blockDim.x <= 1024).
+__device__ int block_inclusive_scan(int v, int *s_tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  if (lane == 31) s_tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int x = lane < nw ? s_tmp[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int o = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += o;
+    }
+    if (lane < nw) s_tmp[lane] = x;
+  }
+  __syncthreads();
+  if (warp > 0) v += s_tmp[warp - 1];
+  __syncthreads();
+  return v;
+}
+
+// ------------------------------------------------------------ plan kernel --
+
+__global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
+  const int gid = blockIdx.x;
+  const int s = gid / p.h_kv;
+  const int g = gid - s * p.h_kv;
+  const fathom_session &se = session_of(p, s);
+  const int d = p.d, G = p.G;
+  const int c = threadIdx.x;
+  const PlanLayout L = plan_layout(d);
+  unsigned char *plan = p.plans + (size_t)gid * L.bytes;
+  PlanHeader *hdr = reinterpret_cast<PlanHeader *>(plan);
+  uint16_t *stage_begin = reinterpret_cast<uint16_t *>(plan + L.off_stage_begin);
+  uint8_t *stage_nrows = plan + L.off_stage_nrows;
+  uint16_t *stage_rows = reinterpret_cast<uint16_t *>(plan + L.off_stage_rows);
+  uint32_t *info = reinterpret_cast<uint32_t *>(plan + L.off_info);
+  uint32_t *feat = reinterpret_cast<uint32_t *>(plan + L.off_feat);
+  float4 *wts = reinterpret_cast<float4 *>(plan + L.off_w);
+
+  __shared__ int s_tmp[32];
+  __shared__ double s_k[4][8];
+  __shared__ int s_stage_base[64];
+  __shared__ int s_total[2];
+
+  int tstar = 0, nfeat = 0;
+  uint32_t fbits = 0;
+  float W[4] = {0.f, 0.f, 0.f, 0.f};
+  double kpart[4] = {0.0, 0.0, 0.0, 0.0};
+  if (c < d) {
+    const float m = se.qmin[(int64_t)g * d + c];
+    const float sc = se.qscale[(int64_t)g * d + c];
+    int t[4] = {0, 0, 0, 0};
+    for (int hh = 0; hh < G; ++hh) {
+      const int64_t hq = (int64_t)(g * G + hh) * d + c;
+      t[hh] = se.alloc[hq];
+      const float qv = load_q(se.q, p.q_bf16, hq);
+      tstar = max(tstar, t[hh]);
+      W[hh] = t[hh] > 0 ? (qv * sc) * 16.0f : 0.0f;
+      const double cell = (double)(1 << (4 - t[hh]));
+      kpart[hh] = (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5)) - (double)W[hh];
+    }
+    for (int tf = 1; tf <= 4; ++tf) {
+      uint32_t mask = 0;
+      for (int hh = 0; hh < G; ++hh) mask |= (t[hh] == tf ? 1u : 0u) << hh;
+      if (mask) {
+        fbits |= ((uint32_t)tf | (mask << 3)) << (8 * nfeat);
+        ++nfeat;
+      }
+    }
+  }
+  // per-head constants
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int hh = 0; hh < G; ++hh) {
+    double v = kpart[hh];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if (lane == 0) s_k[hh][warp] = v;
+  }
+  // entry index and first plane of every channel with t* > 0
+  const int packed = (tstar > 0 ? 1 : 0) | (tstar << 12);
+  const int incl = block_inclusive_scan(packed, s_tmp);
+  const int e = (incl & 0xfff) - 1;            // entry index if tstar > 0
+  const int p_incl = incl >> 12;               // planes up to and including c
+  const int p_excl = p_incl - tstar;
+  if (threadIdx.x == blockDim.x - 1) {
+    s_total[0] = incl & 0xfff;  // entries
+    s_total[1] = incl >> 12;    // union planes
+  }
+  const int stage = tstar > 0 ? (p_incl - 1) / kStageSpan : -1;
+  const int prev_stage = tstar > 0 ? (p_excl > 0 ? (p_excl - 1) / kStageSpan : -1) : -1;
+  // the first entry of a stage is the one whose previous plane lies in an earlier stage
+  if (tstar > 0 && (p_excl == 0 || prev_stage != stage)) {
+    s_stage_base[stage] = p_excl;
+    stage_begin[stage] = (uint16_t)e;
+  }
+  __syncthreads();
+  const int nent = s_total[0];
+  const int nplanes = s_total[1];
+  const int nstage = nplanes > 0 ? (nplanes - 1) / kStageSpan + 1 : 1;
+  if (tstar > 0) {
+    const int slot0 = p_excl - s_stage_base[stage];
+    info[e] = (uint32_t)c | ((uint32_t)tstar << 8) | ((uint32_t)slot0 << 11) |
+              ((uint32_t)nfeat << 16);
+    feat[e] = fbits;
+    wts[e] = make_float4(W[0], W[1], W[2], W[3]);
+    for (int j = 0; j < tstar; ++j)
+      stage_rows[stage * kStageRows + slot0 + j] = (uint16_t)(c * 4 + j);
+  }
+  if (threadIdx.x < nstage) {
+    const int st = threadIdx.x;
+    const int base = nplanes > 0 ? s_stage_base[st] : 0;
+    const int end = (st + 1 < nstage) ? s_stage_base[st + 1] : nplanes;
+    stage_nrows[st] = (uint8_t)(end - base);
+  }
+  if (threadIdx.x == 0) {
+    if (nplanes == 0) stage_begin[0] = 0;
+    stage_begin[nstage] = (uint16_t)nent;
+    hdr->nent = nent;
+    hdr->nstage = nstage;
+    hdr->union_planes = nplanes;
+    const int nw = (blockDim.x + 31) >> 5;
+    for (int hh = 0; hh < 4; ++hh) {
+      double sum = 0.0;
+      if (hh < G)
+        for (int w = 0; w < nw; ++w) sum += s_k[hh][w];
+      hdr->K[hh] = (float)sum;
+      hdr->tau[hh] = -INFINITY;
+    }
+    atomicAdd(&p.status->union_planes, (uint32_t)nplanes);
+  }
+}
+
+// ------------------------------------------------------------ scan kernel --
+
+struct TileLoc {
+  int s, g, ti;     // session, KV head, tile within (session, KV head)
+  int64_t n, W;     // session keys and plane words
+  const uint32_t *planes;
+};
+
+struct Item {
+  int t;      // tile index in the launch's tile space (-1 = none)
+  int st;     // stage within the tile
+  int slot;   // plan slot in shared memory
+  int nst;    // stages of this tile
+};
+
+template <int MODE>
+__device__ __forceinline__ int64_t tiles_per_group(int64_t n, const ScanParams &p) {
+  return MODE == kModeSample ? sample_tiles(n, p.sample_rank, p.flags) : filter_tiles(n);
+}
+
+template <int MODE>
+__device__ __forceinline__ TileLoc locate(const ScanParams &p, const int *s_tprefix, int t) {
+  int lo = 0, hi = p.S;  // find s with prefix[s] <= t < prefix[s+1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_tprefix[mid] <= t) lo = mid; else hi = mid;
+  }
+  TileLoc L;
+  L.s = lo;
+  const fathom_session &se = session_of(p, lo);
+  L.n = se.n;
+  L.W = plane_words(L.n);
+  L.planes = se.planes;
+  const int per = (int)tiles_per_group<MODE>(L.n, p);
+  const int r = t - s_tprefix[lo];
+  L.g = r / per;
+  L.ti = r - L.g * per;
+  return L;
+}
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const PlanLayout PL = plan_layout(p.d);
+  uint32_t *sbuf = reinterpret_cast<uint32_t *>(smem);
+  unsigned char *splans = smem + kNumBuf * kStageBytes;
+  int *s_tprefix = reinterpret_cast<int *>(splans + kNumPlanSlots * PL.bytes);
+  __shared__ int s_tmp[32];
+  __shared__ int s_slot_gid[kNumPlanSlots];
+
+  // ---- tile space: every (session, KV head) contributes its tiles --------
+  for (int base = 0; base < p.S; base += kScanThreads) {
+    const int s = base + tid;
+    int v = 0;
+    if (s < p.S) v = (int)(tiles_per_group<MODE>(session_of(p, s).n, p) * p.h_kv);
+    const int carry = base > 0 ? s_tprefix[base] : 0;
+    __syncthreads();
+    const int incl = block_inclusive_scan(v, s_tmp);
+    if (s < p.S) s_tprefix[s + 1] = carry + incl;
+    if (base == 0 && tid == 0) s_tprefix[0] = 0;
+    __syncthreads();
+  }
+  const int total = s_tprefix[p.S];
+  const int t_begin = (int)(((int64_t)blockIdx.x * total) / gridDim.x);
+  const int t_end = (int)(((int64_t)(blockIdx.x + 1) * total) / gridDim.x);
+  if (t_begin >= t_end) return;
+  if (tid < kNumPlanSlots) s_slot_gid[tid] = -1;
+  __syncthreads();
+
+  // ---- plan slots ---------------------------------------------------------
+  // Loads the plan of (session s, KV head g) into a slot not used by the two
+  // items ahead of it, unless it is resident already.  Called uniformly.
+  auto ensure_plan = [&](int gid, int busy0, int busy1) -> int {
+    int slot = -1;
+#pragma unroll
+    for (int i = 0; i < kNumPlanSlots; ++i)
+      if (s_slot_gid[i] == gid) slot = i;
+    if (slot >= 0) return slot;
+#pragma unroll
+    for (int i = kNumPlanSlots - 1; i >= 0; --i)
+      if (i != busy0 && i != busy1) slot = i;
+    __syncthreads();
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.plans + (size_t)gid * PL.bytes);
+    uint4 *dst = reinterpret_cast<uint4 *>(splans + slot * PL.bytes);
+    for (int i = tid; i < PL.bytes / 16; i += kScanThreads) dst[i] = src[i];
+    __syncthreads();
+    if (tid < G) {
+      PlanHeader *hdr = reinterpret_cast<PlanHeader *>(splans + slot * PL.bytes);
+      float tau = -INFINITY;
+      if (MODE == kModeFilter) {
+        const int s = gid / p.h_kv, g = gid - s * p.h_kv;
+        const uint32_t key = p.tau[(int64_t)s * p.h_q + g * G + tid];
+        tau = key == 0u ? -INFINITY : key_float(key);
+      }
+      hdr->tau[tid] = tau;
+    }
+    if (tid == 0) s_slot_gid[slot] = gid;
+    __syncthreads();
+    return slot;
+  };
+
+  auto first_item = [&](int t, int busy0, int busy1) -> Item {
+    Item it;
+    it.t = t;
+    it.st = 0;
+    if (t >= t_end) {
+      it.t = -1;
+      it.slot = -1;
+      it.nst = 0;
+      return it;
+    }
+    const TileLoc L = locate<MODE>(p, s_tprefix, t);
+    it.slot = ensure_plan(L.s * p.h_kv + L.g, busy0, busy1);
+    it.nst = reinterpret_cast<const PlanHeader *>(splans + it.slot * PL.bytes)->nstage;
+    return it;
+  };
+  auto next_item = [&](const Item &a, int busy0, int busy1) -> Item {
+    if (a.t < 0) return a;
+    if (a.st + 1 < a.nst) {
+      Item b = a;
+      b.st += 1;
+      return b;
+    }
+    return first_item(a.t + 1, busy0, busy1);
+  };
+
+  // ---- staged copies of one item's plane rows -----------------------------
+  auto issue = [&](const Item &it, int buf) {
+    if (it.t < 0) return;
+    const TileLoc L = locate<MODE>(p, s_tprefix, it.t);
+    const unsigned char *plan = splans + it.slot * PL.bytes;
+    const int nrows = plan[PL.off_stage_nrows + it.st];
+    const uint16_t *rows = reinterpret_cast<const uint16_t *>(plan + PL.off_stage_rows) +
+                           it.st * kStageRows;
+    uint32_t *dst_base = sbuf + buf * (kStageBytes / 4);
+    const uint32_t *gbase = L.planes + (int64_t)L.g * p.d * 4 * L.W;
+    for (int id = tid; id < nrows * 32; id += kScanThreads) {
+      const int slot = id >> 5, q = id & 31;
+      const uint32_t *row = gbase + (int64_t)rows[slot] * L.W;
+      int64_t word;
+      bool ok;
+      if (MODE == kModeSample) {
+        const int64_t sj = (int64_t)L.ti * kSampleSectorsPerTile + (q >> 1);
+        word = sj * kSampleStride * kSectorWords + (q & 1) * 4;
+        ok = sj < sampled_sectors(L.n) && word < L.W;
+      } else {
+        word = (int64_t)L.ti * kTileWords + q * 4;
+        ok = word < L.W;
+      }
+      cp_async16(dst_base + slot * kTileWords + q * 4, ok ? (const void *)(row + word) : (const void *)row,
+                 ok ? 16u : 0u);
+    }
+  };
+
+  // ---- per-thread scores: 32 tokens x G heads -----------------------------
+  // acc[h][r][p]: .x is byte 2p, .y byte 2p+1 of build register r, i.e.
+  // tokens 32 w + 8 (2p) + r and 32 w + 8 (2p + 1) + r of this thread's word w.
+  float2 acc[G][8][2];
+
+  auto compute = [&](const Item &it, int buf) {
+    const unsigned char *plan = splans + it.slot * PL.bytes;
+    const PlanHeader *hdr = reinterpret_cast<const PlanHeader *>(plan);
+    if (it.st == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float k0 = hdr->K[h];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          acc[h][r][0] = make_float2(k0, k0);
+          acc[h][r][1] = make_float2(k0, k0);
+        }
+      }
+    }
+    const uint16_t *stage_begin = reinterpret_cast<const uint16_t *>(plan + PL.off_stage_begin);
+    const uint32_t *info = reinterpret_cast<const uint32_t *>(plan + PL.off_info);
+    const uint32_t *feats = reinterpret_cast<const uint32_t *>(plan + PL.off_feat);
+    const float4 *wts = reinterpret_cast<const float4 *>(plan + PL.off_w);
+    const uint32_t *sb = sbuf + buf * (kStageBytes / 4) + tid;
+    const int e0 = stage_begin[it.st], e1 = stage_begin[it.st + 1];
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t inf = info[e];
+      const int tstar = (inf >> 8) & 7;
+      const int slot0 = (inf >> 11) & 31;
+      const int nfeat = (inf >> 16) & 7;
+      const uint32_t *src = sb + slot0 * kTileWords;
+      // Build 8 registers of 4 tokens each: byte kk of R[r] is
+      // 0x80 | y << 3 for token 8 kk + r of the word, y = union prefix code
+      // left-aligned in 4 bits (plane j lands on bit 6 - j).
+      uint32_t R[8];
+      const uint32_t p0 = src[0];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) R[r] = (rotr(p0, (r - 6) & 31) & 0x40404040u) | 0x80808080u;
+      if (tstar > 1) {
+        const uint32_t p1 = src[kTileWords];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) R[r] |= rotr(p1, (r - 5) & 31) & 0x20202020u;
+        if (tstar > 2) {
+          const uint32_t p2 = src[2 * kTileWords];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) R[r] |= rotr(p2, (r - 4) & 31) & 0x10101010u;
+          if (tstar > 3) {
+            const uint32_t p3 = src[3 * kTileWords];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) R[r] |= rotr(p3, (r - 3) & 31) & 0x08080808u;
+          }
+        }
+      }
+      const float4 w4 = wts[e];
+      const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const uint32_t fb = feats[e];
+      for (int f = 0; f < nfeat; ++f) {
+        const uint32_t byte = (fb >> (8 * f)) & 0xffu;
+        const int tf = byte & 7;
+        const uint32_t mask = byte >> 3;
+        // keep the first tf planes: byte mask 0xff << (7 - tf)
+        const uint32_t keep = (0xffu << (7 - tf)) & 0xffu;
+        const uint32_t km = keep * 0x01010101u;
+        uint32_t Rf[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) Rf[r] = R[r] & km;
+        float2 wpair[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) wpair[h] = make_float2(wv[h], wv[h]);
+        // x = 1 + y/16 as fp32: [0x3f][byte][0][0]
+#define FATHOM_APPLY(MASKV)                                                            \
+  {                                                                                    \
+    _Pragma("unroll") for (int r = 0; r < 8; ++r) {                                    \
+      _Pragma("unroll") for (int pp = 0; pp < 2; ++pp) {                               \
+        const float x0 = __uint_as_float(__byte_perm(Rf[r], 0x3f000000u, 0x7054u | ((2 * pp) << 8)));     \
+        const float x1 = __uint_as_float(__byte_perm(Rf[r], 0x3f000000u, 0x7054u | ((2 * pp + 1) << 8))); \
+        const float2 xx = make_float2(x0, x1);                                         \
+        _Pragma("unroll") for (int h = 0; h < G; ++h) {                                \
+          if ((MASKV) & (1u << h)) acc[h][r][pp] = __ffma2_rn(xx, wpair[h], acc[h][r][pp]); \
+        }                                                                              \
+      }                                                                                \
+    }                                                                                  \
+  }
+        switch (mask) {
+          case 1: FATHOM_APPLY(1u) break;
+          case 2: if (G > 1) FATHOM_APPLY(2u) break;
+          case 3: if (G > 1) FATHOM_APPLY(3u) break;
+          case 4: if (G > 2) FATHOM_APPLY(4u) break;
+          case 5: if (G > 2) FATHOM_APPLY(5u) break;
+          case 6: if (G > 2) FATHOM_APPLY(6u) break;
+          case 7: if (G > 2) FATHOM_APPLY(7u) break;
+          case 8: if (G > 3) FATHOM_APPLY(8u) break;
+          case 9: if (G > 3) FATHOM_APPLY(9u) break;
+          case 10: if (G > 3) FATHOM_APPLY(10u) break;
+          case 11: if (G > 3) FATHOM_APPLY(11u) break;
+          case 12: if (G > 3) FATHOM_APPLY(12u) break;
+          case 13: if (G > 3) FATHOM_APPLY(13u) break;
+          case 14: if (G > 3) FATHOM_APPLY(14u) break;
+          case 15: if (G > 3) FATHOM_APPLY(15u) break;
+          default: break;
+        }
+#undef FATHOM_APPLY
+      }
+    }
+  };
+
+  // ---- results of a finished tile -------------------------------------------
+  auto emit = [&](const Item &it) {
+    const TileLoc L = locate<MODE>(p, s_tprefix, it.t);
+    const PlanHeader *hdr = reinterpret_cast<const PlanHeader *>(splans + it.slot * PL.bytes);
+    const int64_t head0 = (int64_t)L.s * p.h_q + L.g * G;
+    if (MODE == kModeSample) {
+      const int64_t sj = (int64_t)L.ti * kSampleSectorsPerTile + (tid >> 3);
+      if (sj >= sampled_sectors(L.n)) return;
+      const int64_t tok0 = (sj * kSampleStride * kSectorWords + (tid & 7)) * 32;
+      const int64_t slot0 = sj * 256 + (tid & 7) * 32;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        uint32_t *dst = p.sample + (head0 + h) * p.m_max + slot0;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int b = 8 * kk + r;
+            const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
+            dst[b] = (tok0 + b < L.n) ? float_key(sc) : 0u;
+          }
+      }
+      return;
+    }
+    const int64_t tok0 = ((int64_t)L.ti * kTileWords + tid) * 32;
+    if (p.debug_scores) {
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int64_t tok = tok0 + 8 * kk + r;
+            const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
+            if (tok < L.n) p.debug_scores[(head0 + h) * L.n + tok] = sc;
+          }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float tau = hdr->tau[h];
+      uint32_t m = 0;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int b = 8 * kk + r;
+          const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
+          m |= ((tok0 + b < L.n) && (sc >= tau) ? 1u : 0u) << b;
+        }
+      const int cnt = __popc(m);
+      if (__any_sync(0xffffffffu, cnt != 0)) {
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        unsigned base = 0;
+        if (lane == 31) base = atomicAdd(&p.counts[head0 + h], (unsigned)incl);
+        base = __shfl_sync(0xffffffffu, base, 31);
+        if (cnt) {
+          int64_t pos = (int64_t)base + (incl - cnt);
+          unsigned long long *dst = p.cand + (head0 + h) * p.cap;
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const int b = 8 * kk + r;
+              if ((m >> b) & 1u) {
+                const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
+                if (pos < p.cap) dst[pos] = composite(sc, (uint32_t)(tok0 + b));
+                ++pos;
+              }
+            }
+        }
+      }
+    }
+  };
+
+  // ---- software pipeline over (tile, stage) items ---------------------------
+  Item cur = first_item(t_begin, -1, -1);
+  Item nxt = next_item(cur, cur.slot, -1);
+  issue(cur, 0);
+  cp_async_commit();
+  issue(nxt, 1);
+  cp_async_commit();
+  Item iss = next_item(nxt, cur.slot, nxt.slot);
+  int it = 0;
+  while (true) {
+    issue(iss, (it + 2) % kNumBuf);
+    cp_async_commit();
+    cp_async_wait<2>();
+    __syncthreads();
+    compute(cur, it % kNumBuf);
+    if (cur.st == cur.nst - 1) emit(cur);
+    __syncthreads();
+    if (nxt.t < 0) break;
+    cur = nxt;
+    nxt = iss;
+    iss = next_item(iss, cur.slot, nxt.slot);
+    ++it;
+  }
+  cp_async_wait<0>();
+}
+
+// ------------------------------------------------------- threshold kernel --
+
+// Warp 0 finds the digit bin holding the want-th largest among 256 bins
+// (counted from the top); returns (digit, count above it).
+__device__ __forceinline__ void find_bin_from_top(const unsigned *hist, unsigned want, int *s_digit,
+                                                  unsigned *s_above) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    // lane l owns bins 255 - 8l ... 248 - 8l (top first)
+    unsigned local[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      local[i] = hist[255 - 8 * lane - i];
+      sum += local[i];
+    }
+    unsigned incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    const unsigned excl = incl - sum;
+    if (excl < want && want <= incl) {
+      unsigned run = excl;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (run < want && want <= run + local[i]) {
+          *s_digit = 255 - 8 * lane - i;
+          *s_above = run;
+        }
+        run += local[i];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) threshold_kernel(ScanParams p) {
+  const int64_t h = blockIdx.x;
+  const int s = (int)(h / p.h_q);
+  const int64_t n = session_of(p, s).n;
+  __shared__ unsigned hist[256];
+  __shared__ int s_digit;
+  __shared__ unsigned s_above;
+  if (!sampling_on(n, p.sample_rank, p.flags)) {
+    if (threadIdx.x == 0) p.tau[h] = 0u;
+    return;
+  }
+  const int64_t m = sampled_sectors(n) * 256;
+  const uint32_t *keys = p.sample + h * p.m_max;
+  uint32_t prefix = 0, pmask = 0;
+  unsigned want = (unsigned)p.sample_rank;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    hist[threadIdx.x] = 0;
+    if (threadIdx.x == 0) s_digit = -1;
+    __syncthreads();
+    for (int64_t i = threadIdx.x; i < m; i += blockDim.x) {
+      const uint32_t k = keys[i];
+      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    find_bin_from_top(hist, want, &s_digit, &s_above);
+    __syncthreads();
+    if (s_digit < 0) {  // fewer than r sampled keys: keep everything
+      if (threadIdx.x == 0) p.tau[h] = 0u;
+      return;
+    }
+    prefix |= (uint32_t)s_digit << shift;
+    pmask |= 255u << shift;
+    want -= s_above;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.tau[h] = prefix;
+}
+
+// ---------------------------------------------------------- merge kernel --
+
+// k-th largest (1-based) of cnt distinct 64-bit composites, k <= cnt.
+__device__ unsigned long long block_kth(const unsigned long long *a, int64_t cnt, unsigned k,
+                                        unsigned *hist, int *s_digit, unsigned *s_above) {
+  unsigned long long prefix = 0ull, pmask = 0ull;
+  unsigned want = k;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    if (threadIdx.x == 0) *s_digit = -1;
+    __syncthreads();
+    for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+      const unsigned long long v = a[i];
+      if ((v & pmask) == prefix) atomicAdd(&hist[(unsigned)(v >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    find_bin_from_top(hist, want, s_digit, s_above);
+    __syncthreads();
+    prefix |= (unsigned long long)(*s_digit) << shift;
+    pmask |= 255ull << shift;
+    want -= *s_above;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+// Exact single-block answer for one head: stream all n keys, score each from
+// its allocated prefixes (fp32), keep a candidate buffer above a running
+// k-th best, compact it when it fills.  Used when the sampled threshold
+// fails.  Returns the number of buffered candidates (= min(k, n)).
+__device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned long long *buf,
+                                 unsigned long long *s_sort, unsigned *hist, int *s_digit,
+                                 unsigned *s_above) {
+  const fathom_session &se = session_of(p, s);
+  const int d = p.d;
+  const int g = hl / p.G;
+  const int64_t n = se.n;
+  const int64_t W = plane_words(n);
+  __shared__ float s_qs[FATHOM_MAX_D];
+  __shared__ uint8_t s_t[FATHOM_MAX_D];
+  __shared__ double s_kc[32];
+  __shared__ unsigned long long s_nbuf;
+  double kc = 0.0;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const int t = se.alloc[(int64_t)hl * d + c];
+    const float qv = load_q(se.q, p.q_bf16, (int64_t)hl * d + c);
+    const float m = se.qmin[(int64_t)g * d + c], sc = se.qscale[(int64_t)g * d + c];
+    s_t[c] = (uint8_t)t;
+    s_qs[c] = qv * sc;
+    const double cell = (double)(1 << (4 - t));
+    kc += (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) kc += __shfl_xor_sync(0xffffffffu, kc, off);
+  if ((threadIdx.x & 31) == 0) s_kc[threadIdx.x >> 5] = kc;
+  if (threadIdx.x == 0) s_nbuf = 0;
+  __syncthreads();
+  double ksum = 0.0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) ksum += s_kc[w];
+  const float K = (float)ksum;
+  const uint32_t *gp = se.planes + (int64_t)g * d * 4 * W;
+  unsigned long long theta = 0ull;
+  const unsigned k = (unsigned)p.k;
+  for (int64_t base = 0; base < n; base += blockDim.x) {
+    const int64_t i = base + threadIdx.x;
+    if (i < n) {
+      float sc = K;
+      for (int c = 0; c < d; ++c) {
+        const int t = s_t[c];
+        if (t == 0) continue;
+        uint32_t y = 0;
+        for (int j = 0; j < t; ++j)
+          y |= ((gp[((int64_t)c * 4 + j) * W + (i >> 5)] >> (i & 31)) & 1u) << (3 - j);
+        sc = fmaf(s_qs[c], (float)y, sc);
+      }
+      const unsigned long long v = composite(sc, (uint32_t)i);
+      if (v > theta) buf[atomicAdd(&s_nbuf, 1ull)] = v;
+    }
+    __syncthreads();
+    const int64_t nb = (int64_t)s_nbuf;
+    if (nb > p.cap - (int64_t)blockDim.x) {
+      theta = block_kth(buf, nb, k, hist, s_digit, s_above);
+      __shared__ unsigned s_fill;
+      if (threadIdx.x == 0) s_fill = 0;
+      __syncthreads();
+      for (int64_t j = threadIdx.x; j < nb; j += blockDim.x)
+        if (buf[j] >= theta) {
+          const unsigned at = atomicAdd(&s_fill, 1u);
+          if (at < k) s_sort[at] = buf[j];
+        }
+      __syncthreads();
+      for (int j = threadIdx.x; j < (int)k; j += blockDim.x) buf[j] = s_sort[j];
+      if (threadIdx.x == 0) s_nbuf = k;
+      __syncthreads();
+      // the k kept are the best so far; a later key matters only above the
+      // k-th of them, which is theta
+    }
+  }
+  __syncthreads();
+  return (int64_t)s_nbuf;
+}
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int kpow2) {
+  extern __shared__ unsigned long long s_sort[];  // [kpow2]
+  __shared__ unsigned hist[256];
+  __shared__ int s_digit;
+  __shared__ unsigned s_above;
+  __shared__ unsigned s_fill;
+  const int64_t h = blockIdx.x;
+  const int s = (int)(h / p.h_q);
+  const int hl = (int)(h - (int64_t)s * p.h_q);
+  const fathom_session &se = session_of(p, s);
+  const int64_t n = se.n;
+  const int k = p.k;
+  unsigned long long *buf = p.cand + h * p.cap;
+  int64_t cnt = p.counts[h];
+  const uint32_t tauk = p.tau[h];
+  const int64_t need = n < k ? n : k;
+  const bool ok = cnt <= p.cap && (tauk == 0u || cnt >= need) && !(p.flags & FATHOM_FLAG_FORCE_FALLBACK);
+  if (!ok) {
+    cnt = fallback_head(p, s, hl, buf, s_sort, hist, &s_digit, &s_above);
+    if (threadIdx.x == 0) atomicAdd(&p.status->fallback_heads, 1u);
+  }
+  if (threadIdx.x == 0) atomicMax(&p.status->max_candidates, (unsigned)(cnt < 0xffffffffll ? cnt : 0xffffffffll));
+  const int take = (int)(cnt < k ? cnt : k);
+  unsigned long long bar = 0ull;
+  if (cnt > k) bar = block_kth(buf, cnt, (unsigned)k, hist, &s_digit, &s_above);
+  if (threadIdx.x == 0) s_fill = 0;
+  __syncthreads();
+  for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+    const unsigned long long v = buf[i];
+    if (v >= bar) {
+      const unsigned at = atomicAdd(&s_fill, 1u);
+      if (at < (unsigned)take) s_sort[at] = v;
+    }
+  }
+  for (int i = take + threadIdx.x; i < kpow2; i += blockDim.x) s_sort[i] = 0ull;
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= kpow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < kpow2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0;
+          const unsigned long long a = s_sort[i], b = s_sort[j];
+          if (desc ? (a < b) : (a > b)) {
+            s_sort[i] = b;
+            s_sort[j] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int r = threadIdx.x; r < k; r += blockDim.x) {
+    int32_t idx = -1;
+    float sc = -INFINITY;
+    if (r < take) {
+      const unsigned long long v = s_sort[r];
+      idx = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+      sc = key_float((uint32_t)(v >> 32));
+    }
+    se.out_idx[(int64_t)hl * k + r] = idx;
+    se.out_score[(int64_t)hl * k + r] = sc;
+  }
+}
+
+// ------------------------------------------------------------- launchers --
+
+static int g_num_sms = 0;
+
+static cudaError_t num_sms(int *out) {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  *out = g_num_sms;
+  return cudaSuccess;
+}
+
+int scan_smem_bytes(int d, int S) {
+  return kNumBuf * kStageBytes + kNumPlanSlots * plan_layout(d).bytes + 4 * (S + 1);
+}
+
+template <int G, int MODE>
+static cudaError_t launch_scan_gm(const ScanParams &p, cudaStream_t stream) {
+  const int smem = scan_smem_bytes(p.d, p.S);
+  cudaError_t e = cudaFuncSetAttribute(scan_kernel<G, MODE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, scan_kernel<G, MODE>, kScanThreads,
+                                                    smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  int sms = 0;
+  e = num_sms(&sms);
+  if (e != cudaSuccess) return e;
+  scan_kernel<G, MODE><<<sms * per_sm, kScanThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t launch_scan_m(const ScanParams &p, cudaStream_t stream) {
+  switch (p.G) {
+    case 1: return launch_scan_gm<1, MODE>(p, stream);
+    case 2: return launch_scan_gm<2, MODE>(p, stream);
+    case 4: return launch_scan_gm<4, MODE>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream) {
+  const int heads = p.S * p.h_q;
+  const int groups = p.S * p.h_kv;
+  plan_kernel<<<groups, 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (any_sampling) {
+    e = launch_scan_m<kModeSample>(p, stream);
+    if (e != cudaSuccess) return e;
+    threshold_kernel<<<heads, 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.prof_begin) {
+    e = cudaEventRecord(p.prof_begin, stream);
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_scan_m<kModeFilter>(p, stream);
+  if (e != cudaSuccess) return e;
+  if (p.prof_end) {
+    e = cudaEventRecord(p.prof_end, stream);
+    if (e != cudaSuccess) return e;
+  }
+  int kpow2 = 1;
+  while (kpow2 < p.k) kpow2 <<= 1;
+  const int msmem = kpow2 * 8;
+  e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
+  if (e != cudaSuccess) return e;
+  merge_kernel<<<heads, kMergeThreads, msmem, stream>>>(p, kpow2);
+  return cudaGetLastError();
+}
+
+}  // namespace fathom

@@ -1,0 +1,294 @@
+"""ctypes binding of libfathom.so (the C ABI in include/fathom.h).
+
+Argument marshalling only: every step of the scan runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  There
+is no CPU path: if the library is missing or the device is not a CUDA GPU,
+calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfathom.so")
+
+OK = 0
+ERR_INVALID_ARGUMENT = 1
+ERR_UNSUPPORTED = 2
+ERR_WORKSPACE_TOO_SMALL = 3
+ERR_CUDA = 4
+ERR_DEVICE_CHECK = 5
+
+F32 = 0
+BF16 = 1
+PLANES_DEVICE = 0
+PLANES_HOST_MAPPED = 1
+FLAG_NO_SAMPLING = 1
+FLAG_FORCE_FALLBACK = 2
+
+EXPORTED = [
+    "fathom_last_error", "fathom_plane_words", "fathom_planes_bytes", "fathom_pack_planes",
+    "fathom_allocate", "fathom_scan_topk_workspace_size", "fathom_scan_topk",
+    "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
+    "fathom_scan_read_report", "fathom_profile_scan_kernel",
+]
+
+
+class FathomError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("fathom status %d: %s" % (status, message))
+        self.status = status
+
+
+class ScanArgs(ctypes.Structure):
+    _fields_ = [
+        ("planes", ctypes.c_void_p), ("planes_location", ctypes.c_int),
+        ("qmin", ctypes.c_void_p), ("qscale", ctypes.c_void_p),
+        ("q", ctypes.c_void_p), ("q_dtype", ctypes.c_int),
+        ("alloc", ctypes.c_void_p), ("n", ctypes.c_int64),
+        ("d", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("k", ctypes.c_int),
+        ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
+        ("debug_scores", ctypes.c_void_p), ("flags", ctypes.c_uint32),
+    ]
+
+
+class Session(ctypes.Structure):
+    _fields_ = [
+        ("planes", ctypes.c_void_p), ("qmin", ctypes.c_void_p), ("qscale", ctypes.c_void_p),
+        ("q", ctypes.c_void_p), ("alloc", ctypes.c_void_p), ("n", ctypes.c_int64),
+        ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
+    ]
+
+
+class BatchedArgs(ctypes.Structure):
+    _fields_ = [
+        ("sessions", ctypes.c_void_p), ("num_sessions", ctypes.c_int), ("n_max", ctypes.c_int64),
+        ("d", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("k", ctypes.c_int),
+        ("q_dtype", ctypes.c_int), ("planes_location", ctypes.c_int), ("flags", ctypes.c_uint32),
+    ]
+
+
+class ScanReport(ctypes.Structure):
+    _fields_ = [("fallback_heads", ctypes.c_uint32), ("device_faults", ctypes.c_uint32),
+                ("max_candidates", ctypes.c_uint32), ("union_planes", ctypes.c_uint32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfathom.so; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libfathom.so is not built (python -m bit_plane_kv_scan_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.fathom_last_error.restype = ctypes.c_char_p
+        L.fathom_last_error.argtypes = []
+        L.fathom_plane_words.restype = i64
+        L.fathom_plane_words.argtypes = [i64]
+        L.fathom_planes_bytes.restype = sz
+        L.fathom_planes_bytes.argtypes = [i64, ci, ci]
+        L.fathom_pack_planes.restype = ci
+        L.fathom_pack_planes.argtypes = [vp, i64, ci, ci, vp, vp]
+        L.fathom_allocate.restype = ci
+        L.fathom_allocate.argtypes = [vp, ci, vp, ci, ci, ci, ci, vp, vp]
+        L.fathom_scan_topk_workspace_size.restype = sz
+        L.fathom_scan_topk_workspace_size.argtypes = [ctypes.POINTER(ScanArgs)]
+        L.fathom_scan_topk.restype = ci
+        L.fathom_scan_topk.argtypes = [ctypes.POINTER(ScanArgs), vp, sz, vp]
+        L.fathom_scan_topk_batched_workspace_size.restype = sz
+        L.fathom_scan_topk_batched_workspace_size.argtypes = [ctypes.POINTER(BatchedArgs)]
+        L.fathom_scan_topk_batched.restype = ci
+        L.fathom_scan_topk_batched.argtypes = [ctypes.POINTER(BatchedArgs), vp, sz, vp]
+        L.fathom_scan_read_report.restype = ci
+        L.fathom_scan_read_report.argtypes = [vp, ctypes.POINTER(ScanReport), vp]
+        L.fathom_profile_scan_kernel.restype = None
+        L.fathom_profile_scan_kernel.argtypes = [vp, vp]
+        _lib = L
+        return L
+
+
+def _check(status: int):
+    if status != OK:
+        raise FathomError(status, lib().fathom_last_error().decode())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(q: torch.Tensor) -> int:
+    if q.dtype == torch.bfloat16:
+        return BF16
+    if q.dtype == torch.float32:
+        return F32
+    raise TypeError("q must be bfloat16 or float32, got %s" % q.dtype)
+
+
+def plane_words(n: int) -> int:
+    return int(lib().fathom_plane_words(n))
+
+
+def pack_planes(codes: torch.Tensor, stream=None) -> torch.Tensor:
+    """[h_kv, n, d/2] uint8 codes (CUDA) -> [h_kv, d, 4, W] plane words (int32 storage)."""
+    if codes.dtype != torch.uint8 or codes.dim() != 3 or not codes.is_contiguous():
+        raise TypeError("codes must be a contiguous uint8 [h_kv, n, d/2] tensor")
+    h_kv, n, half = codes.shape
+    d = 2 * half
+    planes = torch.empty((h_kv, d, 4, plane_words(n)), dtype=torch.int32, device=codes.device)
+    _check(lib().fathom_pack_planes(_ptr(codes), n, d, h_kv, _ptr(planes), _stream(stream)))
+    return planes
+
+
+def allocate(q: torch.Tensor, sigma: torch.Tensor, budget: int, stream=None,
+             out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """q [h_q, d] (bf16/f32), sigma [h_kv, d] f32 -> bits per channel uint8 [h_q, d]."""
+    h_q, d = q.shape
+    h_kv = sigma.shape[0]
+    if out is None:
+        out = torch.empty((h_q, d), dtype=torch.uint8, device=q.device)
+    _check(lib().fathom_allocate(_ptr(q.contiguous()), _dtype_code(q), _ptr(sigma.contiguous()),
+                                 h_q, h_kv, d, int(budget), _ptr(out), _stream(stream)))
+    return out
+
+
+class Workspace:
+    """A reusable device workspace that grows to the largest request."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = torch.empty(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=self.device)
+        off = (-self.buf.data_ptr()) % 256
+        return self.buf[off:off + nbytes]
+
+
+_default_ws = {}
+
+
+def _workspace(ws: Optional[Workspace], device) -> Workspace:
+    if ws is not None:
+        return ws
+    device = torch.device(device)
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def scan_args(planes, qmin, qscale, q, alloc, k: int, n: int, out_idx, out_score,
+              debug_scores=None, flags: int = 0, host_mapped: bool = False) -> ScanArgs:
+    h_q, d = q.shape
+    h_kv = qmin.shape[0]
+    return ScanArgs(planes=planes.data_ptr(),
+                    planes_location=PLANES_HOST_MAPPED if host_mapped else PLANES_DEVICE,
+                    qmin=qmin.data_ptr(), qscale=qscale.data_ptr(), q=q.data_ptr(),
+                    q_dtype=_dtype_code(q), alloc=alloc.data_ptr(), n=int(n), d=d, h_q=h_q,
+                    h_kv=h_kv, k=int(k), out_idx=out_idx.data_ptr(),
+                    out_score=out_score.data_ptr(),
+                    debug_scores=None if debug_scores is None else debug_scores.data_ptr(),
+                    flags=int(flags))
+
+
+def scan_topk(planes: torch.Tensor, qmin: torch.Tensor, qscale: torch.Tensor, q: torch.Tensor,
+              alloc: torch.Tensor, k: int, n: int, *, host_mapped: bool = False,
+              debug_scores: bool = False, flags: int = 0, workspace: Optional[Workspace] = None,
+              stream=None, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """Top-k keys per query head.  Returns (idx int32 [h_q,k], score f32 [h_q,k]) and,
+    with debug_scores=True, also every score f32 [h_q, n]."""
+    dev = q.device
+    h_q = q.shape[0]
+    if out is None:
+        out = (torch.empty((h_q, k), dtype=torch.int32, device=dev),
+               torch.empty((h_q, k), dtype=torch.float32, device=dev))
+    dbg = torch.empty((h_q, n), dtype=torch.float32, device=dev) if debug_scores else None
+    args = scan_args(planes, qmin, qscale, q, alloc, k, n, out[0], out[1], dbg, flags, host_mapped)
+    L = lib()
+    need = L.fathom_scan_topk_workspace_size(ctypes.byref(args))
+    if need == 0:
+        _check(L.fathom_scan_topk(ctypes.byref(args), None, 0, _stream(stream)))
+    ws = _workspace(workspace, dev)
+    buf = ws.get(need)
+    _check(L.fathom_scan_topk(ctypes.byref(args), _ptr(buf), need, _stream(stream)))
+    if debug_scores:
+        return out[0], out[1], dbg
+    return out
+
+
+def scan_topk_batched(sessions: Sequence[dict], k: int, d: int, h_q: int, h_kv: int,
+                      q_dtype: torch.dtype = torch.bfloat16, *, host_mapped: bool = False,
+                      flags: int = 0, workspace: Optional[Workspace] = None, stream=None,
+                      device=None):
+    """Many sessions in one launch set.  Each session dict holds planes, qmin, qscale, q,
+    alloc, n (and optionally out_idx/out_score).  Returns a list of (idx, score)."""
+    device = torch.device(device or sessions[0]["q"].device)
+    S = len(sessions)
+    arr = (Session * S)()
+    outs: List[Tuple[torch.Tensor, torch.Tensor]] = []
+    n_max = 0
+    for i, s in enumerate(sessions):
+        oi = s.get("out_idx")
+        osc = s.get("out_score")
+        if oi is None:
+            oi = torch.empty((h_q, k), dtype=torch.int32, device=device)
+            osc = torch.empty((h_q, k), dtype=torch.float32, device=device)
+        outs.append((oi, osc))
+        arr[i] = Session(planes=s["planes"].data_ptr(), qmin=s["qmin"].data_ptr(),
+                         qscale=s["qscale"].data_ptr(), q=s["q"].data_ptr(),
+                         alloc=s["alloc"].data_ptr(), n=int(s["n"]), out_idx=oi.data_ptr(),
+                         out_score=osc.data_ptr())
+        n_max = max(n_max, int(s["n"]))
+    raw = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+    dev_desc = raw.to(device, non_blocking=False)
+    args = BatchedArgs(sessions=dev_desc.data_ptr(), num_sessions=S, n_max=n_max, d=d, h_q=h_q,
+                       h_kv=h_kv, k=int(k), q_dtype=BF16 if q_dtype == torch.bfloat16 else F32,
+                       planes_location=PLANES_HOST_MAPPED if host_mapped else PLANES_DEVICE,
+                       flags=int(flags))
+    L = lib()
+    need = L.fathom_scan_topk_batched_workspace_size(ctypes.byref(args))
+    if need == 0:
+        _check(L.fathom_scan_topk_batched(ctypes.byref(args), None, 0, _stream(stream)))
+    ws = _workspace(workspace, device)
+    buf = ws.get(need)
+    _check(L.fathom_scan_topk_batched(ctypes.byref(args), _ptr(buf), need, _stream(stream)))
+    # The descriptor tensor may be freed now: torch's caching allocator only
+    # hands its block to later work ordered after these launches on this stream.
+    ws.keepalive = dev_desc
+    return outs
+
+
+def profile_scan_kernel(begin: Optional[torch.cuda.Event], end: Optional[torch.cuda.Event]):
+    """Record begin/end around the filtering scan kernel of later scans (None clears)."""
+    if begin is None or end is None:
+        lib().fathom_profile_scan_kernel(None, None)
+        return
+    lib().fathom_profile_scan_kernel(ctypes.c_void_p(begin.cuda_event),
+                                     ctypes.c_void_p(end.cuda_event))
+
+
+def read_report(workspace: Optional[Workspace] = None, device=None, stream=None) -> ScanReport:
+    ws = _workspace(workspace, device or "cuda")
+    rep = ScanReport()
+    _check(lib().fathom_scan_read_report(_ptr(ws.buf[(-ws.buf.data_ptr()) % 256:]),
+                                         ctypes.byref(rep), _stream(stream)))
+    return rep

@@ -1,0 +1,215 @@
+/*
+ * fathom.h -- C ABI of the B200 (sm_100a) Fathom query-adaptive key scan.
+ *
+ * Fathom ("Fathom: Per-Query Read Depth for Sparse Decoding over Offloaded
+ * KV Caches", arXiv 2609.17652; summarised in "Fathom Makes KV-Cache Scans
+ * Query-Adaptive for Long-Context Decoding", cctest.ai) ranks all n cached
+ * keys for each decode step's top-k.  Its 4-bit K cache is stored as
+ * channel-major bit planes, so the first t planes of a channel are that
+ * channel's t-bit quantiser; each query spends a budget of B bits per key
+ * over its channels by reverse water-filling, and only the allocated plane
+ * prefixes are read.
+ *
+ * Four steps, three calls on the hot path:
+ *   fathom_pack_planes   4-bit codes -> bit planes (once per cache, off the
+ *                        per-step path);
+ *   fathom_allocate      per query head, bits per channel (the allocation);
+ *   fathom_scan_topk     scores of all n keys from the allocated prefixes and
+ *                        the per-head top-k (one session);
+ *   fathom_scan_topk_batched   the same for many sessions in one launch set.
+ *
+ * Conventions shared by every call
+ *   - The caller owns every buffer.  The library never allocates or frees;
+ *     scans take a caller-sized workspace (see *_workspace_size).
+ *   - Pointers are CUDA device pointers unless a parameter says otherwise.
+ *     Plane stores may instead live in pinned, mapped host memory
+ *     (FATHOM_PLANES_HOST_MAPPED): the scan then reads only the allocated
+ *     prefixes across the host link.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     stream-ordered and asynchronous: none synchronises the host except
+ *     fathom_scan_read_report.
+ *   - Every call validates its arguments on the host before any launch and
+ *     returns a status; on error nothing is launched and
+ *     fathom_last_error() holds a message.  No C++ exception crosses the ABI.
+ *   - Notation: KV heads g < h_kv, query heads h < h_q with G = h_q / h_kv
+ *     query heads per KV head (head h reads KV head h / G), channels c < d,
+ *     tokens i < n, plane j < 4 (j = 0 is the code's most significant bit).
+ */
+#ifndef FATHOM_H
+#define FATHOM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FATHOM_API __attribute__((visibility("default")))
+#else
+#define FATHOM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fathom_status {
+  FATHOM_OK = 0,
+  FATHOM_ERR_INVALID_ARGUMENT = 1,     /* bad size, null or wrong-kind pointer */
+  FATHOM_ERR_UNSUPPORTED = 2,          /* valid but outside this build's limits */
+  FATHOM_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes below *_workspace_size */
+  FATHOM_ERR_CUDA = 4,                 /* a CUDA runtime call or launch failed */
+  FATHOM_ERR_DEVICE_CHECK = 5          /* a device-side check recorded a fault */
+} fathom_status;
+
+typedef enum fathom_dtype { FATHOM_F32 = 0, FATHOM_BF16 = 1 } fathom_dtype;
+
+typedef enum fathom_planes_location {
+  FATHOM_PLANES_DEVICE = 0,      /* planes in device memory (HBM) */
+  FATHOM_PLANES_HOST_MAPPED = 1  /* planes in pinned host memory mapped into the device */
+} fathom_planes_location;
+
+/* Limits of this build. */
+#define FATHOM_MAX_D 256    /* d is a multiple of 32, 32 <= d <= 256 */
+#define FATHOM_MAX_GROUP 4  /* G = h_q / h_kv is 1, 2 or 4 */
+#define FATHOM_MAX_K 8192   /* 1 <= k <= 8192 */
+
+/* Test knobs for fathom_scan_args.flags (0 in normal use). */
+#define FATHOM_FLAG_NO_SAMPLING 1u     /* skip the threshold sample: every key is a candidate */
+#define FATHOM_FLAG_FORCE_FALLBACK 2u  /* take the exact single-block fallback for every head */
+
+/* Last error message of the calling thread ("" if none). */
+FATHOM_API const char *fathom_last_error(void);
+
+/* ---------------------------------------------------------------------------
+ * Bit-plane store layout (method paragraph 2, "stored in channel-major bit
+ * planes"; abstract, "a prefix of t planes is exactly the channel's t-bit
+ * quantizer"):
+ *   planes[g][c][j][w], uint32, w < W = fathom_plane_words(n);
+ *   bit b of word w of plane j holds bit (3 - j) of the code of token
+ *   32 w + b; rows are padded to a multiple of 128 tokens (16 bytes) and
+ *   every bit of a token >= n is 0.
+ * The t planes of a channel's prefix are one contiguous run of t*W words.
+ */
+FATHOM_API int64_t fathom_plane_words(int64_t n);
+FATHOM_API size_t fathom_planes_bytes(int64_t n, int d, int h_kv);
+
+/* fathom_pack_planes -- build the bit-plane store from a 4-bit K cache.
+ *   codes   [h_kv][n][d/2] uint8, token-major, two channels per byte, low
+ *           nibble = even channel: the per-channel asymmetric 4-bit codes a
+ *           quantised serving stack holds (abstract: "the store is the 4-bit
+ *           K copy a quantized serving stack already holds").  Read only.
+ *   planes  [h_kv][d][4][fathom_plane_words(n)] uint32, written in full
+ *           (padding zeroed).  16-byte aligned.
+ * n >= 0 (n = 0 writes nothing), d as FATHOM_MAX_D, h_kv >= 1.
+ */
+FATHOM_API fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int d, int h_kv,
+                                 uint32_t *planes, void *stream);
+
+/* fathom_allocate -- per-query bit allocation by reverse water-filling
+ * (method paragraph 3: "a reverse water-filling rule to assign more bits to
+ * channels that matter more for the current query... a closed-form
+ * solution"; abstract: "over the variance-weighted importance of its
+ * channels").
+ *   q       [h_q][d], FATHOM_BF16 or FATHOM_F32.
+ *   sigma   [h_kv][d] float, the channel statistics sigma_c (head h uses row
+ *           h / G).  Importance w_c = q_c^2 sigma_c^2 (fp64).
+ *   alloc   [h_q][d] uint8 out: t_c in 0..4 with sum_c t_c = budget_bits.
+ * The continuous rule is b_c = clip(log2(w_c / theta) / 2, 0, 4) with theta
+ * set so that sum_c b_c = B.  Its integer form, computed exactly: take the B
+ * largest of the 4d slot keys w_c 4^-tau (tau = 0..3), ties broken by lower
+ * channel then lower tau, and let t_c count channel c's slots.  This is the
+ * exact optimum of sum_c w_c 4^-t_c subject to sum_c t_c = B and equals the
+ * largest-remainder rounding of the closed form.  0 <= budget_bits <= 4d.
+ * For many sessions pass them concatenated: h_q = S*H_q, sigma [S*H_kv][d].
+ */
+FATHOM_API fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, const float *sigma, int h_q,
+                              int h_kv, int d, int budget_bits, uint8_t *alloc, void *stream);
+
+/* fathom_scan_topk -- score all n keys of one session from the allocated
+ * plane prefixes and return each query head's top-k (method paragraph 1:
+ * "scan a large number of keys to identify the top-k candidates"; abstract:
+ * "the scan that ranks all n keys for a top-k step").
+ *
+ * Score of key i for query head h (KV head g = h / G):
+ *   s_h(i) = sum_c q_c * deq_{t_c}(v_{t_c}(i, c)),
+ * v_t the value of the first t planes of channel c and
+ * deq_t(v) = m_c + s_c (2^(4-t) v + (2^(4-t) - 1) / 2), the centre of the
+ * t-bit cell (t = 0: the constant m_c + 7.5 s_c).  Scores accumulate in fp32.
+ * Output per head: the k keys with the largest s_h, ordered by score
+ * descending then index ascending; if k > n the tail is index -1, score -inf.
+ * Per KV head the scan reads, for each channel, the longest prefix any of its
+ * G query heads was allocated (the union); each head uses only its own.
+ */
+typedef struct fathom_scan_args {
+  const uint32_t *planes;  /* [h_kv][d][4][W] (device, or host-mapped pinned) */
+  int planes_location;     /* fathom_planes_location */
+  const float *qmin;       /* [h_kv][d] m_c, float */
+  const float *qscale;     /* [h_kv][d] s_c, float */
+  const void *q;           /* [h_q][d], q_dtype */
+  int q_dtype;             /* fathom_dtype */
+  const uint8_t *alloc;    /* [h_q][d] from fathom_allocate */
+  int64_t n;               /* keys, 0 <= n < 2^31 */
+  int d, h_q, h_kv, k;
+  int32_t *out_idx;        /* [h_q][k] out */
+  float *out_score;        /* [h_q][k] out */
+  float *debug_scores;     /* optional [h_q][n] out: every score (tests); NULL normally */
+  uint32_t flags;          /* FATHOM_FLAG_* test knobs, 0 normally */
+} fathom_scan_args;
+
+/* Bytes of workspace fathom_scan_topk needs for these arguments (0 on bad
+ * arguments).  The workspace is device memory, 256-byte aligned, owned by the
+ * caller, reused across calls; calls sharing one workspace must not overlap. */
+FATHOM_API size_t fathom_scan_topk_workspace_size(const fathom_scan_args *args);
+FATHOM_API fathom_status fathom_scan_topk(const fathom_scan_args *args, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/* Batched ragged sessions ("many sessions resident at once", abstract): one
+ * set of launches scores every session; sessions share d, h_q, h_kv, k and
+ * the dtype and differ in n and buffers.  `sessions` is a DEVICE array of S
+ * descriptors (pointers in it are not checked on the host). */
+typedef struct fathom_session {
+  const uint32_t *planes;  /* [h_kv][d][4][fathom_plane_words(n)] */
+  const float *qmin;       /* [h_kv][d] */
+  const float *qscale;     /* [h_kv][d] */
+  const void *q;           /* [h_q][d] */
+  const uint8_t *alloc;    /* [h_q][d] */
+  int64_t n;               /* 0 <= n <= n_max */
+  int32_t *out_idx;        /* [h_q][k] */
+  float *out_score;        /* [h_q][k] */
+} fathom_session;
+
+typedef struct fathom_batched_args {
+  const fathom_session *sessions; /* device array [num_sessions] */
+  int num_sessions;               /* 1 <= S <= 1024 */
+  int64_t n_max;                  /* an upper bound on every session's n */
+  int d, h_q, h_kv, k;
+  int q_dtype;                    /* fathom_dtype */
+  int planes_location;            /* fathom_planes_location, all sessions */
+  uint32_t flags;                 /* FATHOM_FLAG_* */
+} fathom_batched_args;
+
+FATHOM_API size_t fathom_scan_topk_batched_workspace_size(const fathom_batched_args *args);
+FATHOM_API fathom_status fathom_scan_topk_batched(const fathom_batched_args *args, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/* Profiling hook: while set, every scan launch set of the calling thread
+ * records `begin` (a cudaEvent_t) on its stream just before the filtering scan
+ * kernel -- the kernel that streams the union plane prefixes -- and `end`
+ * just after it, so a caller can time that kernel alone with
+ * cudaEventElapsedTime.  Pass NULL, NULL to clear.  Never synchronises. */
+FATHOM_API void fathom_profile_scan_kernel(void *begin, void *end);
+
+/* What the last scan on a workspace recorded.  Synchronises `stream`. */
+typedef struct fathom_scan_report {
+  uint32_t fallback_heads;  /* heads whose sampled threshold failed; answered exactly by the fallback */
+  uint32_t device_faults;   /* device-side check failures (0 expected) */
+  uint32_t max_candidates;  /* largest per-head candidate count */
+  uint32_t union_planes;    /* sum over sessions and KV heads of the union prefix planes */
+} fathom_scan_report;
+
+FATHOM_API fathom_status fathom_scan_read_report(const void *workspace, fathom_scan_report *report,
+                                      void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FATHOM_H */

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI: the library loads, exports everything
+include/fathom.h declares, and rejects bad arguments before any launch.
+No GPU needed: every call here fails validation (or only sizes things)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_plane_kv_scan_b200 import build as fbuild
+from bit_plane_kv_scan_b200 import fathom as F
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fbuild.build()
+    return F.lib()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "fathom.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fathom_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for want in ("fathom_pack_planes", "fathom_allocate", "fathom_scan_topk",
+                 "fathom_scan_topk_batched", "fathom_scan_topk_workspace_size"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert names
+    for name in names:
+        assert hasattr(L, name), name
+    assert sorted(F.EXPORTED) == names
+
+
+def test_plane_words(L):
+    assert [L.fathom_plane_words(n) for n in (0, 1, 127, 128, 129, 1 << 20)] == \
+        [0, 4, 4, 4, 8, 32768]
+    assert L.fathom_planes_bytes(1 << 20, 128, 8) == 8 * 128 * 4 * 32768 * 4
+
+
+def _status(call):
+    return call
+
+
+def test_pack_rejects_bad_shapes(L):
+    assert L.fathom_pack_planes(None, 100, 33, 1, None, None) == F.ERR_UNSUPPORTED
+    assert L.fathom_pack_planes(None, 100, 512, 1, None, None) == F.ERR_UNSUPPORTED
+    assert L.fathom_pack_planes(None, -1, 128, 1, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_pack_planes(None, 100, 128, 0, None, None) == F.ERR_INVALID_ARGUMENT
+    # null codes
+    assert L.fathom_pack_planes(None, 100, 128, 1, None, None) == F.ERR_INVALID_ARGUMENT
+    assert b"codes" in L.fathom_last_error()
+    # n = 0 is a no-op
+    assert L.fathom_pack_planes(None, 0, 128, 1, None, None) == F.OK
+
+
+def test_pack_rejects_host_pointers(L):
+    buf = ctypes.create_string_buffer(4096)
+    st = L.fathom_pack_planes(ctypes.addressof(buf), 32, 32, 1, ctypes.addressof(buf), None)
+    assert st == F.ERR_INVALID_ARGUMENT
+    assert b"device pointer" in L.fathom_last_error()
+
+
+def test_allocate_rejects_bad_arguments(L):
+    assert L.fathom_allocate(None, F.BF16, None, 32, 8, 100, 92, None, None) == F.ERR_UNSUPPORTED
+    assert L.fathom_allocate(None, F.BF16, None, 30, 8, 128, 92, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate(None, F.BF16, None, 32, 8, 128, 513, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate(None, F.BF16, None, 32, 8, 128, -1, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate(None, 7, None, 32, 8, 128, 92, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate(None, F.BF16, None, 32, 8, 128, 92, None, None) == F.ERR_INVALID_ARGUMENT
+
+
+def _args(**kw):
+    a = dict(planes=None, planes_location=F.PLANES_DEVICE, qmin=None, qscale=None, q=None,
+             q_dtype=F.BF16, alloc=None, n=1 << 20, d=128, h_q=32, h_kv=8, k=2048,
+             out_idx=None, out_score=None, debug_scores=None, flags=0)
+    a.update(kw)
+    return F.ScanArgs(**a)
+
+
+def test_scan_workspace_size_and_limits(L):
+    ws = L.fathom_scan_topk_workspace_size(ctypes.byref(_args()))
+    assert ws > 0 and ws % 256 == 0
+    # candidate buffers dominate: 32 heads x capacity x 8 bytes
+    assert ws >= 32 * 8 * 8 * 2048
+    for bad in (dict(d=100), dict(h_q=24), dict(h_q=64), dict(k=0), dict(k=8193),
+                dict(n=-1), dict(n=1 << 31), dict(q_dtype=9), dict(planes_location=5)):
+        assert L.fathom_scan_topk_workspace_size(ctypes.byref(_args(**bad))) == 0, bad
+    # G = 1 and G = 2 are supported
+    assert L.fathom_scan_topk_workspace_size(ctypes.byref(_args(h_q=8))) > 0
+    assert L.fathom_scan_topk_workspace_size(ctypes.byref(_args(h_q=16))) > 0
+    # no sampling needs room for every key as a candidate
+    big = L.fathom_scan_topk_workspace_size(ctypes.byref(_args(flags=F.FLAG_NO_SAMPLING)))
+    assert big >= 32 * 8 * (1 << 20)
+
+
+def test_scan_rejects_before_launch(L):
+    assert L.fathom_scan_topk(None, None, 0, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_scan_topk(ctypes.byref(_args(h_q=24)), None, 0, None) == F.ERR_UNSUPPORTED
+    assert L.fathom_scan_topk(ctypes.byref(_args()), None, 0, None) == F.ERR_INVALID_ARGUMENT
+    assert b"qmin" in L.fathom_last_error()
+
+
+def test_batched_rejects_bad_arguments(L):
+    a = F.BatchedArgs(sessions=None, num_sessions=0, n_max=1000, d=128, h_q=32, h_kv=8, k=1024,
+                      q_dtype=F.BF16, planes_location=F.PLANES_DEVICE, flags=0)
+    assert L.fathom_scan_topk_batched_workspace_size(ctypes.byref(a)) == 0
+    assert L.fathom_scan_topk_batched(ctypes.byref(a), None, 0, None) == F.ERR_INVALID_ARGUMENT
+    a.num_sessions = 32
+    assert L.fathom_scan_topk_batched_workspace_size(ctypes.byref(a)) > 0
+    assert L.fathom_scan_topk_batched(ctypes.byref(a), None, 0, None) == F.ERR_INVALID_ARGUMENT
+    assert b"sessions" in L.fathom_last_error()
+
+
+def test_report_rejects_null(L):
+    assert L.fathom_scan_read_report(None, None, None) == F.ERR_INVALID_ARGUMENT

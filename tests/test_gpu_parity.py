@@ -1,0 +1,326 @@
+"""Parity of the CUDA scan (through the C ABI) with the CPU oracle.
+
+Rules and tolerances: tests/parity.py.  Small cases compare every output;
+the full-size workloads (131k, 1M, 32 ragged sessions, host-resident planes)
+run in the launch configuration the benchmark times and compare every
+allocation, the full top-k of a subset of heads against the oracle's
+brute force, and every returned score against the oracle's score at that
+index.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthkv
+from parity import check_dense, check_scores_at, check_topk, check_topk_sampled, score_scale
+
+pytestmark = pytest.mark.gpu
+
+F = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global F
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import bit_plane_kv_scan_b200 as fb
+    from bit_plane_kv_scan_b200 import build
+    build.build()
+    F = fb
+    F.lib()
+    yield
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _planes_np(planes):
+    return _np(planes).view(np.uint32)
+
+
+def run_gpu(case, budget, k, flags=0, debug=False, host_mapped=False):
+    dev = torch.device("cuda")
+    codes = case.codes.to(dev)
+    planes = F.pack_planes(codes)
+    if host_mapped:
+        hp = torch.empty(planes.shape, dtype=planes.dtype, pin_memory=True)
+        hp.copy_(planes)
+        planes_used = hp
+    else:
+        planes_used = planes
+    q = case.q_storage().to(dev)
+    sigma = case.sigma.to(dev)
+    alloc = F.allocate(q, sigma, budget)
+    out = F.scan_topk(planes_used, case.qmin.to(dev), case.qscale.to(dev), q, alloc, k, case.n,
+                      debug_scores=debug, flags=flags, host_mapped=host_mapped)
+    torch.cuda.synchronize()
+    return planes, alloc, out
+
+
+def oracle_head(case_np, h, t_h):
+    codes, qmin, qscale, q = case_np
+    G = q.shape[0] // codes.shape[0]
+    g = h // G
+    return oracle.scores_from_codes(codes[g], qmin[g], qscale[g], q[h], t_h)
+
+
+def case_np(case):
+    return (_np(case.codes), _np(case.qmin), _np(case.qscale), _np(case.q).astype(np.float64))
+
+
+# ------------------------------------------------------------------ pack --
+
+@pytest.mark.parametrize("n,d,h_kv", [(1, 32, 1), (31, 64, 2), (4096, 128, 1), (4097, 128, 2),
+                                      (33333, 256, 1), (100000, 96, 3)])
+def test_pack_bit_exact(n, d, h_kv):
+    rng = np.random.default_rng(n + d)
+    codes = rng.integers(0, 256, size=(h_kv, n, d // 2), dtype=np.uint8)
+    planes = F.pack_planes(torch.from_numpy(codes).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(_planes_np(planes), oracle.pack_planes(codes))
+
+
+def test_pack_full_size_1m():
+    case = synthkv.make_case(seed=2, n=1 << 20, h_kv=8, h_q=32, device="cuda", keep_keys=False)
+    planes = F.pack_planes(case.codes)
+    torch.cuda.synchronize()
+    got = _planes_np(planes)
+    codes = _np(case.codes)
+    # the oracle packs two KV heads in full; the rest are checked on sampled words
+    for g in (0, 7):
+        np.testing.assert_array_equal(got[g:g + 1], oracle.pack_planes(codes[g:g + 1]))
+    rng = np.random.default_rng(0)
+    for g in range(8):
+        for w in rng.integers(0, got.shape[-1], 16):
+            sl = codes[g:g + 1, 32 * w:32 * w + 32]
+            ref = oracle.pack_planes(sl)[0, :, :, 0]
+            np.testing.assert_array_equal(got[g, :, :, w], ref)
+
+
+# -------------------------------------------------------------- allocate --
+
+def _alloc_cases():
+    rng = np.random.default_rng(42)
+    out = []
+    for d in (32, 128, 256):
+        q = rng.normal(size=(8, d)) * np.exp(rng.normal(size=(8, d)))
+        sigma = np.exp(rng.uniform(np.log(0.1), np.log(10), size=(2, d)))
+        out.append(("random_d%d" % d, q, sigma))
+    d = 128
+    q = np.zeros((4, d))
+    q[0, ::7] = 1.0                     # many equal weights
+    q[1, :] = 2.0 ** rng.integers(-4, 4, d)  # weights that tie across channels after 4^-tau
+    q[2, :5] = [1, -1, 2, -2, 0.5]      # mostly zero weights
+    q[3, :] = 1.0                       # all equal
+    out.append(("ties", q, np.ones((1, d))))
+    return out
+
+
+@pytest.mark.parametrize("name,q,sigma", _alloc_cases(), ids=lambda x: x if isinstance(x, str) else "")
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_allocate_bit_exact(name, q, sigma, dtype):
+    d = q.shape[1]
+    qt = torch.from_numpy(q).to(dtype)
+    qd = qt.float().numpy().astype(np.float64)  # the exact values the library sees
+    sig = torch.from_numpy(sigma).float()
+    for B in sorted(x for x in {0, 1, 5, 68, 92, 136, 4 * d - 1, 4 * d} if x <= 4 * d):
+        got = _np(F.allocate(qt.cuda(), sig.cuda(), B))
+        want = oracle.allocate_heads(qd, sig.numpy().astype(np.float64), B)
+        np.testing.assert_array_equal(got, want, err_msg="%s B=%d" % (name, B))
+
+
+# ------------------------------------------------------------ small scans --
+
+def _full_check(case, budget, k, flags=0, what=""):
+    planes, alloc, (idx, sc, dbg) = run_gpu(case, budget, k, flags=flags, debug=True)
+    cn = case_np(case)
+    want_alloc = oracle.allocate_heads(cn[3], _np(case.sigma), budget)
+    np.testing.assert_array_equal(_np(alloc), want_alloc)
+    np.testing.assert_array_equal(_planes_np(planes), oracle.pack_planes(cn[0]))
+    G = case.group
+    idx, sc, dbg = _np(idx), _np(sc), _np(dbg)
+    for h in range(case.h_q):
+        g = h // G
+        ref = oracle_head(cn, h, want_alloc[h])
+        scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
+        check_dense(dbg[h], ref, scale, "%s head %d" % (what, h))
+        check_topk(idx[h], sc[h], ref, k, scale, "%s head %d" % (what, h))
+
+
+def test_tiny_4k_config():
+    """The tiny single-head workload: n=4096, d=128, fp32 query, B=92, k=64."""
+    c = synthkv.CONFIGS["tiny_4k"]
+    case = synthkv.make_case(c["seed"], c["n"], c["h_kv"], c["h_q"], c["d"], c["q_dtype"])
+    _full_check(case, 92, 64, what="tiny_4k")
+
+
+@pytest.mark.parametrize("n", [1, 33, 4095, 4097, 12345])
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_ragged_n_and_groups(n, G):
+    case = synthkv.make_case(seed=100 + n + G, n=n, h_kv=2, h_q=2 * G, d=128, q_dtype="bf16")
+    for B, k in ((92, 7), (17, 100)):
+        _full_check(case, B, k, what="n=%d G=%d B=%d k=%d" % (n, G, B, k))
+
+
+@pytest.mark.parametrize("d", [32, 64, 256])
+def test_other_widths(d):
+    case = synthkv.make_case(seed=d, n=5000, h_kv=1, h_q=4, d=d, q_dtype="bf16")
+    _full_check(case, d // 2, 33, what="d=%d" % d)
+
+
+@pytest.mark.parametrize("B", [0, 1, 512])
+def test_degenerate_budgets(B):
+    """B = 0: every score is the per-query constant and the top-k is the first
+    k indices; B = 4d: the full 4-bit dequantised dot product."""
+    case = synthkv.make_case(seed=7, n=3000, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+    _full_check(case, B, 50, what="B=%d" % B)
+    if B == 0:
+        _, _, (idx, sc) = run_gpu(case, 0, 50)
+        assert (_np(idx) == np.arange(50)[None, :]).all()
+
+
+def test_k_larger_than_n_and_empty():
+    case = synthkv.make_case(seed=8, n=40, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+    _full_check(case, 92, 64, what="k>n")
+    empty = synthkv.make_case(seed=9, n=0 + 1, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+    dev = torch.device("cuda")
+    q = empty.q_storage().to(dev)
+    alloc = F.allocate(q, empty.sigma.to(dev), 92)
+    planes = torch.zeros((1, 128, 4, 4), dtype=torch.int32, device=dev)
+    idx, sc = F.scan_topk(planes, empty.qmin.to(dev), empty.qscale.to(dev), q, alloc, 5, 0)
+    torch.cuda.synchronize()
+    assert (_np(idx) == -1).all() and np.isneginf(_np(sc)).all()
+
+
+def test_sampled_threshold_path_and_fallbacks():
+    """n large enough that the sampled threshold is used (k=64 samples from
+    n >= 8192); the forced fallback and the no-sampling path must give the
+    same answer."""
+    case = synthkv.make_case(seed=21, n=40000, h_kv=2, h_q=8, d=128, q_dtype="bf16")
+    _full_check(case, 92, 64, what="sampled")
+    _, _, base = run_gpu(case, 92, 64)
+    rep = F.read_report()
+    assert rep.fallback_heads == 0
+    _full_check(case, 92, 64, flags=F.FLAG_FORCE_FALLBACK, what="fallback")
+    _, _, forced = run_gpu(case, 92, 64, flags=F.FLAG_FORCE_FALLBACK)
+    rep = F.read_report()
+    assert rep.fallback_heads == 8
+    _full_check(case, 92, 64, flags=F.FLAG_NO_SAMPLING, what="no-sampling")
+    _, _, nos = run_gpu(case, 92, 64, flags=F.FLAG_NO_SAMPLING)
+    np.testing.assert_array_equal(_np(base[0]), _np(nos[0]))
+    np.testing.assert_array_equal(_np(base[1]), _np(nos[1]))
+
+
+def test_fallback_with_compaction():
+    """Forced fallback on a context long enough that the single-block stream
+    compacts its candidate buffer several times."""
+    case = synthkv.make_case(seed=22, n=300000, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+    _, alloc, (idx, sc) = run_gpu(case, 92, 1000, flags=F.FLAG_FORCE_FALLBACK)
+    cn = case_np(case)
+    for h in range(4):
+        ref = oracle_head(cn, h, _np(alloc)[h])
+        check_topk(_np(idx)[h], _np(sc)[h], ref, 1000, score_scale(cn[3][h], cn[1][0], cn[2][0]),
+                   "fallback head %d" % h)
+
+
+# ------------------------------------------------------ full-size configs --
+
+def _check_config(case, budget, k, heads_full, what, host_mapped=False):
+    _, alloc, (idx, sc) = run_gpu(case, budget, k, host_mapped=host_mapped)
+    cn = case_np(case)
+    want_alloc = oracle.allocate_heads(cn[3], _np(case.sigma), budget)
+    got_alloc = _np(alloc)
+    np.testing.assert_array_equal(got_alloc, want_alloc)
+    idx, sc = _np(idx), _np(sc)
+    G = case.group
+    for h in range(case.h_q):
+        g = h // G
+        scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
+        kk = min(k, case.n)
+        ref_at = oracle.scores_at(cn[0][g], cn[1][g], cn[2][g], cn[3][h], want_alloc[h],
+                                  idx[h, :kk].astype(np.int64))
+        check_topk_sampled(idx[h], sc[h], ref_at, k, case.n, scale, "%s head %d" % (what, h))
+        if h in heads_full:
+            ref = oracle_head(cn, h, want_alloc[h])
+            check_topk(idx[h], sc[h], ref, k, scale, "%s head %d" % (what, h))
+    return idx, sc
+
+
+@pytest.fixture(scope="module")
+def layer_131k():
+    c = synthkv.CONFIGS["qwen3_8b_layer_131k"]
+    return synthkv.make_case(c["seed"], c["n"], c["h_kv"], c["h_q"], c["d"], c["q_dtype"],
+                             device="cuda", keep_keys=False)
+
+
+@pytest.mark.parametrize("B", [68, 92, 136])
+def test_qwen3_8b_layer_131k(layer_131k, B):
+    _check_config(layer_131k, B, 2048, heads_full=set(range(32)), what="131k B=%d" % B)
+
+
+@pytest.fixture(scope="module")
+def decode_1m():
+    c = synthkv.CONFIGS["decode_1m"]
+    return synthkv.make_case(c["seed"], c["n"], c["h_kv"], c["h_q"], c["d"], c["q_dtype"],
+                             device="cuda", keep_keys=False)
+
+
+@pytest.mark.parametrize("B", [92, 136])
+def test_decode_1m(decode_1m, B):
+    # full brute force on one query head of every KV head; sampled checks on all
+    _check_config(decode_1m, B, 2048, heads_full={0, 5, 10, 15, 16, 21, 26, 31},
+                  what="1M B=%d" % B)
+    rep = F.read_report()
+    assert rep.fallback_heads == 0
+
+
+def test_host_resident_1m_budget_sweep():
+    """Planes in pinned host memory: same results as device-resident planes,
+    and oracle-checked, for every budget of the sweep."""
+    c = synthkv.CONFIGS["host_resident_1m"]
+    case = synthkv.make_case(c["seed"], c["n"], c["h_kv"], c["h_q"], c["d"], c["q_dtype"],
+                             device="cuda", keep_keys=False)
+    for B in c["budgets"]:
+        idx_h, sc_h = _check_config(case, B, 2048, heads_full={3} if B in (92, 512) else set(),
+                                    what="host B=%d" % B, host_mapped=True)
+        _, _, (idx_d, sc_d) = run_gpu(case, B, 2048)
+        np.testing.assert_array_equal(idx_h, _np(idx_d))
+        np.testing.assert_array_equal(sc_h, _np(sc_d))
+
+
+def test_ragged_32_sessions_batched():
+    c = synthkv.CONFIGS["ragged_32_sessions"]
+    sessions = synthkv.make_ragged(c["seed"], c["sessions"], c["n_lo"], c["n_hi"], c["h_kv"],
+                                   c["h_q"], c["d"], c["q_dtype"], device="cuda")
+    dev = torch.device("cuda")
+    k, B = c["k"], 92
+    # one allocation launch for every session's query heads
+    q_all = torch.cat([s.q_storage() for s in sessions]).to(dev)
+    sig_all = torch.cat([s.sigma for s in sessions]).to(dev)
+    alloc_all = F.allocate(q_all, sig_all, B)
+    descs = []
+    for i, s in enumerate(sessions):
+        descs.append(dict(planes=F.pack_planes(s.codes), qmin=s.qmin, qscale=s.qscale,
+                          q=q_all[i * 32:(i + 1) * 32], alloc=alloc_all[i * 32:(i + 1) * 32],
+                          n=s.n))
+    outs = F.scan_topk_batched(descs, k, 128, 32, 8, torch.bfloat16)
+    torch.cuda.synchronize()
+    want_alloc = oracle.allocate_heads(_np(q_all.float()).astype(np.float64), _np(sig_all), B)
+    np.testing.assert_array_equal(_np(alloc_all), want_alloc)
+    for i, s in enumerate(sessions):
+        cn = case_np(s)
+        idx, sc = _np(outs[i][0]), _np(outs[i][1])
+        for h in range(32):
+            g = h // 4
+            t_h = want_alloc[i * 32 + h]
+            scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
+            ref_at = oracle.scores_at(cn[0][g], cn[1][g], cn[2][g], cn[3][h], t_h,
+                                      idx[h, :min(k, s.n)].astype(np.int64))
+            check_topk_sampled(idx[h], sc[h], ref_at, k, s.n, scale, "session %d head %d" % (i, h))
+            if i in (0, 13, 31) and h in (0, 9, 18, 27):
+                ref = oracle_head(cn, h, t_h)
+                check_topk(idx[h], sc[h], ref, k, scale, "session %d head %d" % (i, h))
