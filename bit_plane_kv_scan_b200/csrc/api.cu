@@ -145,6 +145,11 @@ fathom_status check_scan_common(int64_t n, int d, int h_q, int h_kv, int k, int 
 
 }  // namespace
 
+namespace fathom {
+// Lets other translation units of the library report an error message.
+void set_error_message(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace fathom
+
 extern "C" {
 
 const char *fathom_last_error(void) { return g_err; }

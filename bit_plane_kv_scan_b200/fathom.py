@@ -36,8 +36,9 @@ EXPORTED = [
     "fathom_last_error", "fathom_plane_words", "fathom_planes_bytes", "fathom_pack_planes",
     "fathom_allocate", "fathom_scan_topk_workspace_size", "fathom_scan_topk",
     "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
-    "fathom_scan_read_report", "fathom_profile_scan_kernel",
+    "fathom_scan_read_report", "fathom_profile_scan_kernel", "fathom_scan_topk_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class FathomError(RuntimeError):
@@ -115,6 +116,8 @@ def lib() -> ctypes.CDLL:
         L.fathom_scan_read_report.argtypes = [vp, ctypes.POINTER(ScanReport), vp]
         L.fathom_profile_scan_kernel.restype = None
         L.fathom_profile_scan_kernel.argtypes = [vp, vp]
+        L.fathom_scan_topk_noalloc.restype = ci
+        L.fathom_scan_topk_noalloc.argtypes = [ctypes.POINTER(ScanArgs), vp]
         _lib = L
         return L
 

@@ -191,6 +191,34 @@ FATHOM_API size_t fathom_scan_topk_batched_workspace_size(const fathom_batched_a
 FATHOM_API fathom_status fathom_scan_topk_batched(const fathom_batched_args *args, void *workspace,
                                        size_t workspace_bytes, void *stream);
 
+/* fathom_scan_topk_noalloc -- fathom_scan_topk for callers that cannot
+ * allocate device memory.  The paper has no counterpart; this is a service of
+ * this library.
+ *
+ * Some callers may not call cudaMalloc: a plugin running inside an inference
+ * server that owns all device memory through its own pool and forbids
+ * plugins from allocating, or a latency-critical decode loop where an
+ * allocation can block or synchronise the device.  They still provide the
+ * inputs and outputs in `args`, but no workspace: this entry point uses a
+ * fixed scratch array compiled into the library, FATHOM_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) of device memory that every GPU which loads the library holds
+ * until the process exits.
+ *   - Sizes whose workspace (fathom_scan_topk_workspace_size) exceeds the
+ *     scratch are rejected with FATHOM_ERR_WORKSPACE_TOO_SMALL; nothing is
+ *     launched.  The 1M-token, 32-query-head, k = 2048 step fits.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.  The
+ *     first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, which may load the library's kernels onto that
+ *     device); make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the previous call's data;
+ *     each call clears the counters that must start at zero.  Calls whose
+ *     work overlaps on the GPU (different streams, or different host threads
+ *     without ordering) race on the scratch: order them.
+ *   - Results are those of fathom_scan_topk on the same arguments.
+ */
+#define FATHOM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+FATHOM_API fathom_status fathom_scan_topk_noalloc(const fathom_scan_args *args, void *stream);
+
 /* Profiling hook: while set, every scan launch set of the calling thread
  * records `begin` (a cudaEvent_t) on its stream just before the filtering scan
  * kernel -- the kernel that streams the union plane prefixes -- and `end`
