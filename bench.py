@@ -1,19 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of one Fathom decode step: allocation + bit-plane scan + top-k.
 
-Workload (default): the 1M-token decode step -- n = 1,048,576 keys, 8 KV heads
-x d = 128 channels stored as 4-bit channel-major bit planes (512 MiB), 32 bf16
+Default workload: the 1M-token decode step -- n = 1,048,576 keys, 8 KV heads x
+d = 128 channels stored as 4-bit channel-major bit planes (512 MiB), 32 bf16
 query heads (GQA 4), budget B = 92 bits per key, top-k = 2048 per query head.
-Inputs are seeded synthetic (synthkv); the planes are packed once, before
-timing, and stay resident in HBM.
+Other workloads (--config): qwen3_8b_layer_131k, host_resident_1m (planes in
+pinned host memory, read across the host link), ragged_32_sessions (one
+batched launch set for 32 sessions), tiny_4k.  Inputs are seeded synthetic
+(synthkv); the planes are packed once, before timing.
 
 One step = fathom_allocate + fathom_scan_topk (plan, sample scan, threshold,
 filtering scan, merge).  Device time per step comes from CUDA events on the
 launching stream; L2 is flushed (256 MiB write) between steps, outside the
 events.  The dominant kernel (the filtering scan) is timed alone with events
-recorded around it by the library's profiling hook.
+the library records around it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--config NAME] [--budget B]
 
 Under torchrun each rank scores its own session (seed + rank): weak scaling,
 no collective on the data path; the step time is the max over ranks.
@@ -39,9 +42,10 @@ sys.path.insert(0, ROOT)
 METRIC = "Gkeys/s scanned+top-k at 1M ctx, B=92 bits; achieved HBM GB/s vs B200 peak"
 UNIT = "Gkeys/s"
 FLUSH_BYTES = 256 << 20
+LAUNCHES_PER_STEP = 6  # allocate, plan, sample scan, threshold, filtering scan, merge
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -50,15 +54,10 @@ def parse():
     ap.add_argument("--config", default="decode_1m")
     ap.add_argument("--budget", type=int, default=92)
     ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--tensor-cores", action="store_true",
+                    help="run the scan on the tcgen05 kernel instead of the CUDA-core kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
-
-
-def workload_desc(cfg, budget, k):
-    return ("%s: n=%d keys, %d KV heads x d=%d (4-bit channel-major bit planes), %d %s query "
-            "heads (GQA %d), B=%d bits/key, top-k=%d" % (
-                cfg["name"], cfg["n"], cfg["h_kv"], cfg["d"], cfg["h_q"], cfg["q_dtype"],
-                cfg["h_q"] // cfg["h_kv"], budget, k))
+    return ap.parse_args(argv)
 
 
 def load_peaks():
@@ -69,6 +68,8 @@ def load_peaks():
     except Exception:
         return 6650.0, "fallback"
 
+
+# ------------------------------------------------------------------ timing --
 
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
@@ -162,6 +163,8 @@ def physical_gpu_index(local_rank: int) -> int:
     return local_rank
 
 
+# ------------------------------------------------------------ multi-rank --
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -169,7 +172,8 @@ def dist_setup():
     return world, rank, local
 
 
-def reduce_max(x: float, world: int, device) -> float:
+def reduce_max(x: float, world: int, device=None) -> float:
+    """The max of x over all ranks (every rank calls it)."""
     if world == 1:
         return x
     import torch
@@ -179,10 +183,27 @@ def reduce_max(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def reduce_sum(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def job_throughput(keys_this_rank: float, ms_this_rank: float, world: int, device=None):
+    """Whole-job keys/s (in G): all ranks' keys over the slowest rank's time."""
+    keys = reduce_sum(keys_this_rank, world, device)
+    ms = reduce_max(ms_this_rank, world, device)
+    return keys / (ms * 1e-3) / 1e9, ms
 
 
 def get_cfg(name):
@@ -190,6 +211,29 @@ def get_cfg(name):
     cfg = dict(synthkv.CONFIGS[name])
     cfg["name"] = name
     return cfg
+
+
+def workload_desc(cfg, budget, k):
+    if cfg["name"] == "ragged_32_sessions":
+        return ("ragged_32_sessions: 32 sessions, n ~ U[%d, %d] keys each, %d KV heads x d=%d, "
+                "%d %s query heads (GQA %d), B=%d bits/key, top-k=%d, one batched launch set" % (
+                    cfg["n_lo"], cfg["n_hi"], cfg["h_kv"], cfg["d"], cfg["h_q"], cfg["q_dtype"],
+                    cfg["h_q"] // cfg["h_kv"], budget, k))
+    where = " in pinned host memory" if cfg["name"] == "host_resident_1m" else ""
+    return ("%s: n=%d keys, %d KV heads x d=%d (4-bit channel-major bit planes%s), %d %s query "
+            "heads (GQA %d), B=%d bits/key, top-k=%d" % (
+                cfg["name"], cfg["n"], cfg["h_kv"], cfg["d"], where, cfg["h_q"], cfg["q_dtype"],
+                cfg["h_q"] // cfg["h_kv"], budget, k))
+
+
+def union_plane_bytes(alloc, n, h_kv, words):
+    """Bytes of the union prefixes one step reads: per KV head, for every
+    channel, the longest prefix any of its query heads was allocated, each
+    plane a row of `words` 32-bit words."""
+    a = np.asarray(alloc)
+    G = a.shape[0] // h_kv
+    tstar = a.reshape(h_kv, G, -1).max(axis=1)
+    return int(tstar.sum()) * words * 4
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -208,6 +252,11 @@ def oracle_sample(case_np, budget, k, heads):
     return time.perf_counter() - t0
 
 
+def case_numpy(case):
+    return (case.codes.cpu().numpy(), case.qmin.cpu().numpy(), case.qscale.cpu().numpy(),
+            case.q.cpu().numpy().astype(np.float64), case.sigma.cpu().numpy())
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle on a bounded sample of the same step."""
     import torch
@@ -220,26 +269,28 @@ def run_reference(args):
     import synthkv
     oracle.build()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    case = synthkv.make_case(cfg["seed"], cfg["n"], cfg["h_kv"], cfg["h_q"], cfg["d"],
-                             cfg["q_dtype"], device=dev, keep_keys=False)
-    cn = (case.codes.cpu().numpy(), case.qmin.cpu().numpy(), case.qscale.cpu().numpy(),
-          case.q.cpu().numpy().astype(np.float64), case.sigma.cpu().numpy())
-    heads_per_step = 1
+    if cfg["name"] == "ragged_32_sessions":
+        case = synthkv.make_ragged(cfg["seed"], 1, cfg["n_lo"], cfg["n_hi"], cfg["h_kv"],
+                                   cfg["h_q"], cfg["d"], cfg["q_dtype"], device=dev)[0]
+    else:
+        case = synthkv.make_case(cfg["seed"], cfg["n"], cfg["h_kv"], cfg["h_q"], cfg["d"],
+                                 cfg["q_dtype"], device=dev, keep_keys=False)
+    cn = case_numpy(case)
     for i in range(args.warmup):
         oracle_sample(cn, args.budget, k, [i % cfg["h_q"]])
     secs = [oracle_sample(cn, args.budget, k, [(args.warmup + i) % cfg["h_q"]])
             for i in range(args.steps)]
     t = float(np.mean(secs))
-    value = heads_per_step * cfg["n"] / t / 1e9
+    value = case.n / t / 1e9
     sample = ("one query head per step (allocation, fp64 scores of all %d keys, brute-force "
-              "top-%d), single thread" % (cfg["n"], k))
+              "top-%d), single thread" % (case.n, k))
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, synthkv)",
-        "config": {"workload": workload_desc(cfg, args.budget, k), "n": cfg["n"],
-                   "budget_bits": args.budget, "k": k, "l2": "n/a (CPU)"},
+        "config": {"workload": workload_desc(cfg, args.budget, k), "budget_bits": args.budget,
+                   "k": k, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -248,6 +299,26 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- native --
+
+def measure_h2d_gbs(device, nbytes=512 << 20):
+    """Pinned host -> device copy bandwidth, the host link's measured peak."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    for _ in range(2):
+        dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 0.0
+    for _ in range(5):
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del src, dst
+    return best
+
 
 def run_native(args):
     import torch
@@ -270,23 +341,60 @@ def run_native(args):
     cfg = get_cfg(args.config)
     k = args.k or cfg["k"]
     B = args.budget
-    n, h_kv, h_q, d = cfg["n"], cfg["h_kv"], cfg["h_q"], cfg["d"]
-    case = synthkv.make_case(cfg["seed"] + rank, n, h_kv, h_q, d, cfg["q_dtype"], device=device,
-                             keep_keys=False)
-    planes = F.pack_planes(case.codes)
-    q = case.q_storage().contiguous()
-    sigma, qmin, qscale = case.sigma, case.qmin, case.qscale
-    alloc = torch.empty((h_q, d), dtype=torch.uint8, device=device)
-    out = (torch.empty((h_q, k), dtype=torch.int32, device=device),
-           torch.empty((h_q, k), dtype=torch.float32, device=device))
+    h_kv, h_q, d = cfg["h_kv"], cfg["h_q"], cfg["d"]
+    flags = F.FLAG_TENSOR_CORES if args.tensor_cores else 0
+    ragged = cfg["name"] == "ragged_32_sessions"
+    host = cfg["name"] == "host_resident_1m"
     ws = F.Workspace(device)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step():
-        F.allocate(q, sigma, B, out=alloc)
-        F.scan_topk(planes, qmin, qscale, q, alloc, k, n, workspace=ws, out=out)
+    if ragged:
+        cases = synthkv.make_ragged(cfg["seed"] + 1000 * rank, cfg["sessions"], cfg["n_lo"],
+                                    cfg["n_hi"], h_kv, h_q, d, cfg["q_dtype"], device=device)
+    else:
+        cases = [synthkv.make_case(cfg["seed"] + rank, cfg["n"], h_kv, h_q, d, cfg["q_dtype"],
+                                   device=device, keep_keys=False)]
+    S = len(cases)
+    q_all = torch.cat([c.q_storage() for c in cases]).contiguous()
+    sigma_all = torch.cat([c.sigma for c in cases]).contiguous()
+    alloc_all = torch.empty((S * h_q, d), dtype=torch.uint8, device=device)
+    planes = []
+    for c in cases:
+        p = F.pack_planes(c.codes)
+        if host:
+            hp = torch.empty(p.shape, dtype=p.dtype, pin_memory=True)
+            hp.copy_(p)
+            p = hp
+        planes.append(p)
+        c.codes = None  # the scan reads only the planes
+    torch.cuda.synchronize()
+    outs = [(torch.empty((h_q, k), dtype=torch.int32, device=device),
+             torch.empty((h_q, k), dtype=torch.float32, device=device)) for _ in range(S)]
+    n_total = sum(c.n for c in cases)
 
+    def make_step(q_src):
+        if ragged:
+            descs = [dict(planes=planes[i], qmin=cases[i].qmin, qscale=cases[i].qscale,
+                          q=q_src[i * h_q:(i + 1) * h_q], alloc=alloc_all[i * h_q:(i + 1) * h_q],
+                          n=cases[i].n, out_idx=outs[i][0], out_score=outs[i][1])
+                     for i in range(S)]
+            scan = F.BatchedScan(descs, k, d, h_q, h_kv, q_src.dtype, flags=flags,
+                                 device=device)
+
+            def step():
+                F.allocate(q_src, sigma_all, B, out=alloc_all)
+                scan(ws)
+        else:
+            c = cases[0]
+
+            def step():
+                F.allocate(q_src, sigma_all, B, out=alloc_all)
+                F.scan_topk(planes[0], c.qmin, c.qscale, q_src, alloc_all, k, c.n,
+                            host_mapped=host, flags=flags, workspace=ws, out=outs[0])
+        return step
+
+    step = make_step(q_all)
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         step()
@@ -316,35 +424,42 @@ def run_native(args):
     step_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(sb, se)]))
     kern_ms = float(np.mean([event_ms(a, b) for a, b in zip(kb, ke)]))
     rep = F.read_report(ws)
-    t_step = reduce_max(step_ms, world, device)
+    keys_per_step = h_q * n_total
+    value, t_step = job_throughput(keys_per_step, step_ms, world, device)
     t_kern = reduce_max(kern_ms, world, device)
 
     # algorithmic bytes of the filtering scan: the union plane prefixes of
-    # every KV head (one plane row = W words), the per-head inputs it reads
-    # (q, alloc, m, s) and the candidates it writes (about 2k per head).
-    W = F.plane_words(n)
-    union_bytes = int(rep.union_planes) * W * 4
-    small_bytes = h_q * d * (q.element_size() + 1) + 2 * h_kv * d * 4
+    # every (session, KV head) plus the small per-head inputs (q, alloc, m, s)
+    alloc_np = alloc_all.cpu().numpy()
+    union_bytes = sum(union_plane_bytes(alloc_np[i * h_q:(i + 1) * h_q], c.n, h_kv,
+                                        F.plane_words(c.n)) for i, c in enumerate(cases))
+    small_bytes = S * (h_q * d * (q_all.element_size() + 1) + 2 * h_kv * d * 4)
     alg_bytes = union_bytes + small_bytes
-    peak, peak_kind = load_peaks()
     achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+    if host:
+        peak, peak_kind, bound = measure_h2d_gbs(device), "measured pinned host->device copy", \
+            "host-link"
+    else:
+        peak, peak_kind = load_peaks()
+        bound = "hbm"
 
     # end to end through the public API with host buffers: q uploaded from
     # pinned memory, top-k read back to pinned memory, inside the timed region
-    q_host = q.cpu().pin_memory()
-    q_dev = torch.empty_like(q)
-    idx_host = torch.empty((h_q, k), dtype=torch.int32, pin_memory=True)
-    sc_host = torch.empty((h_q, k), dtype=torch.float32, pin_memory=True)
-    eb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ee = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    q_host = q_all.cpu().pin_memory()
+    q_dev = torch.empty_like(q_all)
+    out_host = [(torch.empty((h_q, k), dtype=torch.int32, pin_memory=True),
+                 torch.empty((h_q, k), dtype=torch.float32, pin_memory=True)) for _ in range(S)]
+    inner = make_step(q_dev)
 
     def e2e_step():
         q_dev.copy_(q_host, non_blocking=True)
-        F.allocate(q_dev, sigma, B, out=alloc)
-        F.scan_topk(planes, qmin, qscale, q_dev, alloc, k, n, workspace=ws, out=out)
-        idx_host.copy_(out[0], non_blocking=True)
-        sc_host.copy_(out[1], non_blocking=True)
+        inner()
+        for (hi, hs), (di, ds) in zip(out_host, outs):
+            hi.copy_(di, non_blocking=True)
+            hs.copy_(ds, non_blocking=True)
 
+    eb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     for _ in range(3):
         flush.zero_()
         e2e_step()
@@ -356,26 +471,24 @@ def run_native(args):
         e2e_step()
         ee[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = reduce_max(float(np.mean([a.elapsed_time(b) for a, b in zip(eb, ee)])), world,
-                        device)
+    e2e_ms_local = float(np.mean([a.elapsed_time(b) for a, b in zip(eb, ee)]))
+    e2e_value, e2e_ms = job_throughput(keys_per_step, e2e_ms_local, world, device)
     h2d = q_host.numel() * q_host.element_size()
-    d2h = idx_host.numel() * 4 + sc_host.numel() * 4
-
-    keys_per_step = h_q * n * world
-    value = keys_per_step / (t_step * 1e-3) / 1e9
-    e2e_value = keys_per_step / (e2e_ms * 1e-3) / 1e9
+    d2h = S * h_q * k * 8
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not ragged:
         import oracle
         oracle.build()
-        cn = (case.codes.cpu().numpy(), qmin.cpu().numpy(), qscale.cpu().numpy(),
-              case.q.cpu().numpy().astype(np.float64), sigma.cpu().numpy())
+        c = cases[0]
+        c.codes = synthkv.make_case(cfg["seed"], cfg["n"], h_kv, h_q, d, cfg["q_dtype"],
+                                    device=device, keep_keys=False).codes
+        cn = case_numpy(c)
         heads = list(range(8))
         secs = oracle_sample(cn, B, k, heads)
-        cpu = {"value": len(heads) * n / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+        cpu = {"value": len(heads) * c.n / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "query heads 0-7 (KV heads 0-1) of this step: allocation, fp64 scores "
-                         "of all %d keys, brute-force top-%d; single thread, %.1f s" % (n, k, secs)}
+                         "of all %d keys, brute-force top-%d; single thread, %.1f s" % (c.n, k, secs)}
 
     if rank == 0:
         res = {
@@ -384,18 +497,19 @@ def run_native(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded, synthkv: Qwen3-8B-shaped GQA keys with outlier "
                     "channels, 4-bit min-max codes)",
-            "config": {"workload": workload_desc(cfg, B, k), "n": n, "h_kv": h_kv, "h_q": h_q,
-                       "d": d, "budget_bits": B, "k": k, "per_rank_sessions": 1,
+            "config": {"workload": workload_desc(cfg, B, k), "sessions_per_rank": S,
+                       "keys_per_rank": n_total, "h_kv": h_kv, "h_q": h_q, "d": d,
+                       "budget_bits": B, "k": k, "scan_kernel": "tcgen05" if flags else "cuda-core",
                        "l2": "flushed between steps (256 MiB write, outside the events)"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
-                         "peak_kind": peak_kind, "kernel": "scan_kernel<4,1> (filtering scan)",
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind, "kernel": "filtering scan",
                          "kernel_ms": t_kern, "algorithmic_bytes": alg_bytes,
                          "union_planes": int(rep.union_planes)},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 6 * K,
-            "tokens_per_s": n * world / (t_step * 1e-3),
+            "gpu_launches": LAUNCHES_PER_STEP * K,
+            "tokens_per_s": n_total * world / (t_step * 1e-3),
             "fallback_heads": int(rep.fallback_heads),
             "max_candidates": int(rep.max_candidates),
             "clocks": clocks,

@@ -14,6 +14,7 @@ cudaError_t launch_pack(const uint8_t *codes, int64_t n, int d, int h_kv, uint32
 cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
                             int budget, uint8_t *alloc, cudaStream_t stream);
 cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream);
+int tc_plan_bytes(int d);
 }  // namespace fathom
 
 using namespace fathom;
@@ -106,7 +107,9 @@ WsLayout ws_layout(int S, int64_t n_max, int d, int h_q, int h_kv, int k, uint32
   o = up256(o + 4 * heads);
   L.zero_bytes = o;
   L.off_plans = o;
-  o = up256(o + (size_t)groups * plan_layout(d).bytes);
+  const size_t plan_bytes = (size_t)(tc_plan_bytes(d) > plan_layout(d).bytes ? tc_plan_bytes(d)
+                                                                              : plan_layout(d).bytes);
+  o = up256(o + (size_t)groups * plan_bytes);
   L.off_sample = o;
   o = up256(o + (size_t)heads * L.m_max * 4);
   L.off_cand = o;

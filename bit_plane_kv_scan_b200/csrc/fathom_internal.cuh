@@ -10,9 +10,10 @@
 namespace fathom {
 
 // ---------------------------------------------------------------- geometry --
-// A scan tile is 4096 tokens of one (session, KV head): 128 plane words per
-// plane row, one word (32 tokens) per thread of a 128-thread block.
-constexpr int kTileWords = 128;
+// A scan tile is 2048 tokens of one (session, KV head): 64 plane words per
+// plane row.  A 128-thread block gives every word two threads, 16 tokens each
+// (warps 2w and 2w+1 share the words 32w .. 32w+31).
+constexpr int kTileWords = 64;
 constexpr int kTileTokens = kTileWords * 32;
 constexpr int kScanThreads = 128;
 // Plane rows staged in shared memory per pipeline stage, and the stage width
@@ -21,14 +22,16 @@ constexpr int kScanThreads = 128;
 // it, so a stage never holds more than 32 rows).
 constexpr int kStageRows = 32;
 constexpr int kStageSpan = 29;
-constexpr int kStageBytes = kStageRows * kTileWords * 4;  // 16 KiB
+constexpr int kStageBytes = kStageRows * kTileWords * 4;  // 8 KiB
 constexpr int kNumBuf = 3;                                  // stage buffers in flight
 constexpr int kNumPlanSlots = 4;                            // resident KV-head plans
 // Threshold sampling: one 256-token sector (8 words) in every 64.
 constexpr int kSectorWords = 8;
 constexpr int kSampleStride = 64;
-constexpr int kSampleSectorsPerTile = kTileWords / kSectorWords;  // 16
+constexpr int kSampleSectorsPerTile = kTileWords / kSectorWords;  // 8
 constexpr int kMergeThreads = 1024;
+constexpr int64_t kThresholdSmemKeys = 40960;  // sampled keys staged in shared memory (160 KiB)
+constexpr int64_t kMergeSmemCand = 12288;      // candidates staged in shared memory (96 KiB)
 constexpr int kFallbackSlack = 2048;
 
 enum ScanMode { kModeSample = 0, kModeFilter = 1 };
@@ -51,13 +54,13 @@ static_assert(sizeof(WsStatus) == 256, "status block is 256 bytes");
 //   info   = c | t* << 8 | slot0 << 11 | nfeat << 16 (slot0: first staged row);
 //   feat   = up to 4 bytes, each (tf | mask << 3): the query heads in `mask`
 //            read the first tf planes of this channel;
-//   W      = per query head 16 q_c s_c (0 where that head reads nothing).
+//   W      = per query head 32 q_c s_c (0 where that head reads nothing).
 struct PlanHeader {
   int nent;
   int nstage;
   int union_planes;
   int pad0;
-  float K[4];    // per query head constant: C_h - sum of its W over channels it reads
+  float K[4];    // per query head constant: C_h - sum of W/2 over the channels it reads
   float tau[4];  // per query head candidate threshold (filled when a scan block loads it)
   int pad1[4];
 };

@@ -13,27 +13,29 @@
 //    prefix lengths ("features") with the heads that use each.  Per head the
 //    score is rewritten as
 //        s_h(i) = K_h + sum_{c: t_c > 0} W_c * x_{t_c}(i, c),
-//        W_c = 16 q_c s_c,  x_t = 1 + y_t / 16,
+//        W_c = 32 q_c s_c,  x_t = 1/2 + y_t / 32,
 //    y_t the code's top t bits left-aligned in 4 bits (y_t = 2^(4-t) v_t),
-//    K_h = sum_c q_c (m_c + s_c (2^(4-t_c) - 1) / 2) - sum_{c: t_c > 0} W_c.
-//    x_t is built exactly as an fp32 bit pattern (exponent 0, y_t in the
-//    top four fraction bits), so one byte permute and one FMA per
-//    (token, channel, feature) replace t_c conditional adds per head.
-//  * scan_kernel, persistent blocks of 128 threads over 4096-token tiles:
+//    K_h = sum_c q_c (m_c + s_c (2^(4-t_c) - 1) / 2) - sum_{c: t_c > 0} W_c / 2.
+//    x_t is an exact fp32 bit pattern (exponent -1, y_t in the top four
+//    fraction bits), so one byte permute per (token, channel, feature) and
+//    one packed FMA per (token pair, head) replace t_c conditional adds.
+//  * scan_kernel, persistent blocks of 128 threads over 2048-token tiles:
 //    the union plane rows of a tile are staged into shared memory with
-//    16-byte cp.async copies, three stages in flight; each thread owns one
-//    plane word (32 tokens) and keeps its 32 x G scores in registers
-//    (packed fp32x2 FMAs); it writes the tokens whose score clears the
-//    head's sampled threshold as (score, index) candidates.
-//  * A sample pass of the same kernel scores one 256-token sector in 64
-//    and threshold_kernel takes the r-th largest sampled score per head as
-//    that threshold (expected ~2k candidates per head, no dense score write).
+//    16-byte cp.async copies, three stages in flight; two threads share a
+//    plane word and each keeps 16 tokens x G heads of scores in registers
+//    (fp32x2 FMAs); the filtering pass writes the tokens whose score clears
+//    the head's sampled threshold as (score, index) candidates.
+//  * A sample pass of the same kernel scores one 256-token sector in 64 and
+//    threshold_kernel takes the r-th largest sampled score per head as that
+//    threshold (expected ~2k candidates per head, no dense score write).
 //  * merge_kernel, one block per head: exact radix select of the k-th
 //    largest (score, -index) composite among the candidates, then a sort.
 //    When a threshold turns out invalid (fewer than k candidates, or more
 //    than the buffer holds) the block recomputes that head exactly with a
 //    streaming single-block scan.
 #include <float.h>
+
+#include <type_traits>
 
 #include "fathom_internal.cuh"
 
@@ -58,7 +60,15 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ uint32_t rotr(uint32_t x, int s) { return __funnelshift_r(x, x, s); }
+// x shifted right by S (S > 0) or left by -S.  Right shifts are written as
+// the high half of a multiply and left shifts as a multiply, so that they
+// may issue on the FMA pipe rather than the busier integer ALU pipe.
+// Call sites pass compile-time shifts (unrolled loops), so the branches fold.
+__device__ __forceinline__ uint32_t shift_by(uint32_t x, int s) {
+  if (s > 0) return __umulhi(x, 1u << (32 - s));
+  if (s < 0) return x * (1u << (-s));
+  return x;
+}
 
 // Block-wide inclusive scan of one int per thread (blockDim.x <= 1024).
 __device__ int block_inclusive_scan(int v, int *s_tmp) {
@@ -84,6 +94,14 @@ __device__ int block_inclusive_scan(int v, int *s_tmp) {
   if (warp > 0) v += s_tmp[warp - 1];
   __syncthreads();
   return v;
+}
+
+// Adds one to hist[digit] for every lane with digit >= 0, one shared-memory
+// atomic per distinct digit in the warp.  All 32 lanes must call it.
+__device__ __forceinline__ void hist_add_warp(unsigned *hist, int digit) {
+  const unsigned peers = __match_any_sync(0xffffffffu, digit);
+  if (digit >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1)
+    atomicAdd(&hist[digit], (unsigned)__popc(peers));
 }
 
 // ------------------------------------------------------------ plan kernel --
@@ -123,9 +141,10 @@ __global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
       t[hh] = se.alloc[hq];
       const float qv = load_q(se.q, p.q_bf16, hq);
       tstar = max(tstar, t[hh]);
-      W[hh] = t[hh] > 0 ? (qv * sc) * 16.0f : 0.0f;
+      W[hh] = t[hh] > 0 ? (qv * sc) * 32.0f : 0.0f;
       const double cell = (double)(1 << (4 - t[hh]));
-      kpart[hh] = (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5)) - (double)W[hh];
+      kpart[hh] =
+          (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5)) - 0.5 * (double)W[hh];
     }
     for (int tf = 1; tf <= 4; ++tf) {
       uint32_t mask = 0;
@@ -147,8 +166,8 @@ __global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
   // entry index and first plane of every channel with t* > 0
   const int packed = (tstar > 0 ? 1 : 0) | (tstar << 12);
   const int incl = block_inclusive_scan(packed, s_tmp);
-  const int e = (incl & 0xfff) - 1;            // entry index if tstar > 0
-  const int p_incl = incl >> 12;               // planes up to and including c
+  const int e = (incl & 0xfff) - 1;  // entry index if tstar > 0
+  const int p_incl = incl >> 12;     // planes up to and including c
   const int p_excl = p_incl - tstar;
   if (threadIdx.x == blockDim.x - 1) {
     s_total[0] = incl & 0xfff;  // entries
@@ -201,16 +220,16 @@ __global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
 // ------------------------------------------------------------ scan kernel --
 
 struct TileLoc {
-  int s, g, ti;     // session, KV head, tile within (session, KV head)
-  int64_t n, W;     // session keys and plane words
+  int s, g, ti;  // session, KV head, tile within (session, KV head)
+  int64_t n, W;  // session keys and plane words
   const uint32_t *planes;
 };
 
 struct Item {
-  int t;      // tile index in the launch's tile space (-1 = none)
-  int st;     // stage within the tile
-  int slot;   // plan slot in shared memory
-  int nst;    // stages of this tile
+  int t;     // tile index in the launch's tile space (-1 = none)
+  int st;    // stage within the tile
+  int slot;  // plan slot in shared memory
+  int nst;   // stages of this tile
 };
 
 template <int MODE>
@@ -238,11 +257,79 @@ __device__ __forceinline__ TileLoc locate(const ScanParams &p, const int *s_tpre
   return L;
 }
 
+// One channel of the plan for this thread's 16 tokens (bit positions
+// 8 kk + r of its word, r = HALF .. HALF + 3).
+//  R[i], byte kk = y << 3 for token 8 kk + HALF + i, y = the union prefix
+//  code left-aligned in 4 bits (plane j lands on bit 6 - j).
+//  Each feature masks R to its prefix length, turns every byte into the
+//  fp32 x = 1/2 + y/32 with one byte permute ([0x3f][byte][0][0]), and adds
+//  W_h x to the scores of the heads that read it.
+template <int G, int HALF>
+__device__ __forceinline__ void scan_entry(const uint32_t *src, int tstar, int nfeat, uint32_t fb,
+                                           const float4 w4, float2 (&acc)[G][4][2]) {
+  uint32_t R[4];
+  const uint32_t p0 = src[0];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) R[i] = shift_by(p0, HALF + i - 6) & 0x40404040u;
+  if (tstar > 1) {
+    const uint32_t p1 = src[kTileWords];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) R[i] |= shift_by(p1, HALF + i - 5) & 0x20202020u;
+    if (tstar > 2) {
+      const uint32_t p2 = src[2 * kTileWords];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) R[i] |= shift_by(p2, HALF + i - 4) & 0x10101010u;
+      if (tstar > 3) {
+        const uint32_t p3 = src[3 * kTileWords];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) R[i] |= shift_by(p3, HALF + i - 3) & 0x08080808u;
+      }
+    }
+  }
+  const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+  for (int f = 0; f < nfeat; ++f) {
+    const uint32_t byte = (fb >> (8 * f)) & 0xffu;
+    const int tf = byte & 7;
+    const uint32_t mask = byte >> 3;
+    uint32_t Rf[4];
+    if (tf == tstar) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Rf[i] = R[i];
+    } else {
+      // keep planes j < tf: bits 6 .. 7 - tf of every byte
+      const uint32_t keep = (((1u << tf) - 1u) << (7 - tf)) * 0x01010101u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) Rf[i] = R[i] & keep;
+    }
+    float2 xx[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp)
+        xx[i][pp] = make_float2(
+            __uint_as_float(__byte_perm(Rf[i], 0x3f000000u, 0x7054u | ((2 * pp) << 8))),
+            __uint_as_float(__byte_perm(Rf[i], 0x3f000000u, 0x7054u | ((2 * pp + 1) << 8))));
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      if (mask & (1u << h)) {
+        const float2 ww = make_float2(wv[h], wv[h]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) acc[h][i][pp] = __ffma2_rn(xx[i][pp], ww, acc[h][i][pp]);
+      }
+    }
+  }
+}
+
 template <int G, int MODE>
-__global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
+__global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int half = warp & 1;                 // which 16 tokens of the word
+  const int word = (warp >> 1) * 32 + lane;  // word of the tile this thread reads
   const PlanLayout PL = plan_layout(p.d);
   uint32_t *sbuf = reinterpret_cast<uint32_t *>(smem);
   unsigned char *splans = smem + kNumBuf * kStageBytes;
@@ -327,37 +414,53 @@ __global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
   };
 
   // ---- staged copies of one item's plane rows -----------------------------
+  constexpr int kChunks = kTileWords / 4;  // 16-byte copies per staged row
   auto issue = [&](const Item &it, int buf) {
     if (it.t < 0) return;
     const TileLoc L = locate<MODE>(p, s_tprefix, it.t);
     const unsigned char *plan = splans + it.slot * PL.bytes;
     const int nrows = plan[PL.off_stage_nrows + it.st];
-    const uint16_t *rows = reinterpret_cast<const uint16_t *>(plan + PL.off_stage_rows) +
-                           it.st * kStageRows;
+    const uint16_t *rows =
+        reinterpret_cast<const uint16_t *>(plan + PL.off_stage_rows) + it.st * kStageRows;
     uint32_t *dst_base = sbuf + buf * (kStageBytes / 4);
     const uint32_t *gbase = L.planes + (int64_t)L.g * p.d * 4 * L.W;
-    for (int id = tid; id < nrows * 32; id += kScanThreads) {
-      const int slot = id >> 5, q = id & 31;
+    for (int id = tid; id < nrows * kChunks; id += kScanThreads) {
+      const int slot = id / kChunks, q = id % kChunks;
       const uint32_t *row = gbase + (int64_t)rows[slot] * L.W;
-      int64_t word;
+      int64_t gw;
       bool ok;
       if (MODE == kModeSample) {
         const int64_t sj = (int64_t)L.ti * kSampleSectorsPerTile + (q >> 1);
-        word = sj * kSampleStride * kSectorWords + (q & 1) * 4;
-        ok = sj < sampled_sectors(L.n) && word < L.W;
+        gw = sj * kSampleStride * kSectorWords + (q & 1) * 4;
+        ok = sj < sampled_sectors(L.n) && gw < L.W;
       } else {
-        word = (int64_t)L.ti * kTileWords + q * 4;
-        ok = word < L.W;
+        gw = (int64_t)L.ti * kTileWords + q * 4;
+        ok = gw < L.W;
       }
-      cp_async16(dst_base + slot * kTileWords + q * 4, ok ? (const void *)(row + word) : (const void *)row,
-                 ok ? 16u : 0u);
+      cp_async16(dst_base + slot * kTileWords + q * 4,
+                 ok ? (const void *)(row + gw) : (const void *)row, ok ? 16u : 0u);
     }
   };
 
-  // ---- per-thread scores: 32 tokens x G heads -----------------------------
-  // acc[h][r][p]: .x is byte 2p, .y byte 2p+1 of build register r, i.e.
-  // tokens 32 w + 8 (2p) + r and 32 w + 8 (2p + 1) + r of this thread's word w.
-  float2 acc[G][8][2];
+  // ---- per-thread scores: 16 tokens x G heads -----------------------------
+  // acc[h][i][pp]: .x is byte 2pp and .y byte 2pp+1 of register i, i.e. the
+  // tokens at bits 8 (2pp) + 4 half + i and 8 (2pp + 1) + 4 half + i of the word.
+  float2 acc[G][4][2];
+
+  auto stage_entries = [&](const unsigned char *plan, const uint32_t *sb, int e0, int e1,
+                           auto half_tag) {
+    constexpr int HALF = decltype(half_tag)::value;
+    const uint32_t *info = reinterpret_cast<const uint32_t *>(plan + PL.off_info);
+    const uint32_t *feats = reinterpret_cast<const uint32_t *>(plan + PL.off_feat);
+    const float4 *wts = reinterpret_cast<const float4 *>(plan + PL.off_w);
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t inf = info[e];
+      const int tstar = (inf >> 8) & 7;
+      const int slot0 = (inf >> 11) & 31;
+      const int nfeat = (inf >> 16) & 7;
+      scan_entry<G, HALF>(sb + slot0 * kTileWords, tstar, nfeat, feats[e], wts[e], acc);
+    }
+  };
 
   auto compute = [&](const Item &it, int buf) {
     const unsigned char *plan = splans + it.slot * PL.bytes;
@@ -367,97 +470,24 @@ __global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
       for (int h = 0; h < G; ++h) {
         const float k0 = hdr->K[h];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          acc[h][r][0] = make_float2(k0, k0);
-          acc[h][r][1] = make_float2(k0, k0);
+        for (int i = 0; i < 4; ++i) {
+          acc[h][i][0] = make_float2(k0, k0);
+          acc[h][i][1] = make_float2(k0, k0);
         }
       }
     }
     const uint16_t *stage_begin = reinterpret_cast<const uint16_t *>(plan + PL.off_stage_begin);
-    const uint32_t *info = reinterpret_cast<const uint32_t *>(plan + PL.off_info);
-    const uint32_t *feats = reinterpret_cast<const uint32_t *>(plan + PL.off_feat);
-    const float4 *wts = reinterpret_cast<const float4 *>(plan + PL.off_w);
-    const uint32_t *sb = sbuf + buf * (kStageBytes / 4) + tid;
+    const uint32_t *sb = sbuf + buf * (kStageBytes / 4) + word;
     const int e0 = stage_begin[it.st], e1 = stage_begin[it.st + 1];
-    for (int e = e0; e < e1; ++e) {
-      const uint32_t inf = info[e];
-      const int tstar = (inf >> 8) & 7;
-      const int slot0 = (inf >> 11) & 31;
-      const int nfeat = (inf >> 16) & 7;
-      const uint32_t *src = sb + slot0 * kTileWords;
-      // Build 8 registers of 4 tokens each: byte kk of R[r] is
-      // 0x80 | y << 3 for token 8 kk + r of the word, y = union prefix code
-      // left-aligned in 4 bits (plane j lands on bit 6 - j).
-      uint32_t R[8];
-      const uint32_t p0 = src[0];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) R[r] = (rotr(p0, (r - 6) & 31) & 0x40404040u) | 0x80808080u;
-      if (tstar > 1) {
-        const uint32_t p1 = src[kTileWords];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) R[r] |= rotr(p1, (r - 5) & 31) & 0x20202020u;
-        if (tstar > 2) {
-          const uint32_t p2 = src[2 * kTileWords];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) R[r] |= rotr(p2, (r - 4) & 31) & 0x10101010u;
-          if (tstar > 3) {
-            const uint32_t p3 = src[3 * kTileWords];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) R[r] |= rotr(p3, (r - 3) & 31) & 0x08080808u;
-          }
-        }
-      }
-      const float4 w4 = wts[e];
-      const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-      const uint32_t fb = feats[e];
-      for (int f = 0; f < nfeat; ++f) {
-        const uint32_t byte = (fb >> (8 * f)) & 0xffu;
-        const int tf = byte & 7;
-        const uint32_t mask = byte >> 3;
-        // keep the first tf planes: byte mask 0xff << (7 - tf)
-        const uint32_t keep = (0xffu << (7 - tf)) & 0xffu;
-        const uint32_t km = keep * 0x01010101u;
-        uint32_t Rf[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) Rf[r] = R[r] & km;
-        float2 wpair[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) wpair[h] = make_float2(wv[h], wv[h]);
-        // x = 1 + y/16 as fp32: [0x3f][byte][0][0]
-#define FATHOM_APPLY(MASKV)                                                            \
-  {                                                                                    \
-    _Pragma("unroll") for (int r = 0; r < 8; ++r) {                                    \
-      _Pragma("unroll") for (int pp = 0; pp < 2; ++pp) {                               \
-        const float x0 = __uint_as_float(__byte_perm(Rf[r], 0x3f000000u, 0x7054u | ((2 * pp) << 8)));     \
-        const float x1 = __uint_as_float(__byte_perm(Rf[r], 0x3f000000u, 0x7054u | ((2 * pp + 1) << 8))); \
-        const float2 xx = make_float2(x0, x1);                                         \
-        _Pragma("unroll") for (int h = 0; h < G; ++h) {                                \
-          if ((MASKV) & (1u << h)) acc[h][r][pp] = __ffma2_rn(xx, wpair[h], acc[h][r][pp]); \
-        }                                                                              \
-      }                                                                                \
-    }                                                                                  \
-  }
-        switch (mask) {
-          case 1: FATHOM_APPLY(1u) break;
-          case 2: if (G > 1) FATHOM_APPLY(2u) break;
-          case 3: if (G > 1) FATHOM_APPLY(3u) break;
-          case 4: if (G > 2) FATHOM_APPLY(4u) break;
-          case 5: if (G > 2) FATHOM_APPLY(5u) break;
-          case 6: if (G > 2) FATHOM_APPLY(6u) break;
-          case 7: if (G > 2) FATHOM_APPLY(7u) break;
-          case 8: if (G > 3) FATHOM_APPLY(8u) break;
-          case 9: if (G > 3) FATHOM_APPLY(9u) break;
-          case 10: if (G > 3) FATHOM_APPLY(10u) break;
-          case 11: if (G > 3) FATHOM_APPLY(11u) break;
-          case 12: if (G > 3) FATHOM_APPLY(12u) break;
-          case 13: if (G > 3) FATHOM_APPLY(13u) break;
-          case 14: if (G > 3) FATHOM_APPLY(14u) break;
-          case 15: if (G > 3) FATHOM_APPLY(15u) break;
-          default: break;
-        }
-#undef FATHOM_APPLY
-      }
-    }
+    // the half is fixed per warp: one branch per stage, not per entry
+    if (half)
+      stage_entries(plan, sb, e0, e1, std::integral_constant<int, 4>{});
+    else
+      stage_entries(plan, sb, e0, e1, std::integral_constant<int, 0>{});
+  };
+
+  auto score_of = [&](int h, int i, int kk) -> float {
+    return (kk & 1) ? acc[h][i][kk >> 1].y : acc[h][i][kk >> 1].x;
   };
 
   // ---- results of a finished tile -------------------------------------------
@@ -465,36 +495,35 @@ __global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
     const TileLoc L = locate<MODE>(p, s_tprefix, it.t);
     const PlanHeader *hdr = reinterpret_cast<const PlanHeader *>(splans + it.slot * PL.bytes);
     const int64_t head0 = (int64_t)L.s * p.h_q + L.g * G;
+    const int r0 = 4 * half;
     if (MODE == kModeSample) {
-      const int64_t sj = (int64_t)L.ti * kSampleSectorsPerTile + (tid >> 3);
+      const int64_t sj = (int64_t)L.ti * kSampleSectorsPerTile + (word >> 3);
       if (sj >= sampled_sectors(L.n)) return;
-      const int64_t tok0 = (sj * kSampleStride * kSectorWords + (tid & 7)) * 32;
-      const int64_t slot0 = sj * 256 + (tid & 7) * 32;
+      const int64_t tok0 = (sj * kSampleStride * kSectorWords + (word & 7)) * 32;
+      const int64_t slot0 = sj * 256 + (word & 7) * 32;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         uint32_t *dst = p.sample + (head0 + h) * p.m_max + slot0;
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const int b = 8 * kk + r;
-            const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
-            dst[b] = (tok0 + b < L.n) ? float_key(sc) : 0u;
+            const int b = 8 * kk + r0 + i;
+            dst[b] = (tok0 + b < L.n) ? float_key(score_of(h, i, kk)) : 0u;
           }
       }
       return;
     }
-    const int64_t tok0 = ((int64_t)L.ti * kTileWords + tid) * 32;
+    const int64_t tok0 = ((int64_t)L.ti * kTileWords + word) * 32;
     if (p.debug_scores) {
 #pragma unroll
       for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const int64_t tok = tok0 + 8 * kk + r;
-            const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
-            if (tok < L.n) p.debug_scores[(head0 + h) * L.n + tok] = sc;
+            const int64_t tok = tok0 + 8 * kk + r0 + i;
+            if (tok < L.n) p.debug_scores[(head0 + h) * L.n + tok] = score_of(h, i, kk);
           }
     }
 #pragma unroll
@@ -502,12 +531,11 @@ __global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
       const float tau = hdr->tau[h];
       uint32_t m = 0;
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const int b = 8 * kk + r;
-          const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
-          m |= ((tok0 + b < L.n) && (sc >= tau) ? 1u : 0u) << b;
+          const int b = 8 * kk + r0 + i;
+          m |= ((tok0 + b < L.n) && (score_of(h, i, kk) >= tau) ? 1u : 0u) << (4 * kk + i);
         }
       const int cnt = __popc(m);
       if (__any_sync(0xffffffffu, cnt != 0)) {
@@ -524,13 +552,12 @@ __global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
           int64_t pos = (int64_t)base + (incl - cnt);
           unsigned long long *dst = p.cand + (head0 + h) * p.cap;
 #pragma unroll
-          for (int r = 0; r < 8; ++r)
+          for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const int b = 8 * kk + r;
-              if ((m >> b) & 1u) {
-                const float sc = (kk & 1) ? acc[h][r][kk >> 1].y : acc[h][r][kk >> 1].x;
-                if (pos < p.cap) dst[pos] = composite(sc, (uint32_t)(tok0 + b));
+              if ((m >> (4 * kk + i)) & 1u) {
+                if (pos < p.cap)
+                  dst[pos] = composite(score_of(h, i, kk), (uint32_t)(tok0 + 8 * kk + r0 + i));
                 ++pos;
               }
             }
@@ -568,7 +595,7 @@ __global__ void __launch_bounds__(kScanThreads, 3) scan_kernel(ScanParams p) {
 // ------------------------------------------------------- threshold kernel --
 
 // Warp 0 finds the digit bin holding the want-th largest among 256 bins
-// (counted from the top); returns (digit, count above it).
+// (counted from the top) and the count above it.
 __device__ __forceinline__ void find_bin_from_top(const unsigned *hist, unsigned want, int *s_digit,
                                                   unsigned *s_above) {
   const int lane = threadIdx.x & 31;
@@ -601,7 +628,8 @@ __device__ __forceinline__ void find_bin_from_top(const unsigned *hist, unsigned
   }
 }
 
-__global__ void __launch_bounds__(256) threshold_kernel(ScanParams p) {
+__global__ void __launch_bounds__(512) threshold_kernel(ScanParams p, int smem_keys) {
+  extern __shared__ uint32_t s_keys[];  // [smem_keys]
   const int64_t h = blockIdx.x;
   const int s = (int)(h / p.h_q);
   const int64_t n = session_of(p, s).n;
@@ -614,15 +642,27 @@ __global__ void __launch_bounds__(256) threshold_kernel(ScanParams p) {
   }
   const int64_t m = sampled_sectors(n) * 256;
   const uint32_t *keys = p.sample + h * p.m_max;
+  // the radix passes re-read every key; stage them in shared memory when
+  // they fit (one pass of independent loads instead of four dependent ones)
+  if (m <= smem_keys) {
+    for (int64_t i = threadIdx.x; i < m; i += blockDim.x) s_keys[i] = keys[i];
+    __syncthreads();
+    keys = s_keys;
+  }
   uint32_t prefix = 0, pmask = 0;
   unsigned want = (unsigned)p.sample_rank;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    hist[threadIdx.x] = 0;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     if (threadIdx.x == 0) s_digit = -1;
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < m; i += blockDim.x) {
-      const uint32_t k = keys[i];
-      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    for (int64_t base = 0; base < m; base += blockDim.x) {
+      const int64_t i = base + threadIdx.x;
+      int digit = -1;
+      if (i < m) {
+        const uint32_t k = keys[i];
+        if ((k & pmask) == prefix) digit = (int)((k >> shift) & 255u);
+      }
+      hist_add_warp(hist, digit);
     }
     __syncthreads();
     find_bin_from_top(hist, want, &s_digit, &s_above);
@@ -650,9 +690,14 @@ __device__ unsigned long long block_kth(const unsigned long long *a, int64_t cnt
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     if (threadIdx.x == 0) *s_digit = -1;
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
-      const unsigned long long v = a[i];
-      if ((v & pmask) == prefix) atomicAdd(&hist[(unsigned)(v >> shift) & 255u], 1u);
+    for (int64_t base = 0; base < cnt; base += blockDim.x) {
+      const int64_t i = base + threadIdx.x;
+      int digit = -1;
+      if (i < cnt) {
+        const unsigned long long v = a[i];
+        if ((v & pmask) == prefix) digit = (int)((unsigned)(v >> shift) & 255u);
+      }
+      hist_add_warp(hist, digit);
     }
     __syncthreads();
     find_bin_from_top(hist, want, s_digit, s_above);
@@ -681,6 +726,7 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   __shared__ uint8_t s_t[FATHOM_MAX_D];
   __shared__ double s_kc[32];
   __shared__ unsigned long long s_nbuf;
+  __shared__ unsigned s_fill;
   double kc = 0.0;
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     const int t = se.alloc[(int64_t)hl * d + c];
@@ -721,7 +767,6 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
     const int64_t nb = (int64_t)s_nbuf;
     if (nb > p.cap - (int64_t)blockDim.x) {
       theta = block_kth(buf, nb, k, hist, s_digit, s_above);
-      __shared__ unsigned s_fill;
       if (threadIdx.x == 0) s_fill = 0;
       __syncthreads();
       for (int64_t j = threadIdx.x; j < nb; j += blockDim.x)
@@ -741,8 +786,9 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   return (int64_t)s_nbuf;
 }
 
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int kpow2) {
-  extern __shared__ unsigned long long s_sort[];  // [kpow2]
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int kpow2,
+                                                              int smem_cand) {
+  extern __shared__ unsigned long long s_sort[];  // [kpow2], then [smem_cand] staged candidates
   __shared__ unsigned hist[256];
   __shared__ int s_digit;
   __shared__ unsigned s_above;
@@ -757,12 +803,22 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
   int64_t cnt = p.counts[h];
   const uint32_t tauk = p.tau[h];
   const int64_t need = n < k ? n : k;
-  const bool ok = cnt <= p.cap && (tauk == 0u || cnt >= need) && !(p.flags & FATHOM_FLAG_FORCE_FALLBACK);
+  const bool ok = cnt <= p.cap && (tauk == 0u || cnt >= need) &&
+                  !(p.flags & FATHOM_FLAG_FORCE_FALLBACK);
   if (!ok) {
     cnt = fallback_head(p, s, hl, buf, s_sort, hist, &s_digit, &s_above);
     if (threadIdx.x == 0) atomicAdd(&p.status->fallback_heads, 1u);
   }
-  if (threadIdx.x == 0) atomicMax(&p.status->max_candidates, (unsigned)(cnt < 0xffffffffll ? cnt : 0xffffffffll));
+  if (threadIdx.x == 0)
+    atomicMax(&p.status->max_candidates, (unsigned)(cnt < 0xffffffffll ? cnt : 0xffffffffll));
+  // the radix passes re-read every candidate; stage them in shared memory
+  // when they fit
+  if (cnt <= smem_cand) {
+    unsigned long long *staged = s_sort + kpow2;
+    for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) staged[i] = buf[i];
+    __syncthreads();
+    buf = staged;
+  }
   const int take = (int)(cnt < k ? cnt : k);
   unsigned long long bar = 0ull;
   if (cnt > k) bar = block_kth(buf, cnt, (unsigned)k, hist, &s_digit, &s_above);
@@ -855,16 +911,30 @@ static cudaError_t launch_scan_m(const ScanParams &p, cudaStream_t stream) {
   }
 }
 
+cudaError_t launch_tc_plan(const ScanParams &p, cudaStream_t stream);
+cudaError_t launch_tc_scan(const ScanParams &p, int mode, int sms, cudaStream_t stream);
+
 cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream) {
   const int heads = p.S * p.h_q;
-  const int groups = p.S * p.h_kv;
-  plan_kernel<<<groups, 256, 0, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  int sms = 0;
+  cudaError_t e = num_sms(&sms);
+  if (e != cudaSuccess) return e;
+  const bool tc = (p.flags & FATHOM_FLAG_TENSOR_CORES) != 0;
+  if (tc) {
+    e = launch_tc_plan(p, stream);
+  } else {
+    plan_kernel<<<p.S * p.h_kv, 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   if (any_sampling) {
-    e = launch_scan_m<kModeSample>(p, stream);
+    e = tc ? launch_tc_scan(p, kModeSample, sms, stream) : launch_scan_m<kModeSample>(p, stream);
     if (e != cudaSuccess) return e;
-    threshold_kernel<<<heads, 256, 0, stream>>>(p);
+    const int64_t tkeys = p.m_max < kThresholdSmemKeys ? p.m_max : kThresholdSmemKeys;
+    const int tsmem = (int)(tkeys * 4);
+    e = cudaFuncSetAttribute(threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tsmem);
+    if (e != cudaSuccess) return e;
+    threshold_kernel<<<heads, 512, tsmem, stream>>>(p, (int)tkeys);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -872,7 +942,7 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
     e = cudaEventRecord(p.prof_begin, stream);
     if (e != cudaSuccess) return e;
   }
-  e = launch_scan_m<kModeFilter>(p, stream);
+  e = tc ? launch_tc_scan(p, kModeFilter, sms, stream) : launch_scan_m<kModeFilter>(p, stream);
   if (e != cudaSuccess) return e;
   if (p.prof_end) {
     e = cudaEventRecord(p.prof_end, stream);
@@ -880,10 +950,14 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
   }
   int kpow2 = 1;
   while (kpow2 < p.k) kpow2 <<= 1;
-  const int msmem = kpow2 * 8;
+  // room for about twice the expected candidate count (~2k per head)
+  int64_t mcand = 4 * (int64_t)p.k + 1024;
+  if (mcand > p.cap) mcand = p.cap;
+  if (mcand > kMergeSmemCand) mcand = kMergeSmemCand;
+  const int msmem = (int)((kpow2 + mcand) * 8);
   e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
   if (e != cudaSuccess) return e;
-  merge_kernel<<<heads, kMergeThreads, msmem, stream>>>(p, kpow2);
+  merge_kernel<<<heads, kMergeThreads, msmem, stream>>>(p, kpow2, (int)mcand);
   return cudaGetLastError();
 }
 

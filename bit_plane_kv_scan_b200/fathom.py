@@ -31,6 +31,7 @@ PLANES_DEVICE = 0
 PLANES_HOST_MAPPED = 1
 FLAG_NO_SAMPLING = 1
 FLAG_FORCE_FALLBACK = 2
+FLAG_TENSOR_CORES = 4
 
 EXPORTED = [
     "fathom_last_error", "fathom_plane_words", "fathom_planes_bytes", "fathom_pack_planes",
@@ -238,46 +239,66 @@ def scan_topk(planes: torch.Tensor, qmin: torch.Tensor, qscale: torch.Tensor, q:
     return out
 
 
+class BatchedScan:
+    """A prepared batched scan: the session descriptors are uploaded once, so
+    repeated launches over the same buffers (a decode loop whose q and alloc
+    are rewritten in place) issue no host-to-device copy of their own.  Each
+    session dict holds planes, qmin, qscale, q, alloc, n (and optionally
+    out_idx/out_score)."""
+
+    def __init__(self, sessions: Sequence[dict], k: int, d: int, h_q: int, h_kv: int,
+                 q_dtype: torch.dtype = torch.bfloat16, *, host_mapped: bool = False,
+                 flags: int = 0, device=None):
+        device = torch.device(device or sessions[0]["q"].device)
+        S = len(sessions)
+        arr = (Session * S)()
+        self.outs: List[Tuple[torch.Tensor, torch.Tensor]] = []
+        n_max = 0
+        for i, s in enumerate(sessions):
+            oi = s.get("out_idx")
+            osc = s.get("out_score")
+            if oi is None:
+                oi = torch.empty((h_q, k), dtype=torch.int32, device=device)
+                osc = torch.empty((h_q, k), dtype=torch.float32, device=device)
+            self.outs.append((oi, osc))
+            arr[i] = Session(planes=s["planes"].data_ptr(), qmin=s["qmin"].data_ptr(),
+                             qscale=s["qscale"].data_ptr(), q=s["q"].data_ptr(),
+                             alloc=s["alloc"].data_ptr(), n=int(s["n"]), out_idx=oi.data_ptr(),
+                             out_score=osc.data_ptr())
+            n_max = max(n_max, int(s["n"]))
+        raw = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+        self.device = device
+        self.desc = raw.to(device, non_blocking=False)
+        self.args = BatchedArgs(sessions=self.desc.data_ptr(), num_sessions=S, n_max=n_max, d=d,
+                                h_q=h_q, h_kv=h_kv, k=int(k),
+                                q_dtype=BF16 if q_dtype == torch.bfloat16 else F32,
+                                planes_location=PLANES_HOST_MAPPED if host_mapped
+                                else PLANES_DEVICE, flags=int(flags))
+        self.need = lib().fathom_scan_topk_batched_workspace_size(ctypes.byref(self.args))
+        if self.need == 0:
+            _check(lib().fathom_scan_topk_batched(ctypes.byref(self.args), None, 0, None))
+
+    def __call__(self, workspace: Optional[Workspace] = None, stream=None):
+        ws = _workspace(workspace, self.device)
+        buf = ws.get(self.need)
+        _check(lib().fathom_scan_topk_batched(ctypes.byref(self.args), _ptr(buf), self.need,
+                                              _stream(stream)))
+        # The descriptor tensor lives as long as this object; the workspace
+        # also holds it so a one-shot caller may drop the object at once
+        # (torch's caching allocator hands its block only to later work
+        # ordered after these launches on this stream).
+        ws.keepalive = self.desc
+        return self.outs
+
+
 def scan_topk_batched(sessions: Sequence[dict], k: int, d: int, h_q: int, h_kv: int,
                       q_dtype: torch.dtype = torch.bfloat16, *, host_mapped: bool = False,
                       flags: int = 0, workspace: Optional[Workspace] = None, stream=None,
                       device=None):
     """Many sessions in one launch set.  Each session dict holds planes, qmin, qscale, q,
     alloc, n (and optionally out_idx/out_score).  Returns a list of (idx, score)."""
-    device = torch.device(device or sessions[0]["q"].device)
-    S = len(sessions)
-    arr = (Session * S)()
-    outs: List[Tuple[torch.Tensor, torch.Tensor]] = []
-    n_max = 0
-    for i, s in enumerate(sessions):
-        oi = s.get("out_idx")
-        osc = s.get("out_score")
-        if oi is None:
-            oi = torch.empty((h_q, k), dtype=torch.int32, device=device)
-            osc = torch.empty((h_q, k), dtype=torch.float32, device=device)
-        outs.append((oi, osc))
-        arr[i] = Session(planes=s["planes"].data_ptr(), qmin=s["qmin"].data_ptr(),
-                         qscale=s["qscale"].data_ptr(), q=s["q"].data_ptr(),
-                         alloc=s["alloc"].data_ptr(), n=int(s["n"]), out_idx=oi.data_ptr(),
-                         out_score=osc.data_ptr())
-        n_max = max(n_max, int(s["n"]))
-    raw = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
-    dev_desc = raw.to(device, non_blocking=False)
-    args = BatchedArgs(sessions=dev_desc.data_ptr(), num_sessions=S, n_max=n_max, d=d, h_q=h_q,
-                       h_kv=h_kv, k=int(k), q_dtype=BF16 if q_dtype == torch.bfloat16 else F32,
-                       planes_location=PLANES_HOST_MAPPED if host_mapped else PLANES_DEVICE,
-                       flags=int(flags))
-    L = lib()
-    need = L.fathom_scan_topk_batched_workspace_size(ctypes.byref(args))
-    if need == 0:
-        _check(L.fathom_scan_topk_batched(ctypes.byref(args), None, 0, _stream(stream)))
-    ws = _workspace(workspace, device)
-    buf = ws.get(need)
-    _check(L.fathom_scan_topk_batched(ctypes.byref(args), _ptr(buf), need, _stream(stream)))
-    # The descriptor tensor may be freed now: torch's caching allocator only
-    # hands its block to later work ordered after these launches on this stream.
-    ws.keepalive = dev_desc
-    return outs
+    return BatchedScan(sessions, k, d, h_q, h_kv, q_dtype, host_mapped=host_mapped, flags=flags,
+                       device=device)(workspace, stream)
 
 
 def profile_scan_kernel(begin: Optional[torch.cuda.Event], end: Optional[torch.cuda.Event]):

@@ -75,6 +75,9 @@ typedef enum fathom_planes_location {
 /* Test knobs for fathom_scan_args.flags (0 in normal use). */
 #define FATHOM_FLAG_NO_SAMPLING 1u     /* skip the threshold sample: every key is a candidate */
 #define FATHOM_FLAG_FORCE_FALLBACK 2u  /* take the exact single-block fallback for every head */
+/* Run the scan on the tcgen05 tensor-core kernel (int8 MMA into tensor memory)
+ * instead of the CUDA-core kernel.  Same results; slower at the measured sizes. */
+#define FATHOM_FLAG_TENSOR_CORES 4u
 
 /* Last error message of the calling thread ("" if none). */
 FATHOM_API const char *fathom_last_error(void);

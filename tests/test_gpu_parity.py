@@ -227,10 +227,25 @@ def test_fallback_with_compaction():
                    "fallback head %d" % h)
 
 
+# ------------------------------------------------ tensor-core scan kernel --
+
+@pytest.mark.parametrize("n,G,B,k", [(4096, 1, 92, 64), (4097, 4, 92, 7), (12345, 2, 17, 100),
+                                     (40000, 4, 136, 64), (3000, 4, 0, 50), (3000, 4, 512, 50)])
+def test_tensor_core_scan(n, G, B, k):
+    """The tcgen05 (int8 MMA) form of the scan gives the oracle's answer."""
+    case = synthkv.make_case(seed=300 + n + G, n=n, h_kv=2, h_q=2 * G, d=128, q_dtype="bf16")
+    _full_check(case, B, k, flags=F.FLAG_TENSOR_CORES, what="tc n=%d G=%d B=%d" % (n, G, B))
+
+
+def test_tensor_core_scan_layer_131k(layer_131k):
+    _check_config(layer_131k, 92, 2048, heads_full={0, 13, 26, 31}, what="tc 131k",
+                  flags=F.FLAG_TENSOR_CORES)
+
+
 # ------------------------------------------------------ full-size configs --
 
-def _check_config(case, budget, k, heads_full, what, host_mapped=False):
-    _, alloc, (idx, sc) = run_gpu(case, budget, k, host_mapped=host_mapped)
+def _check_config(case, budget, k, heads_full, what, host_mapped=False, flags=0):
+    _, alloc, (idx, sc) = run_gpu(case, budget, k, host_mapped=host_mapped, flags=flags)
     cn = case_np(case)
     want_alloc = oracle.allocate_heads(cn[3], _np(case.sigma), budget)
     got_alloc = _np(alloc)
