@@ -35,8 +35,6 @@
 //    streaming single-block scan.
 #include <float.h>
 
-#include <type_traits>
-
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -447,21 +445,6 @@ __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
   // tokens at bits 8 (2pp) + 4 half + i and 8 (2pp + 1) + 4 half + i of the word.
   float2 acc[G][4][2];
 
-  auto stage_entries = [&](const unsigned char *plan, const uint32_t *sb, int e0, int e1,
-                           auto half_tag) {
-    constexpr int HALF = decltype(half_tag)::value;
-    const uint32_t *info = reinterpret_cast<const uint32_t *>(plan + PL.off_info);
-    const uint32_t *feats = reinterpret_cast<const uint32_t *>(plan + PL.off_feat);
-    const float4 *wts = reinterpret_cast<const float4 *>(plan + PL.off_w);
-    for (int e = e0; e < e1; ++e) {
-      const uint32_t inf = info[e];
-      const int tstar = (inf >> 8) & 7;
-      const int slot0 = (inf >> 11) & 31;
-      const int nfeat = (inf >> 16) & 7;
-      scan_entry<G, HALF>(sb + slot0 * kTileWords, tstar, nfeat, feats[e], wts[e], acc);
-    }
-  };
-
   auto compute = [&](const Item &it, int buf) {
     const unsigned char *plan = splans + it.slot * PL.bytes;
     const PlanHeader *hdr = reinterpret_cast<const PlanHeader *>(plan);
@@ -479,11 +462,20 @@ __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
     const uint16_t *stage_begin = reinterpret_cast<const uint16_t *>(plan + PL.off_stage_begin);
     const uint32_t *sb = sbuf + buf * (kStageBytes / 4) + word;
     const int e0 = stage_begin[it.st], e1 = stage_begin[it.st + 1];
-    // the half is fixed per warp: one branch per stage, not per entry
-    if (half)
-      stage_entries(plan, sb, e0, e1, std::integral_constant<int, 4>{});
-    else
-      stage_entries(plan, sb, e0, e1, std::integral_constant<int, 0>{});
+    const uint32_t *info = reinterpret_cast<const uint32_t *>(plan + PL.off_info);
+    const uint32_t *feats = reinterpret_cast<const uint32_t *>(plan + PL.off_feat);
+    const float4 *wts = reinterpret_cast<const float4 *>(plan + PL.off_w);
+    for (int e = e0; e < e1; ++e) {
+      const uint32_t inf = info[e];
+      const int tstar = (inf >> 8) & 7;
+      const int slot0 = (inf >> 11) & 31;
+      const int nfeat = (inf >> 16) & 7;
+      const uint32_t *src = sb + slot0 * kTileWords;
+      if (half)
+        scan_entry<G, 4>(src, tstar, nfeat, feats[e], wts[e], acc);
+      else
+        scan_entry<G, 0>(src, tstar, nfeat, feats[e], wts[e], acc);
+    }
   };
 
   auto score_of = [&](int h, int i, int kk) -> float {

@@ -1,119 +1,112 @@
-// Tensor-core form of the Fathom scan for sm_100a (tcgen05, kind::i8).
+// Tensor-core form of the Fathom scan for sm_100a (tcgen05.mma kind::i8,
+// A operand in tensor memory).
 //
 // The score of key i for query head h ("Fathom Makes KV-Cache Scans
 // Query-Adaptive for Long-Context Decoding", method paragraphs 2-3; arXiv
-// 2609.17652 abstract) is
-//   s_h(i) = C_h + sum_{c: t_c > 0} q_c s_c y_{t_c}(i, c),
-//   C_h    = sum_c q_c (m_c + s_c (2^(4-t_c) - 1) / 2),
-// y_t = the top t bits of the 4-bit code, left-aligned (y_t = 2^(4-t) v_t).
-// For the G query heads of one KV head this is a product of two matrices:
-//   A [tokens x features], A = y_f(i) in 0..15 (a "feature" is one
-//     (channel, prefix length) pair some head of the group reads),
-//   B [features x (head, digit)], the weight q_c s_c of a head that reads
-//     the feature, as a fixed-point integer W / Delta_h split into four
-//     signed base-256 int8 digits (0 for the other heads).
-// Integer products accumulate exactly in int32 on the tensor cores
-// (tcgen05.mma kind::i8, M = 128 tokens, N = 16 = 4 heads x 4 digits,
-// K = 32 features); the epilogue forms s_h = C_h + Delta_h sum_m 256^m acc_m.
+// 2609.17652 abstract) is a sum over the bit planes the head reads:
+//   s_h(i) = C_h + sum_{(c, j): j < t_hc} W_hcj b_cj(i),   W_hcj = q_hc s_c 2^(3 - j),
+//   C_h    = sum_c q_hc (m_c + s_c (2^(4 - t_hc) - 1) / 2),
+// b_cj(i) the bit of plane j of channel c for key i.  For the G query heads of
+// one KV head this is one matrix product over the union planes of the group:
+//   A [keys x planes] = the plane bits,
+//   B [planes x (head, digit)] = W_hcj / Delta_h as a 30-bit fixed-point
+//     integer in four signed base-256 int8 digits (0 where the head does not
+//     read the plane),
+// accumulated exactly in int32 by the tensor cores; the epilogue forms
+//   s_h = C_h + Delta_h sum_m 256^m acc_m.
 //
-// Layout (per block, 256 threads, 1024-token tiles):
-//  * the union plane rows of a K-chunk are staged with 16-byte cp.async;
-//  * every thread rebuilds the 4-bit prefix codes of its word (32 tokens)
-//    as bytes in 8 registers and stores them MN-major into the A tile of
-//    the chunk; one elected thread issues the 8 MMAs of the chunk and
-//    commits them to an mbarrier that releases the A buffer;
-//  * the accumulators of a tile (8 M-blocks x 16 columns) live in tensor
-//    memory, double-buffered across tiles; after the last chunk of a tile
-//    each warp reads its 32 lanes back (tcgen05.ld) and writes samples,
-//    candidates or debug scores exactly like the CUDA-core form.
-// Every wait on an mbarrier is bounded in time; a timeout records a device
-// fault in the workspace status, releases tensor memory and ends the block.
+// Layout (B200 design).  A 1024-key tile of one KV head is 32 plane words per
+// plane.  Tensor-memory lane (quarter q, lane l) of M-block (hr, e) stands for
+// word l of the tile and bit position r = q + 4 hr of every byte of that word;
+// the four bytes of its 32-bit column hold, for a pair of planes (p, p'), the
+// bits of keys 8 kk + r for kk = 2e, 2e + 1:
+//   cell = byte_perm(P_p, P_p', e ? 0x7632 : 0x5410) & (0x01010101 << r)
+// (one permute per plane pair and one AND per cell, each byte 0 or 2^r).  The
+// two keys in a cell are separated by B: its 32 columns are (kk', head, digit)
+// and a column reads only the bytes of its kk'.  The 2^r of a lane is undone
+// in the epilogue.
+//
+// Roles (10 warps): warp 8 stages 32 plane rows of a tile ("chunk") into
+// shared memory with 16-byte cp.async copies; warps 0-7 turn a chunk into
+// tensor-memory cells (warp w: lane quarter w % 4, half the chunk's planes)
+// and, one tile later, read the tile's accumulators back, score and filter
+// them; one thread of warp 9 issues the MMAs.  They hand chunks, A buffers
+// and accumulators to each other through mbarriers; every wait is bounded in
+// time and a timeout records a device fault in the workspace status.
+// Accumulators are preset to the bits of 1.5 * 2^23, so that an accumulator
+// read back as a float is 1.5 * 2^23 + acc exactly (|acc| <= 2^22).
 #include "fathom_internal.cuh"
 
 namespace fathom {
 
 // ---------------------------------------------------------------- layout --
-constexpr int kTcThreads = 256;
-constexpr int kTcTileWords = 32;                      // 1024 tokens per tile
-constexpr int kTcMBlocks = kTcTileWords * 32 / 128;   // 8 MMAs of M = 128 per K-chunk
-constexpr int kTcKChunk = 32;                         // features per MMA (kind::i8 K)
-constexpr int kTcMaxRows = 4 * kTcKChunk;             // plane rows a chunk can need
-// A tile (one K-chunk): MN-major, no swizzle.  A core matrix is 16 tokens x
-// 8 features (128 B, 16 B per feature row).  MN blocks are 144 B apart and
-// K blocks 1152 B apart (the 16 B pads make the 16-byte stores of a warp
-// fall on distinct banks); M-blocks are 4624 B apart.
-constexpr int kTcSBO_A = 144;
-constexpr int kTcLBO_A = 8 * kTcSBO_A;                 // 1152
-constexpr int kTcMBlockBytes = 4 * kTcLBO_A + 16;     // 4624
-constexpr int kTcABytes = kTcMBlocks * kTcMBlockBytes;  // 36992
-// B tile (one K-chunk): K-major, no swizzle, 16 rows (head, digit) x 32
-// features: 8-row blocks 128 B apart, 16-feature halves 256 B apart.
-constexpr int kTcSBO_B = 128;
-constexpr int kTcLBO_B = 256;
-constexpr int kTcBBytes = 512;
-constexpr int kTcStageBytes = kTcMaxRows * kTcTileWords * 4;  // 16 KiB
-constexpr int kTcNumStage = 3;
-constexpr int kTcNumPlanSlots = 3;
-constexpr int kTcTmemCols = 2 * kTcMBlocks * 16;  // 256: two tiles of accumulators
+constexpr int kTcTileWords = 32;                        // 1024 keys per tile
+constexpr int kTcChunkPlanes = 32;                      // plane rows per chunk
+constexpr int kTcStageBytes = kTcChunkPlanes * kTcTileWords * 4;  // 4 KiB
+constexpr int kTcNumStages = 16;                        // chunks staged ahead
+constexpr int kTcNumABuf = 4;                           // A buffers in tensor memory
+constexpr int kTcBuildWarps = 8;
+constexpr int kTcProducerWarp = 8;
+constexpr int kTcMmaWarp = 9;
+constexpr int kTcThreads = 10 * 32;
+constexpr int kTcAccCols = 4 * 32;                      // one tile: 4 M-blocks x N = 32
+constexpr int kTcABufCols = 4 * 16;                     // one chunk: 4 M-blocks x 16 columns
+constexpr int kTcTmemCols = 512;                        // 2 x 128 accumulators + 4 x 64 A
+constexpr int kTcAColBase = 2 * kTcAccCols;
 constexpr int kTcSampleSectorsPerTile = kTcTileWords / kSectorWords;  // 4
-// tcgen05 instruction descriptor: D s32, A u8 MN-major, B s8 K-major,
-// M = 128, N = 16, dense.
-constexpr uint32_t kTcIdesc = (2u << 4)       // D format s32
-                              | (0u << 7)     // A format u8
-                              | (1u << 10)    // B format s8
-                              | (1u << 15)    // A MN-major
-                              | (0u << 16)    // B K-major
-                              | ((16u >> 3) << 17)   // N
-                              | ((128u >> 4) << 24); // M
+// B for one K-step (16 planes = 8 columns = 32 int8 K elements): 32 rows
+// (kk', head, digit) x 32 bytes, K-major, no swizzle.  Core matrices are
+// 8 rows x 16 bytes; 8-row groups are 128 B apart (SBO), the two 16-byte K
+// halves 512 B apart (LBO).
+constexpr int kTcKStepBytes = 1024;
+constexpr uint32_t kTcSBO = 128;
+constexpr uint32_t kTcLBO = 512;
+// Instruction descriptor: D s32, A u8 K-major (tensor memory), B s8
+// K-major, N = 32, M = 128, dense.
+constexpr uint32_t kTcIdesc = (2u << 4)             // D format s32
+                              | (0u << 7)           // A format u8
+                              | (1u << 10)          // B format s8
+                              | (0u << 15)          // A K-major
+                              | (0u << 16)          // B K-major
+                              | ((32u >> 3) << 17)  // N
+                              | ((128u >> 4) << 24);  // M
+constexpr uint32_t kTcMagicBits = 0x4b400000u;  // 1.5 * 2^23
+constexpr float kTcMagic = 12582912.0f;
+// A plane count above which the cells hold 0/1 instead of 0/2^r, so that an
+// accumulator stays within 2^22 (|digit| <= 128, 2^r <= 128).
+constexpr int kTcSmallP = 256;
 
 struct TcPlanHeader {
-  int nent;
-  int nchunk;
-  int union_planes;
-  int nrows;
-  float K[4];      // C_h
-  float delta[4];  // Delta_h (a power of two)
-  float tau[4];    // candidate threshold, filled when a block loads the plan
-  int pad[4];
+  int P;       // union planes of the group
+  int nchunk;  // ceil(P / 32)
+  int pad0, pad1;
+  float K[4];  // C_h
+  float D[4];  // Delta_h (a power of two)
+  float pad2[4];
 };
-static_assert(sizeof(TcPlanHeader) == 80, "header size");
+static_assert(sizeof(TcPlanHeader) == 64, "header size");
 
 struct TcPlanLayout {
-  int maxch;
-  int off_chunk_entry;  // uint16 [maxch + 1]
-  int off_chunk_row;    // uint16 [maxch + 1]
-  int off_rows;         // uint16 [4 d]: c * 4 + j of every staged row, by chunk
-  int off_info;         // uint32 [d]: t* | nfeat << 3 | kpos0 << 6 | slot0 << 11
-  int off_feat;         // uint32 [d]: feature f's prefix length in bits 3f .. 3f+2
-  int off_b;            // int8 [maxch][512]
+  int off_rows;  // uint16 [4 d]: c * 4 + j of every union plane, channel-major
+  int off_b;     // int8 [ceil(4 d / 16)][1024]
   int bytes;
 };
 
 __host__ __device__ inline TcPlanLayout tc_plan_layout(int d) {
   TcPlanLayout L;
-  L.maxch = (4 * d) / (kTcKChunk - 3) + 2;
-  int o = (int)sizeof(TcPlanHeader);
-  L.off_chunk_entry = o;
-  o = align16(o + 2 * (L.maxch + 1));
-  L.off_chunk_row = o;
-  o = align16(o + 2 * (L.maxch + 1));
-  L.off_rows = o;
-  o = align16(o + 2 * 4 * d);
-  L.off_info = o;
-  o = align16(o + 4 * d);
-  L.off_feat = o;
-  o = align16(o + 4 * d);
-  L.off_b = o;
-  o = align16(o + kTcBBytes * L.maxch);
-  L.bytes = o;
+  L.off_rows = (int)sizeof(TcPlanHeader);
+  L.off_b = align16(L.off_rows + 2 * 4 * d);
+  L.bytes = L.off_b + ((4 * d + 15) / 16) * kTcKStepBytes;
   return L;
 }
 
 int tc_plan_bytes(int d) { return tc_plan_layout(d).bytes; }
 
-int tc_smem_bytes(int d, int S) {
-  return 2 * kTcABytes + kTcNumStage * kTcStageBytes + kTcNumPlanSlots * tc_plan_layout(d).bytes +
-         4 * (S + 1) + 64;
+static int tc_smem_bytes(int d, int S) {
+  int b = 128 + kTcNumStages * kTcStageBytes + tc_plan_layout(d).bytes + 4 * (S + 1);
+  // more than half an SM's shared memory: one block per SM, so that the
+  // block's 512 tensor-memory columns never wait for another block
+  return b < 120 * 1024 ? 120 * 1024 : b;
 }
 
 // --------------------------------------------------------------- helpers --
@@ -122,16 +115,10 @@ __device__ __forceinline__ uint32_t tc_smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__device__ __forceinline__ void tc_cp_async16(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(tc_smem_u32(dst)), "l"(src),
+__device__ __forceinline__ void tc_cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
                "r"(src_bytes)
                : "memory");
-}
-
-__device__ __forceinline__ uint32_t tc_shift(uint32_t x, int s) {
-  if (s > 0) return __umulhi(x, 1u << (32 - s));
-  if (s < 0) return x * (1u << (-s));
-  return x;
 }
 
 __device__ __forceinline__ uint64_t tc_smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -145,58 +132,96 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 }
-__device__ __forceinline__ void tc_fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t accumulate) {
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kTcIdesc), "r"(accumulate), "r"(0u)
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n" ::"r"(bar)
       : "memory");
 }
-
-__device__ __forceinline__ void tc_commit(uint32_t mbar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                   mbar)
-               : "memory");
+// Arrives on bar once all of this thread's earlier cp.async copies are done.
+__device__ __forceinline__ void mbar_arrive_cp_async(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
 }
 
-// Waits for the completion of the mbarrier phase with the given parity, at
-// most about two seconds.  Returns false on timeout.
-__device__ __forceinline__ bool tc_wait(uint32_t mbar, uint32_t parity) {
+// Waits for the completion of the phase of bar with the given parity, giving
+// up after about a second (2^31 cycles).  Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  if (done) return true;
   const long long t0 = clock64();
   while (true) {
-    uint32_t done;
     asm volatile(
         "{\n\t.reg .pred P;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
         "selp.b32 %0, 1, 0, P;\n\t}\n"
         : "=r"(done)
-        : "r"(mbar), "r"(parity)
+        : "r"(bar), "r"(parity)
         : "memory");
     if (done) return true;
-    if (clock64() - t0 > (1ll << 32)) return false;
+    if (clock64() - t0 > (1ll << 31)) return false;
   }
 }
 
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, int32_t (&v)[16]) {
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16];\n"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(kTcIdesc), "r"(1u)
+      : "memory");
 }
 
-// int32 -> float for |v| < 2^22, exactly, without the conversion unit.
-__device__ __forceinline__ float tc_i2f(int32_t v) {
-  return __int_as_float(v + 0x4b400000) - 12582912.0f;
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+
+// Writes the value x into 32 consecutive columns of this warp's lanes.
+__device__ __forceinline__ void tc_st32_fill(uint32_t taddr, uint32_t x) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};\n" ::"r"(
+          taddr),
+      "r"(x)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
 
 __device__ int tc_block_scan(int v, int *s_tmp) {
@@ -237,29 +262,18 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   const TcPlanLayout L = tc_plan_layout(d);
   unsigned char *plan = p.plans + (size_t)gid * L.bytes;
   TcPlanHeader *hdr = reinterpret_cast<TcPlanHeader *>(plan);
-  uint16_t *chunk_entry = reinterpret_cast<uint16_t *>(plan + L.off_chunk_entry);
-  uint16_t *chunk_row = reinterpret_cast<uint16_t *>(plan + L.off_chunk_row);
   uint16_t *rows = reinterpret_cast<uint16_t *>(plan + L.off_rows);
-  uint32_t *info = reinterpret_cast<uint32_t *>(plan + L.off_info);
-  uint32_t *featw = reinterpret_cast<uint32_t *>(plan + L.off_feat);
   int8_t *bmat = reinterpret_cast<int8_t *>(plan + L.off_b);
 
   __shared__ int s_tmp[32];
   __shared__ double s_red[4][8];
-  __shared__ double s_wmax[4];
-  __shared__ uint8_t s_ts[FATHOM_MAX_D], s_nf[FATHOM_MAX_D];
-  __shared__ uint8_t s_chunk[FATHOM_MAX_D], s_kpos[FATHOM_MAX_D], s_slot[FATHOM_MAX_D];
-  __shared__ int s_nent, s_nchunk;
-
-  // zero the B matrices (unused features and heads must contribute nothing)
-  for (int i = threadIdx.x; i < kTcBBytes * L.maxch / 16; i += blockDim.x)
-    reinterpret_cast<uint4 *>(bmat)[i] = make_uint4(0, 0, 0, 0);
+  __shared__ unsigned long long s_wmax[4];
+  __shared__ int s_P;
 
   int t[4] = {0, 0, 0, 0};
-  double w[4] = {0.0, 0.0, 0.0, 0.0};
-  double kpart[4] = {0.0, 0.0, 0.0, 0.0};
-  int tstar = 0, nfeat = 0;
-  uint32_t ftf = 0;  // prefix length of feature f in bits 3f .. 3f+2
+  double w[4] = {0.0, 0.0, 0.0, 0.0};      // q_c s_c of a head that reads channel c
+  double kpart[4] = {0.0, 0.0, 0.0, 0.0};  // its share of C_h
+  int tstar = 0;
   if (c < d) {
     const double m = se.qmin[(int64_t)g * d + c];
     const double sc = se.qscale[(int64_t)g * d + c];
@@ -272,17 +286,9 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
       const double cell = (double)(1 << (4 - t[hh]));
       kpart[hh] = qv * (m + sc * ((cell - 1.0) * 0.5));
     }
-    for (int tf = 1; tf <= 4; ++tf) {
-      bool used = false;
-      for (int hh = 0; hh < G; ++hh) used |= t[hh] == tf;
-      if (used) {
-        ftf |= (uint32_t)tf << (3 * nfeat);
-        ++nfeat;
-      }
-    }
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x < 4) s_wmax[threadIdx.x] = 0.0;
+  if (threadIdx.x < 4) s_wmax[threadIdx.x] = 0ull;
   __syncthreads();
   for (int hh = 0; hh < 4; ++hh) {
     double v = kpart[hh], a = fabs(w[hh]);
@@ -294,82 +300,58 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
     if (lane == 0) {
       s_red[hh][warp] = v;
       // non-negative doubles order like their bit patterns
-      atomicMax(reinterpret_cast<unsigned long long *>(&s_wmax[hh]),
-                (unsigned long long)__double_as_longlong(a));
+      atomicMax(&s_wmax[hh], (unsigned long long)__double_as_longlong(a));
     }
   }
+  // the union planes of channel c are rows off .. off + t* - 1 of the plan
+  const int incl = tc_block_scan(tstar, s_tmp);
+  const int off = incl - tstar;
+  if (threadIdx.x == blockDim.x - 1) s_P = incl;
   __syncthreads();
-  // entry order and the planes before each channel
-  const int packed = (tstar > 0 ? 1 : 0) | (tstar << 12);
-  const int incl = tc_block_scan(packed, s_tmp);
-  const int e = (incl & 0xfff) - 1;
-  if (tstar > 0) {
-    s_ts[e] = (uint8_t)tstar;
-    s_nf[e] = (uint8_t)nfeat;
+  const int P = s_P;
+  const int nks = (P + 15) / 16;
+  // B of every used K-step starts at zero (padding planes, heads that do not
+  // read a plane, and the other key of every cell contribute nothing)
+  for (int i = threadIdx.x; i < nks * kTcKStepBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4 *>(bmat)[i] = make_uint4(0, 0, 0, 0);
+  double delta[4];
+  for (int hh = 0; hh < 4; ++hh) {
+    // the largest plane weight is 8 max_c |q_c s_c|; W / Delta < 2^30
+    const double wmax = 8.0 * __longlong_as_double((long long)s_wmax[hh]);
+    int ex = 0;
+    frexp(wmax, &ex);  // wmax < 2^ex
+    delta[hh] = wmax > 0.0 ? ldexp(1.0, ex - 30) : 1.0;
   }
-  if (threadIdx.x == blockDim.x - 1) s_nent = incl & 0xfff;
-  __syncthreads();
-  const int nent = s_nent;
-  // pack whole entries into K-chunks of at most 32 features (serial, <= d entries)
   if (threadIdx.x == 0) {
-    int ch = 0, kpos = 0, slot = 0, rowpos = 0;
-    chunk_entry[0] = 0;
-    chunk_row[0] = 0;
-    for (int i = 0; i < nent; ++i) {
-      if (kpos + s_nf[i] > kTcKChunk) {
-        ++ch;
-        chunk_entry[ch] = (uint16_t)i;
-        chunk_row[ch] = (uint16_t)rowpos;
-        kpos = 0;
-        slot = 0;
-      }
-      s_chunk[i] = (uint8_t)ch;
-      s_kpos[i] = (uint8_t)kpos;
-      s_slot[i] = (uint8_t)slot;
-      kpos += s_nf[i];
-      slot += s_ts[i];
-      rowpos += s_ts[i];
-    }
-    const int nchunk = nent > 0 ? ch + 1 : 0;
-    chunk_entry[nchunk] = (uint16_t)nent;
-    chunk_row[nchunk] = (uint16_t)rowpos;
-    s_nchunk = nchunk;
-    hdr->nent = nent;
-    hdr->nchunk = nchunk;
-    hdr->union_planes = rowpos;
-    hdr->nrows = rowpos;
+    hdr->P = P;
+    hdr->nchunk = (P + kTcChunkPlanes - 1) / kTcChunkPlanes;
+    hdr->pad0 = hdr->pad1 = 0;
+    const int nw = (blockDim.x + 31) >> 5;
     for (int hh = 0; hh < 4; ++hh) {
       double sum = 0.0;
-      for (int wv = 0; wv < 8; ++wv) sum += s_red[hh][wv];
+      for (int wv = 0; wv < nw; ++wv) sum += s_red[hh][wv];
       hdr->K[hh] = hh < G ? (float)sum : 0.0f;
-      int ex = 0;
-      frexp(s_wmax[hh], &ex);  // wmax < 2^ex
-      hdr->delta[hh] = s_wmax[hh] > 0.0 ? (float)ldexp(1.0, ex - 30) : 1.0f;
-      hdr->tau[hh] = -INFINITY;
+      hdr->D[hh] = (float)delta[hh];
+      hdr->pad2[hh] = 0.0f;
     }
-    atomicAdd(&p.status->union_planes, (uint32_t)rowpos);
+    atomicAdd(&p.status->union_planes, (uint32_t)P);
   }
   __syncthreads();
-  if (tstar > 0) {
-    const int ch = s_chunk[e], kpos0 = s_kpos[e], slot0 = s_slot[e];
-    info[e] = (uint32_t)tstar | ((uint32_t)nfeat << 3) | ((uint32_t)kpos0 << 6) |
-              ((uint32_t)slot0 << 11);
-    featw[e] = ftf;
-    const int row0 = chunk_row[ch] + slot0;
-    for (int j = 0; j < tstar; ++j) rows[row0 + j] = (uint16_t)(c * 4 + j);
-    int8_t *bch = bmat + (size_t)ch * kTcBBytes;
-    for (int f = 0; f < nfeat; ++f) {
-      const int tf = (ftf >> (3 * f)) & 7;
-      const int k = kpos0 + f;
-      for (int hh = 0; hh < G; ++hh) {
-        if (t[hh] != tf) continue;
-        const double delta = (double)hdr->delta[hh];
-        long long x = llrint(w[hh] / delta);
-        for (int mdig = 0; mdig < 4; ++mdig) {
-          const long long dg = ((x + 128) & 255) - 128;
-          x = (x - dg) >> 8;
-          const int n = 4 * hh + mdig;
-          bch[(n >> 3) * kTcSBO_B + (k >> 4) * kTcLBO_B + (n & 7) * 16 + (k & 15)] = (int8_t)dg;
+  for (int j = 0; j < tstar; ++j) {
+    const int pl = off + j;
+    rows[pl] = (uint16_t)(c * 4 + j);
+    int8_t *bk = bmat + (size_t)(pl >> 4) * kTcKStepBytes;
+    const int col = (pl & 15) >> 1, pp = pl & 1;
+    for (int hh = 0; hh < G; ++hh) {
+      if (j >= t[hh]) continue;
+      long long x = llrint(ldexp(w[hh], 3 - j) / delta[hh]);
+      for (int dg = 0; dg < 4; ++dg) {
+        const long long v = dg < 3 ? ((x + 128) & 255) - 128 : x;
+        x = (x - v) >> 8;
+        for (int kq = 0; kq < 2; ++kq) {
+          const int n = kq * 16 + hh * 4 + dg;
+          const int k = 4 * col + 2 * pp + kq;
+          bk[(n >> 3) * kTcSBO + (k >> 4) * kTcLBO + (n & 7) * 16 + (k & 15)] = (int8_t)v;
         }
       }
     }
@@ -377,12 +359,6 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
 }
 
 // ------------------------------------------------------------ scan kernel --
-
-struct TcLoc {
-  int s, g, ti;
-  int64_t n, W;
-  const uint32_t *planes;
-};
 
 template <int MODE>
 __device__ __forceinline__ int64_t tc_tiles_per_group(int64_t n, const ScanParams &p) {
@@ -392,6 +368,12 @@ __device__ __forceinline__ int64_t tc_tiles_per_group(int64_t n, const ScanParam
   }
   return (plane_words(n) + kTcTileWords - 1) / kTcTileWords;
 }
+
+struct TcLoc {
+  int s, g, ti, per;
+  int64_t n, W;
+  const uint32_t *planes;
+};
 
 template <int MODE>
 __device__ __forceinline__ TcLoc tc_locate(const ScanParams &p, const int *s_tprefix, int t) {
@@ -406,19 +388,12 @@ __device__ __forceinline__ TcLoc tc_locate(const ScanParams &p, const int *s_tpr
   L.n = se.n;
   L.W = plane_words(L.n);
   L.planes = se.planes;
-  const int per = (int)tc_tiles_per_group<MODE>(L.n, p);
+  L.per = (int)tc_tiles_per_group<MODE>(L.n, p);
   const int r = t - s_tprefix[lo];
-  L.g = r / per;
-  L.ti = r - L.g * per;
+  L.g = r / L.per;
+  L.ti = r - L.g * L.per;
   return L;
 }
-
-struct TcItem {
-  int t;      // tile in the launch's tile space (-1 = none)
-  int ch;     // K-chunk of the tile
-  int slot;   // plan slot
-  int nch;    // chunks of the tile
-};
 
 template <int G, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
@@ -428,17 +403,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const int warp = tid >> 5;
   const int d = p.d;
   const TcPlanLayout PL = tc_plan_layout(d);
-  unsigned char *sA = smem;                                  // 2 x kTcABytes
-  uint32_t *sStage = reinterpret_cast<uint32_t *>(smem + 2 * kTcABytes);
-  unsigned char *sPlans = smem + 2 * kTcABytes + kTcNumStage * kTcStageBytes;
-  int *s_tprefix = reinterpret_cast<int *>(sPlans + kTcNumPlanSlots * PL.bytes);
-  __shared__ __align__(8) unsigned long long s_mbar[2];
+  unsigned char *sStage = smem;
+  unsigned char *sPlan = smem + kTcNumStages * kTcStageBytes;
+  const TcPlanHeader *sHdr = reinterpret_cast<const TcPlanHeader *>(sPlan);
+  const uint16_t *sRows = reinterpret_cast<const uint16_t *>(sPlan + PL.off_rows);
+  int *s_tprefix = reinterpret_cast<int *>(sPlan + PL.bytes);
+  __shared__ __align__(8) unsigned long long s_bar[2 * kTcNumStages + 2 * kTcNumABuf + 4];
   __shared__ uint32_t s_tmem;
   __shared__ int s_tmp[32];
-  __shared__ int s_slot_gid[kTcNumPlanSlots];
-  __shared__ int s_fault;
+  __shared__ volatile int s_fault;
 
-  // ---- tile space ----------------------------------------------------------
+  const uint32_t bar0 = tc_smem_u32(&s_bar[0]);
+  auto stage_full = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  auto stage_empty = [&](int i) { return bar0 + 8u * (uint32_t)(kTcNumStages + i); };
+  auto a_full = [&](int i) { return bar0 + 8u * (uint32_t)(2 * kTcNumStages + i); };
+  auto a_empty = [&](int i) { return bar0 + 8u * (uint32_t)(2 * kTcNumStages + kTcNumABuf + i); };
+  auto acc_full = [&](int i) { return bar0 + 8u * (uint32_t)(2 * kTcNumStages + 2 * kTcNumABuf + i); };
+  auto acc_empty = [&](int i) {
+    return bar0 + 8u * (uint32_t)(2 * kTcNumStages + 2 * kTcNumABuf + 2 + i);
+  };
+
+  // ---- tile space: every (session, KV head) contributes its tiles --------
   for (int base = 0; base < p.S; base += kTcThreads) {
     const int s = base + tid;
     int v = 0;
@@ -455,7 +440,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const int t_end = (int)(((int64_t)(blockIdx.x + 1) * total) / gridDim.x);
   if (t_begin >= t_end) return;
 
-  // ---- tensor memory and barriers -----------------------------------------
+  // ---- tensor memory, barriers, preset accumulators ----------------------
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                      tc_smem_u32(&s_tmem)),
@@ -464,333 +449,321 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(tc_smem_u32(&s_mbar[0])) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(tc_smem_u32(&s_mbar[1])) : "memory");
+    for (int i = 0; i < kTcNumStages; ++i) {
+      mbar_init(stage_full(i), 32);             // every producer lane, after its copies
+      mbar_init(stage_empty(i), kTcBuildWarps);
+    }
+    for (int i = 0; i < kTcNumABuf; ++i) {
+      mbar_init(a_full(i), kTcBuildWarps);
+      mbar_init(a_empty(i), 1);                 // tcgen05.commit
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full(i), 1);
+      mbar_init(acc_empty(i), kTcBuildWarps);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     s_fault = 0;
   }
-  if (tid < kTcNumPlanSlots) s_slot_gid[tid] = -1;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  const int quarter = warp & 3;
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+  if (warp < kTcBuildWarps) {
+    // warps q and q + 4 preset one half each of the two accumulator sets
+    const int half = warp >> 2;
+    for (int i = 0; i < 4; ++i)
+      tc_st32_fill(tmem + lane_base + (uint32_t)(half * kTcAccCols + 32 * i), kTcMagicBits);
+    tc_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
-  // ---- plans ---------------------------------------------------------------
-  auto ensure_plan = [&](int gid, int busy0, int busy1) -> int {
-    int slot = -1;
-    for (int i = 0; i < kTcNumPlanSlots; ++i)
-      if (s_slot_gid[i] == gid) slot = i;
-    if (slot >= 0) return slot;
-    for (int i = kTcNumPlanSlots - 1; i >= 0; --i)
-      if (i != busy0 && i != busy1) slot = i;
+  // pipeline counters: chunk items and tiles since the start of the kernel,
+  // and (MMA thread) the last item and tile whose completion was committed
+  uint32_t it = 0, tj = 0;
+  int last_item = -1, last_tile = -1;
+
+  // ---- segments: runs of tiles that share one (session, KV head) ---------
+  int t = t_begin;
+  while (t < t_end) {
     __syncthreads();
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.plans + (size_t)gid * PL.bytes);
-    uint4 *dst = reinterpret_cast<uint4 *>(sPlans + slot * PL.bytes);
-    for (int i = tid; i < PL.bytes / 16; i += kTcThreads) dst[i] = src[i];
-    tc_fence_proxy_async();  // the B tiles are read by the tensor cores
+    if (s_fault) break;
+    const TcLoc L0 = tc_locate<MODE>(p, s_tprefix, t);
+    const int seg_end = min(t_end, t - L0.ti + L0.per);
+    const int ntiles = seg_end - t;
+    const int ti0 = L0.ti;
+    {
+      const int gid = L0.s * p.h_kv + L0.g;
+      const unsigned char *gplan = p.plans + (size_t)gid * PL.bytes;
+      const int P = reinterpret_cast<const TcPlanHeader *>(gplan)->P;
+      const int used = PL.off_b + ((P + 15) / 16) * kTcKStepBytes;
+      for (int i = tid; i < used / 16; i += kTcThreads)
+        reinterpret_cast<uint4 *>(sPlan)[i] = reinterpret_cast<const uint4 *>(gplan)[i];
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // B is read by the MMAs
+    }
     __syncthreads();
-    if (tid < G) {
-      TcPlanHeader *hdr = reinterpret_cast<TcPlanHeader *>(sPlans + slot * PL.bytes);
-      float tau = -INFINITY;
-      if (MODE == kModeFilter) {
-        const int s = gid / p.h_kv, g = gid - s * p.h_kv;
-        const uint32_t key = p.tau[(int64_t)s * p.h_q + g * G + tid];
-        tau = key == 0u ? -INFINITY : key_float(key);
+    const int P = sHdr->P;
+    const int nch = sHdr->nchunk > 0 ? sHdr->nchunk : 1;  // a plane-less group still has tiles
+    const bool big = P > kTcSmallP;                        // 0/1 cells instead of 0/2^r
+    const int64_t head0 = (int64_t)L0.s * p.h_q + L0.g * G;
+
+    if (warp == kTcProducerWarp) {
+      // ---------------------------------------------------------- producer --
+      const uint32_t *gbase = L0.planes + (int64_t)L0.g * d * 4 * L0.W;
+      const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
+      uint32_t i = it;
+      for (int j = 0; j < ntiles && !s_fault; ++j) {
+        const int ti = ti0 + j;
+        for (int c = 0; c < nch; ++c, ++i) {
+          const int st = (int)(i % kTcNumStages);
+          if (i >= (uint32_t)kTcNumStages &&
+              !mbar_wait(stage_empty(st), ((i / kTcNumStages) - 1) & 1)) {
+            s_fault = 1;
+            break;
+          }
+          const int nrows = min(kTcChunkPlanes, P - c * kTcChunkPlanes);
+          const uint32_t dst0 = tc_smem_u32(sStage + st * kTcStageBytes);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int id = lane + 32 * k;  // row id / 8, 16-byte piece id % 8
+            const int row = id >> 3, piece = id & 7;
+            if (row < nrows) {
+              const uint32_t *src = gbase + (int64_t)sRows[c * kTcChunkPlanes + row] * L0.W;
+              int64_t gw;
+              bool ok;
+              if (MODE == kModeSample) {
+                const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (piece >> 1);
+                gw = sj * kSampleStride * kSectorWords + (piece & 1) * 4;
+                ok = sj < nsamp && gw < L0.W;
+              } else {
+                gw = (int64_t)ti * kTcTileWords + piece * 4;
+                ok = gw < L0.W;
+              }
+              tc_cp_async16(dst0 + (uint32_t)(row * 128 + piece * 16),
+                            ok ? (const void *)(src + gw) : (const void *)src, ok ? 16u : 0u);
+            }
+          }
+          mbar_arrive_cp_async(stage_full(st));
+        }
+        if (s_fault) break;
       }
-      hdr->tau[tid] = tau;
-    }
-    if (tid == 0) s_slot_gid[slot] = gid;
-    __syncthreads();
-    return slot;
-  };
-  auto first_item = [&](int t, int busy0, int busy1) -> TcItem {
-    TcItem it;
-    it.t = t;
-    it.ch = 0;
-    if (t >= t_end) {
-      it.t = -1;
-      it.slot = -1;
-      it.nch = 0;
-      return it;
-    }
-    const TcLoc L = tc_locate<MODE>(p, s_tprefix, t);
-    it.slot = ensure_plan(L.s * p.h_kv + L.g, busy0, busy1);
-    const int nch = reinterpret_cast<const TcPlanHeader *>(sPlans + it.slot * PL.bytes)->nchunk;
-    it.nch = nch > 0 ? nch : 1;  // a head with no bits still needs its constant scores
-    return it;
-  };
-  auto next_item = [&](const TcItem &a, int busy0, int busy1) -> TcItem {
-    if (a.t < 0) return a;
-    if (a.ch + 1 < a.nch) {
-      TcItem b = a;
-      b.ch += 1;
-      return b;
-    }
-    return first_item(a.t + 1, busy0, busy1);
-  };
-
-  // ---- staged copies of a chunk's rows ------------------------------------
-  auto issue = [&](const TcItem &it, int buf) {
-    if (it.t < 0) return;
-    const TcLoc L = tc_locate<MODE>(p, s_tprefix, it.t);
-    const unsigned char *plan = sPlans + it.slot * PL.bytes;
-    const TcPlanHeader *hdr = reinterpret_cast<const TcPlanHeader *>(plan);
-    if (hdr->nchunk == 0) return;
-    const uint16_t *chunk_row = reinterpret_cast<const uint16_t *>(plan + PL.off_chunk_row);
-    const uint16_t *rows = reinterpret_cast<const uint16_t *>(plan + PL.off_rows);
-    const int r0 = chunk_row[it.ch], nrows = chunk_row[it.ch + 1] - r0;
-    uint32_t *dst_base = sStage + buf * (kTcStageBytes / 4);
-    const uint32_t *gbase = L.planes + (int64_t)L.g * d * 4 * L.W;
-    for (int id = tid; id < nrows * 8; id += kTcThreads) {
-      const int slot = id >> 3, q = id & 7;
-      const uint32_t *row = gbase + (int64_t)rows[r0 + slot] * L.W;
-      int64_t gw;
-      bool ok;
-      if (MODE == kModeSample) {
-        const int64_t sj = (int64_t)L.ti * kTcSampleSectorsPerTile + (q >> 1);
-        gw = sj * kSampleStride * kSectorWords + (q & 1) * 4;
-        ok = sj < sampled_sectors(L.n) && gw < L.W;
-      } else {
-        gw = (int64_t)L.ti * kTcTileWords + q * 4;
-        ok = gw < L.W;
-      }
-      tc_cp_async16(dst_base + slot * kTcTileWords + q * 4,
-                    ok ? (const void *)(row + gw) : (const void *)row, ok ? 16u : 0u);
-    }
-  };
-
-  // ---- build the A tile of one chunk ---------------------------------------
-  // Thread (warp w, lane l) owns word l of the tile and the chunk's entries
-  // e = w, w + 8, ...  Register R[r], byte kk = the prefix code y (0..15) of
-  // token 32 l + 8 kk + r; {R0..R3} and {R4..R7} are the 16-token MN rows
-  // 2 (l % 4) and 2 (l % 4) + 1 of M-block l / 4.
-  auto build = [&](const TcItem &it, int sbuf, int abuf) {
-    const unsigned char *plan = sPlans + it.slot * PL.bytes;
-    const TcPlanHeader *hdr = reinterpret_cast<const TcPlanHeader *>(plan);
-    if (hdr->nchunk == 0) return;
-    const uint16_t *chunk_entry = reinterpret_cast<const uint16_t *>(plan + PL.off_chunk_entry);
-    const uint32_t *info = reinterpret_cast<const uint32_t *>(plan + PL.off_info);
-    const uint32_t *featw = reinterpret_cast<const uint32_t *>(plan + PL.off_feat);
-    const uint32_t *src_base = sStage + sbuf * (kTcStageBytes / 4) + lane;
-    unsigned char *a_base = sA + abuf * kTcABytes + (lane >> 2) * kTcMBlockBytes +
-                            (2 * (lane & 3)) * kTcSBO_A;
-    const int e0 = chunk_entry[it.ch], e1 = chunk_entry[it.ch + 1];
-    for (int e = e0 + warp; e < e1; e += kTcThreads / 32) {
-      const uint32_t inf = info[e];
-      const int tstar = inf & 7;
-      const int nfeat = (inf >> 3) & 7;
-      const int kpos0 = (inf >> 6) & 31;
-      const int slot0 = (inf >> 11) & 127;
-      const uint32_t *src = src_base + slot0 * kTcTileWords;
-      uint32_t R[8];
-      const uint32_t p0 = src[0];
+      asm volatile("cp.async.wait_all;\n" ::: "memory");
+    } else if (warp == kTcMmaWarp) {
+      // --------------------------------------------------------------- MMA --
+      if (lane == 0) {
+        const uint32_t b_addr = tc_smem_u32(sPlan + PL.off_b);
+        uint32_t i = it, tt = tj;
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j, ++tt) {
+          const int ab = (int)(tt & 1);
+          if (tt >= 2 && (s_fault || !mbar_wait(acc_empty(ab), ((tt >> 1) - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dcol = tmem + (uint32_t)(ab * kTcAccCols);
+          for (int c = 0; c < nch; ++c, ++i) {
+            const int b = (int)(i % kTcNumABuf);
+            if (s_fault || !mbar_wait(a_full(b), (i / kTcNumABuf) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t acol = tmem + (uint32_t)(kTcAColBase + b * kTcABufCols);
 #pragma unroll
-      for (int r = 0; r < 8; ++r) R[r] = tc_shift(p0, r - 3) & 0x08080808u;
-      if (tstar > 1) {
-        const uint32_t p1 = src[kTcTileWords];
+            for (int ks = 0; ks < 2; ++ks) {
+              if (c * kTcChunkPlanes + 16 * ks < P) {
+                const uint64_t bdesc = tc_smem_desc(
+                    b_addr + (uint32_t)((2 * c + ks) * kTcKStepBytes), kTcLBO, kTcSBO);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) R[r] |= tc_shift(p1, r - 2) & 0x04040404u;
-        if (tstar > 2) {
-          const uint32_t p2 = src[2 * kTcTileWords];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) R[r] |= tc_shift(p2, r - 1) & 0x02020202u;
-          if (tstar > 3) {
-            const uint32_t p3 = src[3 * kTcTileWords];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) R[r] |= p3 >> r & 0x01010101u;
+                for (int mb = 0; mb < 4; ++mb)
+                  tc_mma(dcol + (uint32_t)(32 * mb), acol + (uint32_t)(16 * mb + 8 * ks), bdesc);
+              }
+            }
+            tc_commit(a_empty(b));
+            last_item = (int)i;
+            if (c == nch - 1) {
+              tc_commit(acc_full(ab));
+              last_tile = (int)tt;
+            }
           }
         }
+        if (!ok) s_fault = 1;
       }
-      const uint32_t fw = featw[e];
-      for (int f = 0; f < nfeat; ++f) {
-        const int tf = (fw >> (3 * f)) & 7;
-        // keep the top tf bits of every 4-bit code: bits 3 .. 4 - tf of each byte
-        const uint32_t keep = (((1u << tf) - 1u) << (4 - tf)) * 0x01010101u;
-        const int k = kpos0 + f;
-        unsigned char *dst = a_base + (k >> 3) * kTcLBO_A + (k & 7) * 16;
-        *reinterpret_cast<uint4 *>(dst) =
-            make_uint4(R[0] & keep, R[1] & keep, R[2] & keep, R[3] & keep);
-        *reinterpret_cast<uint4 *>(dst + kTcSBO_A) =
-            make_uint4(R[4] & keep, R[5] & keep, R[6] & keep, R[7] & keep);
+    } else {
+      // ----------------------------------------------- build and epilogue --
+      const int half = warp >> 2;  // which K-step of a chunk; which kk pair in the epilogue
+      const uint32_t m0 = 0x01010101u << quarter;        // r = q
+      const uint32_t m1 = 0x01010101u << (quarter + 4);  // r = q + 4
+      float Kh[G], Dh[G][2], tau[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        Kh[h] = sHdr->K[h];
+        Dh[h][0] = big ? sHdr->D[h] : ldexpf(sHdr->D[h], -quarter);
+        Dh[h][1] = big ? sHdr->D[h] : ldexpf(sHdr->D[h], -(quarter + 4));
+        tau[h] = -INFINITY;
+        if (MODE == kModeFilter) {
+          const uint32_t key = p.tau[head0 + h];
+          tau[h] = key == 0u ? -INFINITY : key_float(key);
+        }
       }
-    }
-  };
+      const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
 
-  // ---- the tile's results ----------------------------------------------------
-  // A tile's accumulators are read one item after its last chunk (so the
-  // MMAs complete while the next chunk is being built); what the epilogue
-  // needs from the plan is copied here first, since the plan slot may be
-  // reused by then.
-  struct Pending {
-    int t, accbuf, has_mma, item;
-    float K[G], D[G], tau[G];
-  };
-  auto make_pending = [&](const TcItem &it, int accbuf, int item) -> Pending {
-    const TcPlanHeader *hdr = reinterpret_cast<const TcPlanHeader *>(sPlans + it.slot * PL.bytes);
-    Pending pd;
-    pd.t = it.t;
-    pd.accbuf = accbuf;
-    pd.has_mma = hdr->nchunk > 0;
-    pd.item = item;
+      auto epilogue = [&](int ti, uint32_t tt) -> bool {
+        const int ab = (int)(tt & 1);
+        if (s_fault || !mbar_wait(acc_full(ab), (tt >> 1) & 1)) return false;
+        tc_fence_after();
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      pd.K[h] = hdr->K[h];
-      pd.D[h] = hdr->delta[h];
-      pd.tau[h] = hdr->tau[h];
-    }
-    return pd;
-  };
-  auto epilogue = [&](const Pending &pd) {
-    const TcLoc L = tc_locate<MODE>(p, s_tprefix, pd.t);
-    const int64_t head0 = (int64_t)L.s * p.h_q + L.g * G;
-    const int quarter = warp & 3;
-    // row 32 quarter + lane of M-block b is token 32 (4 b + quarter) + 8 kk + r
-    const int kk = lane & 3, r = 4 * (lane >> 4) + ((lane >> 2) & 3);
+        for (int hr = 0; hr < 2; ++hr) {
+          const uint32_t taddr = tmem + lane_base + (uint32_t)(ab * kTcAccCols + 32 * (2 * hr + half));
+          uint32_t v[32];
+          tc_ld32(taddr, v);
+          tc_st32_fill(taddr, kTcMagicBits);
+          const int r = quarter + 4 * hr;
 #pragma unroll
-    for (int j = 0; j < kTcMBlocks / 2; ++j) {
-      const int b = 2 * j + (warp >> 2);
-      float sc[G];
-      if (pd.has_mma) {
-        int32_t v[16];
-        tc_ld16(tmem + ((uint32_t)(32 * quarter) << 16) +
-                    (uint32_t)(pd.accbuf * kTcMBlocks * 16 + b * 16),
-                v);
+          for (int kq = 0; kq < 2; ++kq) {
+            const int bit = 8 * (2 * half + kq) + r;  // key bit within the word
+            float sc[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float sum = tc_i2f(v[4 * h + 3]);
-          sum = fmaf(sum, 256.0f, tc_i2f(v[4 * h + 2]));
-          sum = fmaf(sum, 256.0f, tc_i2f(v[4 * h + 1]));
-          sum = fmaf(sum, 256.0f, tc_i2f(v[4 * h + 0]));
-          sc[h] = fmaf(pd.D[h], sum, pd.K[h]);
-        }
-      } else {
+            for (int h = 0; h < G; ++h) {
+              const uint32_t *a = v + 16 * kq + 4 * h;
+              float x = __uint_as_float(a[3]) - kTcMagic;
+              x = fmaf(x, 256.0f, __uint_as_float(a[2]) - kTcMagic);
+              x = fmaf(x, 256.0f, __uint_as_float(a[1]) - kTcMagic);
+              x = fmaf(x, 256.0f, __uint_as_float(a[0]) - kTcMagic);
+              sc[h] = fmaf(x, Dh[h][hr], Kh[h]);
+            }
+            if (MODE == kModeSample) {
+              const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (lane >> 3);
+              if (sj < nsamp) {
+                const int64_t tok = (sj * kSampleStride * kSectorWords + (lane & 7)) * 32 + bit;
+                const int64_t sl = sj * 256 + (lane & 7) * 32 + bit;
 #pragma unroll
-        for (int h = 0; h < G; ++h) sc[h] = pd.K[h];
-      }
-      const int wl = 4 * b + quarter;   // word of the tile
-      const int bit = 8 * kk + r;       // token bit within the word
-      if (MODE == kModeSample) {
-        const int64_t sj = (int64_t)L.ti * kTcSampleSectorsPerTile + (wl >> 3);
-        if (sj < sampled_sectors(L.n)) {
-          const int64_t tok = (sj * kSampleStride * kSectorWords + (wl & 7)) * 32 + bit;
-          const int64_t sl = sj * 256 + (wl & 7) * 32 + bit;
+                for (int h = 0; h < G; ++h)
+                  p.sample[(head0 + h) * p.m_max + sl] = tok < L0.n ? float_key(sc[h]) : 0u;
+              }
+            } else {
+              const int64_t tok = ((int64_t)ti * kTcTileWords + lane) * 32 + bit;
+              const bool valid = tok < L0.n;
+              if (p.debug_scores && valid) {
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-            p.sample[(head0 + h) * p.m_max + sl] = tok < L.n ? float_key(sc[h]) : 0u;
-        }
-      } else {
-        const int64_t tok = ((int64_t)L.ti * kTcTileWords + wl) * 32 + bit;
-        const bool valid = tok < L.n;
-        if (p.debug_scores && valid) {
+                for (int h = 0; h < G; ++h) p.debug_scores[(head0 + h) * L0.n + tok] = sc[h];
+              }
+              bool take[G], any = false;
 #pragma unroll
-          for (int h = 0; h < G; ++h) p.debug_scores[(head0 + h) * L.n + tok] = sc[h];
-        }
-        bool take[G], any = false;
+              for (int h = 0; h < G; ++h) {
+                take[h] = valid && sc[h] >= tau[h];
+                any |= take[h];
+              }
+              if (__any_sync(0xffffffffu, any)) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          take[h] = valid && sc[h] >= pd.tau[h];
-          any |= take[h];
-        }
-        if (__any_sync(0xffffffffu, any)) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const unsigned ballot = __ballot_sync(0xffffffffu, take[h]);
-            if (ballot) {
-              unsigned base = 0;
-              if (lane == 0) base = atomicAdd(&p.counts[head0 + h], (unsigned)__popc(ballot));
-              base = __shfl_sync(0xffffffffu, base, 0);
-              if (take[h]) {
-                const unsigned pos = base + __popc(ballot & ((1u << lane) - 1u));
-                if ((int64_t)pos < p.cap)
-                  p.cand[(head0 + h) * p.cap + pos] = composite(sc[h], (uint32_t)tok);
+                for (int h = 0; h < G; ++h) {
+                  const unsigned ballot = __ballot_sync(0xffffffffu, take[h]);
+                  if (ballot) {
+                    unsigned base = 0;
+                    if (lane == 0) base = atomicAdd(&p.counts[head0 + h], (unsigned)__popc(ballot));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (take[h]) {
+                      const unsigned pos = base + __popc(ballot & ((1u << lane) - 1u));
+                      if ((int64_t)pos < p.cap)
+                        p.cand[(head0 + h) * p.cap + pos] = composite(sc[h], (uint32_t)tok);
+                    }
+                  }
+                }
               }
             }
           }
         }
-      }
-    }
-  };
-
-  // ---- pipeline over (tile, chunk) items -----------------------------------
-  const uint32_t mbar0 = tc_smem_u32(&s_mbar[0]);
-  TcItem cur = first_item(t_begin, -1, -1);
-  TcItem nxt = next_item(cur, cur.slot, -1);
-  issue(cur, 0);
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-  issue(nxt, 1);
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-  TcItem iss = next_item(nxt, cur.slot, nxt.slot);
-  int it = 0, tile_seq = 0;
-  bool fault = false, pending = false;
-  Pending pd;
-  while (true) {
-    issue(iss, (it + 2) % kTcNumStage);
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-    asm volatile("cp.async.wait_group 2;\n" ::: "memory");
-    const int abuf = it & 1;
-    // the MMAs that last read this A buffer (item it - 2) must have finished
-    if (it >= 2 && !tc_wait(mbar0 + 8 * abuf, ((it - 2) >> 1) & 1)) s_fault = 1;
-    __syncthreads();
-    if (s_fault) {
-      fault = true;
-      break;
-    }
-    build(cur, it % kTcNumStage, abuf);
-    tc_fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    const unsigned char *plan = sPlans + cur.slot * PL.bytes;
-    const bool has_mma = reinterpret_cast<const TcPlanHeader *>(plan)->nchunk > 0;
-    if (tid == 0) {
-      tc_fence_after();
-      if (has_mma) {
-        const uint32_t a_addr = tc_smem_u32(sA + abuf * kTcABytes);
-        const uint32_t b_addr = tc_smem_u32(plan + PL.off_b + cur.ch * kTcBBytes);
-        const uint64_t bdesc = tc_smem_desc(b_addr, kTcLBO_B, kTcSBO_B);
-#pragma unroll 1
-        for (int mb = 0; mb < kTcMBlocks; ++mb) {
-          const uint64_t adesc = tc_smem_desc(a_addr + mb * kTcMBlockBytes, kTcLBO_A, kTcSBO_A);
-          tc_mma(tmem + (uint32_t)((tile_seq & 1) * kTcMBlocks * 16 + mb * 16), adesc, bdesc,
-                 cur.ch > 0 ? 1u : 0u);
-        }
-      }
-      tc_commit(mbar0 + 8 * abuf);  // also when empty: keeps the barrier phases in step
-    }
-    // results of the previous tile, whose MMAs ran while this chunk was built
-    if (pending) {
-      if (tc_wait(mbar0 + 8 * (pd.item & 1), (pd.item >> 1) & 1)) {
-        tc_fence_after();
-        epilogue(pd);
+        tc_wait_st();
         tc_fence_before();
-      } else {
-        s_fault = 1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty(ab));
+        return true;
+      };
+
+      uint32_t i = it, tt = tj;
+      bool ok = true;
+      for (int j = 0; j < ntiles && ok; ++j, ++tt) {
+        const int ti = ti0 + j;
+        for (int c = 0; c < nch; ++c, ++i) {
+          const int st = (int)(i % kTcNumStages);
+          const int b = (int)(i % kTcNumABuf);
+          if (s_fault || !mbar_wait(stage_full(st), (i / kTcNumStages) & 1)) {
+            ok = false;
+            break;
+          }
+          if (i >= (uint32_t)kTcNumABuf &&
+              (s_fault || !mbar_wait(a_empty(b), ((i / kTcNumABuf) - 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int p0 = c * kTcChunkPlanes + 16 * half;  // first plane of this warp's K-step
+          if (p0 < P) {
+            const uint32_t *srow =
+                reinterpret_cast<const uint32_t *>(sStage + st * kTcStageBytes) + 16 * half * 32 + lane;
+            uint32_t cell[4][8];
+            if (!big) {
+#pragma unroll
+              for (int pr = 0; pr < 8; ++pr) {
+                const uint32_t x0 = srow[(2 * pr) * 32];
+                const uint32_t x1 = srow[(2 * pr + 1) * 32];
+                const uint32_t c0 = __byte_perm(x0, x1, 0x5410);  // keys kk = 0, 1
+                const uint32_t c1 = __byte_perm(x0, x1, 0x7632);  // keys kk = 2, 3
+                cell[0][pr] = c0 & m0;
+                cell[1][pr] = c1 & m0;
+                cell[2][pr] = c0 & m1;
+                cell[3][pr] = c1 & m1;
+              }
+            } else {
+#pragma unroll
+              for (int pr = 0; pr < 8; ++pr) {
+                const uint32_t x0 = srow[(2 * pr) * 32];
+                const uint32_t x1 = srow[(2 * pr + 1) * 32];
+                const uint32_t c0 = __byte_perm(x0, x1, 0x5410);
+                const uint32_t c1 = __byte_perm(x0, x1, 0x7632);
+                cell[0][pr] = (c0 >> quarter) & 0x01010101u;
+                cell[1][pr] = (c1 >> quarter) & 0x01010101u;
+                cell[2][pr] = (c0 >> (quarter + 4)) & 0x01010101u;
+                cell[3][pr] = (c1 >> (quarter + 4)) & 0x01010101u;
+              }
+            }
+            const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + b * kTcABufCols + 8 * half);
+#pragma unroll
+            for (int mb = 0; mb < 4; ++mb) tc_st8(acol + (uint32_t)(16 * mb), cell[mb]);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stage_empty(st));
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(a_full(b));
+        }
+        if (!ok) break;
+        // the previous tile's MMAs ran while this tile was being built
+        if (j > 0 && !epilogue(ti - 1, tt - 1)) ok = false;
       }
-      pending = false;
+      if (ok && !epilogue(ti0 + ntiles - 1, tj + ntiles - 1)) ok = false;
+      if (!ok) s_fault = 1;
     }
-    if (cur.ch == cur.nch - 1) {
-      pd = make_pending(cur, tile_seq & 1, it);
-      pending = true;
-      ++tile_seq;
-    }
-    __syncthreads();
-    if (nxt.t < 0) break;
-    cur = nxt;
-    nxt = iss;
-    iss = next_item(iss, cur.slot, nxt.slot);
-    ++it;
+    it += (uint32_t)(ntiles * nch);
+    tj += (uint32_t)ntiles;
+    t = seg_end;
   }
-  if (pending && !fault) {
-    if (tc_wait(mbar0 + 8 * (pd.item & 1), (pd.item >> 1) & 1)) {
-      tc_fence_after();
-      epilogue(pd);
-    } else {
-      s_fault = 1;
-    }
+
+  // ---- teardown ------------------------------------------------------------
+  // every commit must have landed before the block's barriers and tensor
+  // memory go away (on the normal path they have; after a fault, wait)
+  if (warp == kTcMmaWarp && lane == 0) {
+    if (last_item >= 0)
+      mbar_wait(a_empty(last_item % kTcNumABuf), ((uint32_t)last_item / kTcNumABuf) & 1);
+    if (last_tile >= 0) mbar_wait(acc_full(last_tile & 1), ((uint32_t)last_tile >> 1) & 1);
   }
   __syncthreads();
-  if (s_fault) fault = true;
-  asm volatile("cp.async.wait_all;\n" ::: "memory");
-  if (fault && tid == 0) atomicAdd(&p.status->device_faults, 1u);
+  if (s_fault && tid == 0) atomicAdd(&p.status->device_faults, 1u);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -809,8 +782,6 @@ static cudaError_t launch_tc_gm(const ScanParams &p, int sms, cudaStream_t strea
   cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<G, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  // one block per SM: each block holds 256 tensor-memory columns and more
-  // than half of the shared memory
   tc_scan_kernel<G, MODE><<<sms, kTcThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }

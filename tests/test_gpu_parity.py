@@ -293,6 +293,15 @@ def test_decode_1m(decode_1m, B):
     assert rep.fallback_heads == 0
 
 
+def test_decode_1m_tensor_cores(decode_1m):
+    """The tcgen05 scan on the 1M-token step (the benchmarked launch set)."""
+    _check_config(decode_1m, 92, 2048, heads_full={0, 21}, what="tc 1M",
+                  flags=F.FLAG_TENSOR_CORES)
+    rep = F.read_report()
+    assert rep.fallback_heads == 0
+    assert rep.device_faults == 0
+
+
 def test_host_resident_1m_budget_sweep():
     """Planes in pinned host memory: same results as device-resident planes,
     and oracle-checked, for every budget of the sweep."""
@@ -305,9 +314,17 @@ def test_host_resident_1m_budget_sweep():
         _, _, (idx_d, sc_d) = run_gpu(case, B, 2048)
         np.testing.assert_array_equal(idx_h, _np(idx_d))
         np.testing.assert_array_equal(sc_h, _np(sc_d))
+    # the tcgen05 scan reads host-resident planes too
+    idx_h, sc_h = _check_config(case, 92, 2048, heads_full={3}, what="tc host B=92",
+                                host_mapped=True, flags=F.FLAG_TENSOR_CORES)
+    _, _, (idx_d, sc_d) = run_gpu(case, 92, 2048, flags=F.FLAG_TENSOR_CORES)
+    np.testing.assert_array_equal(idx_h, _np(idx_d))
+    np.testing.assert_array_equal(sc_h, _np(sc_d))
 
 
-def test_ragged_32_sessions_batched():
+@pytest.mark.parametrize("tc", [False, True])
+def test_ragged_32_sessions_batched(tc):
+    flags = F.FLAG_TENSOR_CORES if tc else 0
     c = synthkv.CONFIGS["ragged_32_sessions"]
     sessions = synthkv.make_ragged(c["seed"], c["sessions"], c["n_lo"], c["n_hi"], c["h_kv"],
                                    c["h_q"], c["d"], c["q_dtype"], device="cuda")
@@ -322,8 +339,9 @@ def test_ragged_32_sessions_batched():
         descs.append(dict(planes=F.pack_planes(s.codes), qmin=s.qmin, qscale=s.qscale,
                           q=q_all[i * 32:(i + 1) * 32], alloc=alloc_all[i * 32:(i + 1) * 32],
                           n=s.n))
-    outs = F.scan_topk_batched(descs, k, 128, 32, 8, torch.bfloat16)
+    outs = F.scan_topk_batched(descs, k, 128, 32, 8, torch.bfloat16, flags=flags)
     torch.cuda.synchronize()
+    assert F.read_report().device_faults == 0
     want_alloc = oracle.allocate_heads(_np(q_all.float()).astype(np.float64), _np(sig_all), B)
     np.testing.assert_array_equal(_np(alloc_all), want_alloc)
     for i, s in enumerate(sessions):
