@@ -10,113 +10,101 @@
 // take the B most valuable, ties to the lower channel then lower tau.
 // t_c = channel c's slots taken.
 //
-// One warp per query head.  The water level is found without any log2: the
-// slot values are non-negative doubles, whose bit patterns order like the
-// values, so the warp bisects the 64-bit pattern space for the largest
-// level L with #{slots >= L} >= B (63 rounds of compare + warp-sum).  Slots
-// above L are taken; slots equal to L are taken in (channel, tau) order
-// until B is reached.  Every lane owns d/32 consecutive channels, so a warp
-// prefix sum orders the ties by channel.  Bit-exact with any other exact
-// evaluation of the same ordering: w_c is q*q times sigma*sigma in fp64
-// (both squares exact), and the slot values are exact power-of-two scalings.
+// One block per query head, one thread per slot (slot s = 4 c + tau, so the
+// thread order is the tie order).  The B-th most valuable slot value L is
+// found by an exact radix select over the 64-bit patterns of the slot values
+// (non-negative doubles order like their bit patterns): eight passes of an
+// 8-bit digit histogram.  Slots above L are taken; slots equal to L are taken
+// in slot order until B is reached (a block prefix count).  No log2 is
+// needed, and the result is bit-exact with any exact evaluation of the same
+// ordering: w_c is q*q times sigma*sigma in fp64 (both squares exact), and
+// the slot values are exact power-of-two scalings.
 #include "fathom_internal.cuh"
 
 namespace fathom {
 
-template <int CPL>
-__global__ void __launch_bounds__(128) allocate_kernel(const void *__restrict__ q, int q_bf16,
-                                                       const float *__restrict__ sigma, int h_q,
-                                                       int G, int budget,
-                                                       uint8_t *__restrict__ alloc) {
-  constexpr int d = CPL * 32;
-  const int h = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (h >= h_q) return;
-  const int g = h / G;
+__global__ void __launch_bounds__(1024) allocate_kernel(const void *__restrict__ q, int q_bf16,
+                                                        const float *__restrict__ sigma, int G,
+                                                        int d, int budget,
+                                                        uint8_t *__restrict__ alloc) {
+  const int h = blockIdx.x;
+  const int slot = threadIdx.x;  // 4 c + tau, slot < 4 d = blockDim.x
+  const int c = slot >> 2, tau = slot & 3;
+  const int lane = slot & 31, warp = slot >> 5;
+  __shared__ unsigned hist[256];
+  __shared__ unsigned s_warp[32];
+  __shared__ int s_digit;
+  __shared__ unsigned s_above;
 
-  unsigned long long key[CPL][4];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) {
-    const int c = lane * CPL + i;
-    const double qv = (double)load_q(q, q_bf16, (int64_t)h * d + c);
-    const double sv = (double)sigma[(int64_t)g * d + c];
-    const double w = (qv * qv) * (sv * sv);
-    key[i][0] = (unsigned long long)__double_as_longlong(w);
-    key[i][1] = (unsigned long long)__double_as_longlong(w * 0.25);
-    key[i][2] = (unsigned long long)__double_as_longlong(w * 0.0625);
-    key[i][3] = (unsigned long long)__double_as_longlong(w * 0.015625);
-  }
+  const double qv = (double)load_q(q, q_bf16, (int64_t)h * d + c);
+  const double sv = (double)sigma[(int64_t)(h / G) * d + c];
+  const double w = (qv * qv) * (sv * sv);
+  const double scale[4] = {1.0, 0.25, 0.0625, 0.015625};
+  const unsigned long long key = (unsigned long long)__double_as_longlong(w * scale[tau]);
 
-  int t[CPL];
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) t[i] = 0;
-
+  bool taken = false;
   if (budget > 0) {
-    // largest level L with #{slots >= L} >= budget
-    unsigned long long lo = 0ull, hi = 0x7ff0000000000000ull;
-    while (hi - lo > 1ull) {
-      const unsigned long long mid = lo + ((hi - lo) >> 1);
-      unsigned cnt = 0;
+    // radix select of the budget-th largest key, most significant digit first
+    unsigned long long prefix = 0ull, pmask = 0ull;
+    unsigned want = (unsigned)budget;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
+      __syncthreads();
+      if ((key & pmask) == prefix) atomicAdd(&hist[(unsigned)(key >> shift) & 255u], 1u);
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns bins 255 - 8 l ... 248 - 8 l (largest first)
+        unsigned local[8], sum = 0;
 #pragma unroll
-      for (int i = 0; i < CPL; ++i)
+        for (int i = 0; i < 8; ++i) {
+          local[i] = hist[255 - 8 * lane - i];
+          sum += local[i];
+        }
+        unsigned incl = sum;
 #pragma unroll
-        for (int tau = 0; tau < 4; ++tau) cnt += key[i][tau] >= mid ? 1u : 0u;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= (unsigned)budget) lo = mid; else hi = mid;
-    }
-    unsigned gt = 0, ties = 0;
+        for (int off = 1; off < 32; off <<= 1) {
+          const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const unsigned excl = incl - sum;
+        if (excl < want && want <= incl) {
+          unsigned run = excl;
 #pragma unroll
-    for (int i = 0; i < CPL; ++i)
-#pragma unroll
-      for (int tau = 0; tau < 4; ++tau) {
-        gt += key[i][tau] > lo ? 1u : 0u;
-        ties += key[i][tau] == lo ? 1u : 0u;
-      }
-    const unsigned rem = (unsigned)budget - __reduce_add_sync(0xffffffffu, gt);
-    // exclusive prefix of ties over lanes (lanes hold channels in order)
-    unsigned incl = ties;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    unsigned seen = incl - ties;
-#pragma unroll
-    for (int i = 0; i < CPL; ++i)
-#pragma unroll
-      for (int tau = 0; tau < 4; ++tau) {
-        if (key[i][tau] > lo) {
-          t[i] += 1;
-        } else if (key[i][tau] == lo) {
-          if (seen < rem) t[i] += 1;
-          seen += 1;
+          for (int i = 0; i < 8; ++i) {
+            if (run < want && want <= run + local[i]) {
+              s_digit = 255 - 8 * lane - i;
+              s_above = run;
+            }
+            run += local[i];
+          }
         }
       }
+      __syncthreads();
+      prefix |= (unsigned long long)s_digit << shift;
+      pmask |= 255ull << shift;
+      want -= s_above;
+      __syncthreads();
+    }
+    // prefix = L; `want` slots equal to L are still to be taken, in slot order
+    const bool eq = key == prefix;
+    const unsigned ballot = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) s_warp[warp] = (unsigned)__popc(ballot);
+    __syncthreads();
+    unsigned before = (unsigned)__popc(ballot & ((1u << lane) - 1u));
+    for (int i = 0; i < warp; ++i) before += s_warp[i];
+    taken = key > prefix || (eq && before < want);
   }
-#pragma unroll
-  for (int i = 0; i < CPL; ++i) alloc[(int64_t)h * d + lane * CPL + i] = (uint8_t)t[i];
+  // t_c = the taken slots of channel c: lanes 4 c .. 4 c + 3 of a warp
+  unsigned t = taken ? 1u : 0u;
+  t += __shfl_xor_sync(0xffffffffu, t, 1);
+  t += __shfl_xor_sync(0xffffffffu, t, 2);
+  if (tau == 0) alloc[(int64_t)h * d + c] = (uint8_t)t;
 }
 
 cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
                             int budget, uint8_t *alloc, cudaStream_t stream) {
   const int G = h_q / h_kv;
-  const dim3 grid((unsigned)((h_q + 3) / 4));
-  switch (d / 32) {
-#define FATHOM_ALLOC_CASE(C)                                                              \
-  case C:                                                                                 \
-    allocate_kernel<C><<<grid, 128, 0, stream>>>(q, q_bf16, sigma, h_q, G, budget, alloc); \
-    break;
-    FATHOM_ALLOC_CASE(1)
-    FATHOM_ALLOC_CASE(2)
-    FATHOM_ALLOC_CASE(3)
-    FATHOM_ALLOC_CASE(4)
-    FATHOM_ALLOC_CASE(5)
-    FATHOM_ALLOC_CASE(6)
-    FATHOM_ALLOC_CASE(7)
-    FATHOM_ALLOC_CASE(8)
-#undef FATHOM_ALLOC_CASE
-    default: return cudaErrorInvalidValue;
-  }
+  allocate_kernel<<<h_q, 4 * d, 0, stream>>>(q, q_bf16, sigma, G, d, budget, alloc);
   return cudaGetLastError();
 }
 

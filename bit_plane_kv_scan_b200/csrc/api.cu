@@ -259,6 +259,7 @@ fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_by
   p.G = a->h_q / a->h_kv;
   p.k = a->k;
   p.q_bf16 = a->q_dtype == FATHOM_BF16;
+  p.planes_host = a->planes_location == FATHOM_PLANES_HOST_MAPPED;
   p.flags = a->flags;
   p.debug_scores = a->debug_scores;
   fill_ws(p, L, ws);
@@ -312,6 +313,7 @@ fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, s
   p.G = a->h_q / a->h_kv;
   p.k = a->k;
   p.q_bf16 = a->q_dtype == FATHOM_BF16;
+  p.planes_host = a->planes_location == FATHOM_PLANES_HOST_MAPPED;
   p.flags = a->flags;
   p.debug_scores = nullptr;
   fill_ws(p, L, ws);

@@ -30,8 +30,6 @@ constexpr int kSectorWords = 8;
 constexpr int kSampleStride = 64;
 constexpr int kSampleSectorsPerTile = kTileWords / kSectorWords;  // 8
 constexpr int kMergeThreads = 1024;
-constexpr int64_t kThresholdSmemKeys = 40960;  // sampled keys staged in shared memory (160 KiB)
-constexpr int64_t kMergeSmemCand = 12288;      // candidates staged in shared memory (96 KiB)
 constexpr int kFallbackSlack = 2048;
 
 enum ScanMode { kModeSample = 0, kModeFilter = 1 };
@@ -109,6 +107,7 @@ struct ScanParams {
   int S;
   int d, h_q, h_kv, G, k;
   int q_bf16;
+  int planes_host;  // planes in pinned, mapped host memory
   uint32_t flags;
   int sample_rank;  // r: threshold = r-th largest sampled score
   int64_t cap;      // candidate capacity per query head

@@ -94,12 +94,9 @@ __device__ int block_inclusive_scan(int v, int *s_tmp) {
   return v;
 }
 
-// Adds one to hist[digit] for every lane with digit >= 0, one shared-memory
-// atomic per distinct digit in the warp.  All 32 lanes must call it.
-__device__ __forceinline__ void hist_add_warp(unsigned *hist, int digit) {
-  const unsigned peers = __match_any_sync(0xffffffffu, digit);
-  if (digit >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1)
-    atomicAdd(&hist[digit], (unsigned)__popc(peers));
+// Adds one to hist[digit] for every lane with digit >= 0.
+__device__ __forceinline__ void hist_add(unsigned *hist, int digit) {
+  if (digit >= 0) atomicAdd(&hist[digit], 1u);
 }
 
 // ------------------------------------------------------------ plan kernel --
@@ -584,6 +581,179 @@ __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
   cp_async_wait<0>();
 }
 
+// ---------------------------------------------------- select and sort --
+
+// 64-bit max / min written on 32-bit halves.
+__device__ __forceinline__ unsigned long long u64_max(unsigned long long a, unsigned long long b) {
+  return a > b ? a : b;
+}
+__device__ __forceinline__ unsigned long long u64_min(unsigned long long a, unsigned long long b) {
+  return a < b ? a : b;
+}
+
+// In-thread stages of the bitonic network for one size (strides 4, 2, 1):
+// thread t holds elements base .. base + 7.  For size <= 8 the direction
+// depends on the element, for larger sizes only on the thread.
+__device__ __forceinline__ void bitonic_regs(unsigned long long (&v)[8], int base, int size) {
+#pragma unroll
+  for (int st = 4; st >= 1; st >>= 1) {
+    if (st * 2 > size) continue;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if ((e & st) == 0) {
+        const bool desc = ((base + e) & size) == 0;
+        const unsigned long long a = v[e], b = v[e | st];
+        const unsigned long long hi = u64_max(a, b), lo = u64_min(a, b);
+        v[e] = desc ? hi : lo;
+        v[e | st] = desc ? lo : hi;
+      }
+    }
+  }
+}
+
+// Sorts s[0 .. m) descending (m a power of two, 256 <= m <= 8 blockDim.x).
+// Threads t < m / 8 hold elements 8 t .. 8 t + 7 in registers; the bitonic
+// network's exchanges run inside a thread (stride < 8), across lanes with
+// shuffles (stride < 256) and through shared memory only for the few
+// stages with stride >= 256.  Every thread of the block must call it.
+__device__ void block_sort_desc(unsigned long long *s, int m) {
+  constexpr int E = 8;
+  const int t = threadIdx.x;
+  const bool act = t < (m >> 3);
+  const int base = t * E;
+  unsigned long long v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = act ? s[base + e] : 0ull;
+  for (int size = 2; size <= m; size <<= 1) {
+    // strides >= 8: the pair direction depends only on the thread
+    for (int stride = size >> 1; stride >= E; stride >>= 1) {
+      const bool keep_max = ((base & stride) == 0) == ((base & size) == 0);
+      if (stride >= 32 * E) {
+        __syncthreads();  // earlier readers of s are done
+        if (act) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) s[base + e] = v[e];
+        }
+        __syncthreads();
+        if (act) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const unsigned long long o = s[(base + e) ^ stride];
+            v[e] = keep_max ? u64_max(v[e], o) : u64_min(v[e], o);
+          }
+        }
+      } else if (act) {  // whole warps are idle or active: m / 8 is a multiple of 32
+        const int ls = stride / E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[e], ls);
+          v[e] = keep_max ? u64_max(v[e], o) : u64_min(v[e], o);
+        }
+      }
+    }
+    if (act) bitonic_regs(v, base, size);
+  }
+  __syncthreads();
+  if (act) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) s[base + e] = v[e];
+  }
+  __syncthreads();
+}
+
+// Histogram select over float scores.  Scores are binned into kSelBins equal
+// bins between lo and hi (bin = (score - lo) * scale, monotone in the score).
+// block_hist_find returns the highest bin b such that at least `want` scores
+// lie in bins >= b (0 if there are fewer), and the count above b in *above.
+constexpr int kSelBins = 4096;
+
+__device__ __forceinline__ int sel_bin(float v, float lo, float scale) {
+  const int b = (int)((v - lo) * scale);
+  return b >= kSelBins ? kSelBins - 1 : b;
+}
+
+__device__ int block_hist_find(const unsigned *hist, unsigned want, unsigned *s_wsum, int *s_bin,
+                               unsigned *s_above) {
+  // warp w sums bins [128 w, 128 w + 128) counted from the top
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
+  constexpr int kPer = kSelBins / 32;
+  if (threadIdx.x == 0) {
+    *s_bin = 0;
+    *s_above = 0u;
+  }
+  for (int w = warp; w < 32; w += nw) {
+    unsigned loc = 0;
+#pragma unroll
+    for (int q = 0; q < kPer / 32; ++q) loc += hist[kSelBins - 1 - (w * kPer + q * 32 + lane)];
+    loc = __reduce_add_sync(0xffffffffu, loc);
+    if (lane == 0) s_wsum[w] = loc;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned ws = s_wsum[lane];
+    unsigned incl = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    const unsigned excl = incl - ws;
+    // the range (128 bins) holding the want-th score from the top
+    const unsigned own = __ballot_sync(0xffffffffu, excl < want && want <= incl);
+    if (own) {
+      const int r = __ffs(own) - 1;
+      unsigned run = __shfl_sync(0xffffffffu, excl, r);
+      // lane l takes bins j = 128 r + 4 l .. 4 l + 3 (from the top)
+      unsigned c4[kPer / 32], sum = 0;
+#pragma unroll
+      for (int q = 0; q < kPer / 32; ++q) {
+        c4[q] = hist[kSelBins - 1 - (r * kPer + lane * (kPer / 32) + q)];
+        sum += c4[q];
+      }
+      unsigned in2 = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, in2, off);
+        if (lane >= off) in2 += o;
+      }
+      run += in2 - sum;
+#pragma unroll
+      for (int q = 0; q < kPer / 32; ++q) {
+        if (run < want && want <= run + c4[q]) {
+          *s_bin = kSelBins - 1 - (r * kPer + lane * (kPer / 32) + q);
+          *s_above = run;
+        }
+        run += c4[q];
+      }
+    }
+  }
+  __syncthreads();
+  return *s_bin;
+}
+
+// Block-wide min and max of (lo, hi) over all threads; every thread gets them.
+__device__ __forceinline__ void block_minmax(float &lo, float &hi, float (*s_mm)[32]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+  }
+  if (lane == 0) {
+    s_mm[0][warp] = lo;
+    s_mm[1][warp] = hi;
+  }
+  __syncthreads();
+  lo = s_mm[0][0];
+  hi = s_mm[1][0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+    lo = fminf(lo, s_mm[0][w]);
+    hi = fmaxf(hi, s_mm[1][w]);
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------- threshold kernel --
 
 // Warp 0 finds the digit bin holding the want-th largest among 256 bins
@@ -620,55 +790,91 @@ __device__ __forceinline__ void find_bin_from_top(const unsigned *hist, unsigned
   }
 }
 
-__global__ void __launch_bounds__(512) threshold_kernel(ScanParams p, int smem_keys) {
-  extern __shared__ uint32_t s_keys[];  // [smem_keys]
+// Per head: a threshold that at least r of the sampled scores reach.  The
+// sampled scores are binned between their min and max; the threshold is the
+// smallest sampled score in the bins holding the r best, so it lies at or
+// just below the r-th best.  No threshold (0 = keep every key) when fewer
+// than r keys were sampled.  Up to kThrKeys keys a thread are held in
+// registers (the common case); larger samples are read from memory.
+constexpr int kThrKeys = 16;
+__global__ void __launch_bounds__(1024) threshold_kernel(ScanParams p) {
   const int64_t h = blockIdx.x;
   const int s = (int)(h / p.h_q);
   const int64_t n = session_of(p, s).n;
-  __shared__ unsigned hist[256];
-  __shared__ int s_digit;
+  __shared__ unsigned hist[kSelBins];
+  __shared__ unsigned s_wsum[32];
+  __shared__ float s_mm[2][32];
+  __shared__ int s_bin;
   __shared__ unsigned s_above;
+  __shared__ unsigned s_valid;
+  __shared__ unsigned s_minkey;
   if (!sampling_on(n, p.sample_rank, p.flags)) {
     if (threadIdx.x == 0) p.tau[h] = 0u;
     return;
   }
-  const int64_t m = sampled_sectors(n) * 256;
+  const int m = (int)(sampled_sectors(n) * 256);
   const uint32_t *keys = p.sample + h * p.m_max;
-  // the radix passes re-read every key; stage them in shared memory when
-  // they fit (one pass of independent loads instead of four dependent ones)
-  if (m <= smem_keys) {
-    for (int64_t i = threadIdx.x; i < m; i += blockDim.x) s_keys[i] = keys[i];
-    __syncthreads();
-    keys = s_keys;
+  const bool inreg = m <= kThrKeys * (int)blockDim.x;
+  // element (j, e) of a thread: key 4 (j blockDim + tid) + e
+  uint32_t kk[kThrKeys];
+  if (inreg) {
+#pragma unroll
+    for (int j = 0; j < kThrKeys / 4; ++j) {
+      const int b = 4 * (j * (int)blockDim.x + (int)threadIdx.x);
+      uint4 u = make_uint4(0u, 0u, 0u, 0u);
+      if (b < m) u = *reinterpret_cast<const uint4 *>(keys + b);  // m is a multiple of 256
+      kk[4 * j] = u.x;
+      kk[4 * j + 1] = u.y;
+      kk[4 * j + 2] = u.z;
+      kk[4 * j + 3] = u.w;
+    }
   }
-  uint32_t prefix = 0, pmask = 0;
-  unsigned want = (unsigned)p.sample_rank;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    if (threadIdx.x == 0) s_digit = -1;
-    __syncthreads();
-    for (int64_t base = 0; base < m; base += blockDim.x) {
-      const int64_t i = base + threadIdx.x;
-      int digit = -1;
-      if (i < m) {
-        const uint32_t k = keys[i];
-        if ((k & pmask) == prefix) digit = (int)((k >> shift) & 255u);
+  for (int i = threadIdx.x; i < kSelBins; i += blockDim.x) hist[i] = 0u;
+  if (threadIdx.x == 0) {
+    s_valid = 0u;
+    s_minkey = 0xffffffffu;
+  }
+  // range and count of the sampled scores (key 0 = no key sampled there)
+  float lo = INFINITY, hi = -INFINITY;
+  unsigned valid = 0;
+  auto visit = [&](auto &&fn) {
+    if (inreg) {
+#pragma unroll
+      for (int e = 0; e < kThrKeys; ++e)
+        if (kk[e] != 0u) fn(kk[e]);
+    } else {
+      for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const uint32_t x = keys[i];
+        if (x != 0u) fn(x);
       }
-      hist_add_warp(hist, digit);
     }
-    __syncthreads();
-    find_bin_from_top(hist, want, &s_digit, &s_above);
-    __syncthreads();
-    if (s_digit < 0) {  // fewer than r sampled keys: keep everything
-      if (threadIdx.x == 0) p.tau[h] = 0u;
-      return;
-    }
-    prefix |= (uint32_t)s_digit << shift;
-    pmask |= 255u << shift;
-    want -= s_above;
-    __syncthreads();
+  };
+  visit([&](uint32_t x) {
+    const float v = key_float(x);
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
+    ++valid;
+  });
+  valid = __reduce_add_sync(0xffffffffu, valid);
+  if ((threadIdx.x & 31) == 0) atomicAdd(&s_valid, valid);
+  block_minmax(lo, hi, s_mm);
+  if (s_valid < (unsigned)p.sample_rank) {  // too few samples: keep every key
+    if (threadIdx.x == 0) p.tau[h] = 0u;
+    return;
   }
-  if (threadIdx.x == 0) p.tau[h] = prefix;
+  const float scale = hi > lo ? (float)kSelBins / (hi - lo) : 0.0f;
+  visit([&](uint32_t x) { atomicAdd(&hist[sel_bin(key_float(x), lo, scale)], 1u); });
+  __syncthreads();
+  const int bstar = block_hist_find(hist, (unsigned)p.sample_rank, s_wsum, &s_bin, &s_above);
+  // smallest sampled key in bins >= bstar
+  unsigned mk = 0xffffffffu;
+  visit([&](uint32_t x) {
+    if (sel_bin(key_float(x), lo, scale) >= bstar) mk = min(mk, x);
+  });
+  mk = __reduce_min_sync(0xffffffffu, mk);
+  if ((threadIdx.x & 31) == 0) atomicMin(&s_minkey, mk);
+  __syncthreads();
+  if (threadIdx.x == 0) p.tau[h] = s_minkey;
 }
 
 // ---------------------------------------------------------- merge kernel --
@@ -689,7 +895,7 @@ __device__ unsigned long long block_kth(const unsigned long long *a, int64_t cnt
         const unsigned long long v = a[i];
         if ((v & pmask) == prefix) digit = (int)((unsigned)(v >> shift) & 255u);
       }
-      hist_add_warp(hist, digit);
+      hist_add(hist, digit);
     }
     __syncthreads();
     find_bin_from_top(hist, want, s_digit, s_above);
@@ -778,13 +984,31 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   return (int64_t)s_nbuf;
 }
 
+// One block per head (kMergeThreads = 1024 threads).  Usually the
+// candidates fit in registers (kMergeKeys a thread): they are binned by score
+// (kSelBins equal bins between their min and max, monotone in the score) and
+// the bin b holding the k-th best is found; the candidates from b up are
+// binned again over their own, narrower range, so that a bin holds a handful
+// of keys.  They are placed bin by bin from the top (a counting sort); then
+// each candidate's place inside its bin is its rank there (the count of
+// larger composites in the bin: descending composite = score desc, index
+// asc).  The first k are the answer.  Crowded bins fall back to a register
+// bitonic sort; more candidates than fit take an exact radix select.
+constexpr int kMergeKeys = 8;
+constexpr int kBinSortMax = 256;
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int kpow2,
-                                                              int smem_cand) {
-  extern __shared__ unsigned long long s_sort[];  // [kpow2], then [smem_cand] staged candidates
-  __shared__ unsigned hist[256];
-  __shared__ int s_digit;
+                                                              int sort_cap) {
+  // [sort_cap] placed candidates, then [sort_cap] ranked (sort_cap = 8 blockDim >= kpow2)
+  extern __shared__ unsigned long long s_out[];
+  unsigned long long *s_rank = s_out + sort_cap;
+  __shared__ unsigned hist[kSelBins];
+  __shared__ unsigned s_off[kSelBins];
+  __shared__ unsigned s_wsum[32];
+  __shared__ float s_mm[2][32];
+  __shared__ int s_bin;
   __shared__ unsigned s_above;
   __shared__ unsigned s_fill;
+  __shared__ int s_crowded;
   const int64_t h = blockIdx.x;
   const int s = (int)(h / p.h_q);
   const int hl = (int)(h - (int64_t)s * p.h_q);
@@ -798,55 +1022,152 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
   const bool ok = cnt <= p.cap && (tauk == 0u || cnt >= need) &&
                   !(p.flags & FATHOM_FLAG_FORCE_FALLBACK);
   if (!ok) {
-    cnt = fallback_head(p, s, hl, buf, s_sort, hist, &s_digit, &s_above);
+    cnt = fallback_head(p, s, hl, buf, s_out, hist, &s_bin, &s_above);
     if (threadIdx.x == 0) atomicAdd(&p.status->fallback_heads, 1u);
   }
-  if (threadIdx.x == 0)
+  if (threadIdx.x == 0) {
     atomicMax(&p.status->max_candidates, (unsigned)(cnt < 0xffffffffll ? cnt : 0xffffffffll));
-  // the radix passes re-read every candidate; stage them in shared memory
-  // when they fit
-  if (cnt <= smem_cand) {
-    unsigned long long *staged = s_sort + kpow2;
-    for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) staged[i] = buf[i];
-    __syncthreads();
-    buf = staged;
+    s_crowded = 0;
   }
   const int take = (int)(cnt < k ? cnt : k);
-  unsigned long long bar = 0ull;
-  if (cnt > k) bar = block_kth(buf, cnt, (unsigned)k, hist, &s_digit, &s_above);
-  if (threadIdx.x == 0) s_fill = 0;
-  __syncthreads();
-  for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
-    const unsigned long long v = buf[i];
-    if (v >= bar) {
-      const unsigned at = atomicAdd(&s_fill, 1u);
-      if (at < (unsigned)take) s_sort[at] = v;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthr = blockDim.x;
+  int nsort = 0;  // > 0: sort s_out[0 .. nsort) with the bitonic network
+  if (cnt <= k) {
+    for (int i = tid; i < cnt; i += nthr) s_out[i] = buf[i];
+    nsort = (int)cnt;
+  } else if (cnt <= (int64_t)kMergeKeys * nthr) {
+    // candidate j * blockDim + tid of this thread, 0 when absent
+    unsigned long long c[kMergeKeys];
+    float lo = INFINITY, hi = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kMergeKeys; ++j) {
+      const int i = j * nthr + tid;
+      c[j] = i < cnt ? buf[i] : 0ull;
     }
-  }
-  for (int i = take + threadIdx.x; i < kpow2; i += blockDim.x) s_sort[i] = 0ull;
-  __syncthreads();
-  // bitonic sort, descending
-  for (int size = 2; size <= kpow2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < kpow2; i += blockDim.x) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool desc = (i & size) == 0;
-          const unsigned long long a = s_sort[i], b = s_sort[j];
-          if (desc ? (a < b) : (a > b)) {
-            s_sort[i] = b;
-            s_sort[j] = a;
-          }
+#pragma unroll
+    for (int j = 0; j < kMergeKeys; ++j) {
+      if (c[j] != 0ull) {
+        const float v = key_float((uint32_t)(c[j] >> 32));
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+      }
+    }
+    for (int i = tid; i < kSelBins; i += nthr) hist[i] = 0u;
+    block_minmax(lo, hi, s_mm);  // its barriers also order the clearing
+    const float scale = hi > lo ? (float)kSelBins / (hi - lo) : 0.0f;
+    int bin[kMergeKeys];
+#pragma unroll
+    for (int j = 0; j < kMergeKeys; ++j) {
+      bin[j] = -1;
+      if (c[j] != 0ull) {
+        bin[j] = sel_bin(key_float((uint32_t)(c[j] >> 32)), lo, scale);
+        atomicAdd(&hist[bin[j]], 1u);
+      }
+    }
+    __syncthreads();
+    int bstar = block_hist_find(hist, (unsigned)k, s_wsum, &s_bin, &s_above);
+    // second level: rebin the candidates of bins >= bstar over [their min, hi]
+    {
+      float lo2 = INFINITY, hi2 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kMergeKeys; ++j)
+        if (bin[j] >= bstar) lo2 = fminf(lo2, key_float((uint32_t)(c[j] >> 32)));
+      for (int i = tid; i < kSelBins; i += nthr) hist[i] = 0u;
+      block_minmax(lo2, hi2, s_mm);
+      const float scale2 = hi > lo2 ? (float)kSelBins / (hi - lo2) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < kMergeKeys; ++j) {
+        if (bin[j] >= bstar) {
+          bin[j] = sel_bin(key_float((uint32_t)(c[j] >> 32)), lo2, scale2);
+          atomicAdd(&hist[bin[j]], 1u);
+        } else {
+          bin[j] = -1;
         }
       }
       __syncthreads();
+      bstar = block_hist_find(hist, (unsigned)k, s_wsum, &s_bin, &s_above);
     }
+    // exclusive offsets of the bins in top order: thread t owns top-order
+    // positions 4 t .. 4 t + 3 (bins kSelBins - 1 - 4 t - q)
+    {
+      unsigned cq[4], sum = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        cq[q] = hist[kSelBins - 1 - (4 * tid + q)];
+        sum += cq[q];
+      }
+      unsigned incl = sum;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (lane == 31) s_wsum[warp] = incl;
+      __syncthreads();
+      unsigned base = incl - sum;
+      for (int w = 0; w < warp; ++w) base += s_wsum[w];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        s_off[kSelBins - 1 - (4 * tid + q)] = base;
+        base += cq[q];
+      }
+    }
+    __syncthreads();
+    // counting-sort placement of the candidates of bins >= bstar
+#pragma unroll
+    for (int j = 0; j < kMergeKeys; ++j)
+      if (bin[j] >= bstar) s_out[atomicAdd(&s_off[bin[j]], 1u)] = c[j];
+    __syncthreads();
+    // s_off[b] is now the end of bin b's run: rank each candidate in its run
+#pragma unroll
+    for (int j = 0; j < kMergeKeys; ++j) {
+      if (bin[j] >= bstar) {
+        const int e = (int)s_off[bin[j]], nb = (int)hist[bin[j]];
+        const int b0 = e - nb;
+        if (nb > kBinSortMax) {
+          s_crowded = 1;
+        } else if (b0 < k) {
+          int r = 0;
+          for (int i = b0; i < e; ++i) r += s_out[i] > c[j] ? 1 : 0;
+          s_rank[b0 + r] = c[j];
+        }
+      }
+    }
+    __syncthreads();
+    if (s_crowded) {
+      nsort = (int)s_off[bstar];  // every candidate of bins >= bstar
+    } else {
+      for (int i = tid; i < take; i += nthr) s_out[i] = s_rank[i];
+    }
+  } else {
+    // more candidates than the registers hold: exact radix select of the k-th
+    const unsigned long long bar = block_kth(buf, cnt, (unsigned)k, hist, &s_bin, &s_above);
+    if (tid == 0) s_fill = 0u;
+    __syncthreads();
+    for (int64_t i = tid; i < cnt; i += nthr) {
+      const unsigned long long v = buf[i];
+      if (v >= bar) {
+        const unsigned at = atomicAdd(&s_fill, 1u);
+        if (at < (unsigned)take) s_out[at] = v;
+      }
+    }
+    nsort = take;
   }
-  for (int r = threadIdx.x; r < k; r += blockDim.x) {
+  if (nsort > 0) {
+    int mp = 256;
+    while (mp < nsort) mp <<= 1;
+    __syncthreads();
+    for (int i = nsort + tid; i < mp; i += nthr) s_out[i] = 0ull;
+    __syncthreads();
+    block_sort_desc(s_out, mp);
+  }
+  __syncthreads();
+  for (int r = tid; r < k; r += nthr) {
     int32_t idx = -1;
     float sc = -INFINITY;
     if (r < take) {
-      const unsigned long long v = s_sort[r];
+      const unsigned long long v = s_out[r];
       idx = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
       sc = key_float((uint32_t)(v >> 32));
     }
@@ -922,11 +1243,7 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
   if (any_sampling) {
     e = tc ? launch_tc_scan(p, kModeSample, sms, stream) : launch_scan_m<kModeSample>(p, stream);
     if (e != cudaSuccess) return e;
-    const int64_t tkeys = p.m_max < kThresholdSmemKeys ? p.m_max : kThresholdSmemKeys;
-    const int tsmem = (int)(tkeys * 4);
-    e = cudaFuncSetAttribute(threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tsmem);
-    if (e != cudaSuccess) return e;
-    threshold_kernel<<<heads, 512, tsmem, stream>>>(p, (int)tkeys);
+    threshold_kernel<<<heads, 1024, 0, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -940,16 +1257,15 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
     e = cudaEventRecord(p.prof_end, stream);
     if (e != cudaSuccess) return e;
   }
-  int kpow2 = 1;
+  int kpow2 = 256;
   while (kpow2 < p.k) kpow2 <<= 1;
-  // room for about twice the expected candidate count (~2k per head)
-  int64_t mcand = 4 * (int64_t)p.k + 1024;
-  if (mcand > p.cap) mcand = p.cap;
-  if (mcand > kMergeSmemCand) mcand = kMergeSmemCand;
-  const int msmem = (int)((kpow2 + mcand) * 8);
+  // the k winners and the k-th best's histogram bin are sorted in registers:
+  // up to 8 per thread
+  const int sort_cap = 8 * kMergeThreads;
+  const int msmem = 2 * sort_cap * 8;
   e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
   if (e != cudaSuccess) return e;
-  merge_kernel<<<heads, kMergeThreads, msmem, stream>>>(p, kpow2, (int)mcand);
+  merge_kernel<<<heads, kMergeThreads, msmem, stream>>>(p, kpow2, sort_cap);
   return cudaGetLastError();
 }
 
