@@ -7,7 +7,7 @@
 //   s_h(i) = C_h + sum_{(c, j): j < t_hc} W_hcj b_cj(i),   W_hcj = q_hc s_c 2^(3 - j),
 //   C_h    = sum_c q_hc (m_c + s_c (2^(4 - t_hc) - 1) / 2),
 // b_cj(i) the bit of plane j of channel c for key i.  For the G query heads of
-// one KV head this is one matrix product over the union planes of the group:
+// one KV head this is one matrix product over the P union planes of the group:
 //   A [keys x planes] = the plane bits,
 //   B [planes x (head, digit)] = W_hcj / Delta_h as a 30-bit fixed-point
 //     integer in four signed base-256 int8 digits (0 where the head does not
@@ -15,61 +15,74 @@
 // accumulated exactly in int32 by the tensor cores; the epilogue forms
 //   s_h = C_h + Delta_h sum_m 256^m acc_m.
 //
-// Layout (B200 design).  A 1024-key tile of one KV head is 32 plane words per
-// plane.  Tensor-memory lane (quarter q, lane l) of M-block (hr, e) stands for
-// word l of the tile and bit position r = q + 4 hr of every byte of that word;
-// the four bytes of its 32-bit column hold, for a pair of planes (p, p'), the
-// bits of keys 8 kk + r for kk = 2e, 2e + 1:
-//   cell = byte_perm(P_p, P_p', e ? 0x7632 : 0x5410) & (0x01010101 << r)
-// (one permute per plane pair and one AND per cell, each byte 0 or 2^r).  The
-// two keys in a cell are separated by B: its 32 columns are (kk', head, digit)
-// and a column reads only the bytes of its kk'.  The 2^r of a lane is undone
-// in the epilogue.
+// Layout (B200 design).  A tile is 1024 keys of one KV head: 32 plane words
+// per plane.  Tensor-memory lane (quarter q, lane l) of M-block r (r < 8)
+// stands for key 32 l + 8 q + r of the tile: word l, byte q, bit r.  Plane
+// rows are taken four at a time; the warp of lane quarter q gathers byte q
+// of the four words of its lane with three byte permutes,
+//   T = [x0.byte q, x1.byte q, x2.byte q, x3.byte q],
+// and M-block r receives the 32-bit cell T & (0x01010101 << r): four int8 K
+// elements, one per plane, each 0 or 2^r (undone by the epilogue's scale).
+// Every key has its own row and B has N = 16 columns (head, digit).
 //
-// Roles (10 warps): warp 8 stages 32 plane rows of a tile ("chunk") into
-// shared memory with 16-byte cp.async copies; warps 0-7 turn a chunk into
-// tensor-memory cells (warp w: lane quarter w % 4, half the chunk's planes)
-// and, one tile later, read the tile's accumulators back, score and filter
-// them; one thread of warp 9 issues the MMAs.  They hand chunks, A buffers
-// and accumulators to each other through mbarriers; every wait is bounded in
-// time and a timeout records a device fault in the workspace status.
+// Work split (measured on B200: one thread issues a tcgen05.mma only every
+// ~46 cycles, an mbarrier round trip costs 100-200 cycles, and bulk copies of
+// 128-byte row pieces are limited by their per-copy cost):
+//  * A chunk is 64 plane rows of a tile.  The eight build warps load it
+//    themselves with 16-byte global loads (warp w: rows 8 w .. 8 w + 7),
+//    eight chunks ahead in registers, stage it in shared memory, and
+//    synchronise with named barriers only.
+//  * Warp w (lane quarter w % 4, plane groups 8 (w / 4) .. + 7, i.e. K-step
+//    w / 4 of the chunk) writes its 64 cells per lane to tensor memory in two
+//    32-column stores (A buffer columns: K-step, then M-block, then group);
+//    after a barrier, warp w issues the two MMAs of
+//    M-block w (two K-steps of 32 planes) and commits them: eight issuers,
+//    and every accumulator region always fed by the same thread.
+//  * Warps 8-11 read a finished tile's accumulators back, score, and collect
+//    the keys above the head's threshold in shared memory, flushing them to
+//    the candidate buffer with one global atomic per flush.
 // Accumulators are preset to the bits of 1.5 * 2^23, so that an accumulator
-// read back as a float is 1.5 * 2^23 + acc exactly (|acc| <= 2^22).
+// read back as a float is 1.5 * 2^23 + acc exactly (|acc| <= 2^22).  When
+// P > 256 the cells hold 0/1 instead of 0/2^r so that acc stays within 2^22.
+// Every mbarrier wait is bounded in time; a timeout records a device fault in
+// the workspace status.
 #include "fathom_internal.cuh"
 
 namespace fathom {
 
 // ---------------------------------------------------------------- layout --
 constexpr int kTcTileWords = 32;                        // 1024 keys per tile
-constexpr int kTcChunkPlanes = 32;                      // plane rows per chunk
-constexpr int kTcStageBytes = kTcChunkPlanes * kTcTileWords * 4;  // 4 KiB
-constexpr int kTcNumStages = 16;                        // chunks staged ahead
-constexpr int kTcNumABuf = 4;                           // A buffers in tensor memory
+constexpr int kTcChunkPlanes = 64;                      // plane rows per chunk
+constexpr int kTcKStep = 32;                            // planes per MMA (K = 32 int8)
+constexpr int kTcStageBytes = kTcChunkPlanes * kTcTileWords * 4;  // 8 KiB
 constexpr int kTcBuildWarps = 8;
-constexpr int kTcProducerWarp = 8;
-constexpr int kTcMmaWarp = 9;
-constexpr int kTcThreads = 10 * 32;
-constexpr int kTcAccCols = 4 * 32;                      // one tile: 4 M-blocks x N = 32
-constexpr int kTcABufCols = 4 * 16;                     // one chunk: 4 M-blocks x 16 columns
-constexpr int kTcTmemCols = 512;                        // 2 x 128 accumulators + 4 x 64 A
+constexpr int kTcEpiWarp0 = 8;                          // warps 8-11
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcThreads = (kTcBuildWarps + kTcEpiWarps) * 32;
+constexpr int kTcLoadAhead = 8;                         // chunks in flight per build warp
+constexpr int kTcMBlocks = 8;                           // one per bit position r
+constexpr int kTcN = 16;                                // (head, digit) columns
+constexpr int kTcAccCols = kTcMBlocks * kTcN;           // 128: one tile's accumulators
+constexpr int kTcABufCols = kTcMBlocks * (kTcChunkPlanes / 4);  // 128: one chunk's cells
+constexpr int kTcTmemCols = 512;                        // 2 x 128 accumulators + 2 x 128 A
 constexpr int kTcAColBase = 2 * kTcAccCols;
 constexpr int kTcSampleSectorsPerTile = kTcTileWords / kSectorWords;  // 4
-// B for one K-step (16 planes = 8 columns = 32 int8 K elements): 32 rows
-// (kk', head, digit) x 32 bytes, K-major, no swizzle.  Core matrices are
-// 8 rows x 16 bytes; 8-row groups are 128 B apart (SBO), the two 16-byte K
-// halves 512 B apart (LBO).
-constexpr int kTcKStepBytes = 1024;
+constexpr int kTcCandBuf = 64;                          // candidates buffered per epilogue warp and head
+// B for one K-step: 16 rows (head, digit) x 32 int8 K elements (planes),
+// K-major, no swizzle.  Core matrices are 8 rows x 16 bytes; the two 8-row
+// groups are 128 B apart (SBO), the two 16-byte K halves 256 B apart (LBO).
+constexpr int kTcBChunkBytes = 512;  // per K-step of 32 planes
 constexpr uint32_t kTcSBO = 128;
-constexpr uint32_t kTcLBO = 512;
+constexpr uint32_t kTcLBO = 256;
 // Instruction descriptor: D s32, A u8 K-major (tensor memory), B s8
-// K-major, N = 32, M = 128, dense.
-constexpr uint32_t kTcIdesc = (2u << 4)             // D format s32
-                              | (0u << 7)           // A format u8
-                              | (1u << 10)          // B format s8
-                              | (0u << 15)          // A K-major
-                              | (0u << 16)          // B K-major
-                              | ((32u >> 3) << 17)  // N
-                              | ((128u >> 4) << 24);  // M
+// K-major, N = 16, M = 128, dense.
+constexpr uint32_t kTcIdesc = (2u << 4)                 // D format s32
+                              | (0u << 7)               // A format u8
+                              | (1u << 10)              // B format s8
+                              | (0u << 15)              // A K-major
+                              | (0u << 16)              // B K-major
+                              | ((uint32_t)(kTcN >> 3) << 17)  // N
+                              | ((128u >> 4) << 24);    // M
 constexpr uint32_t kTcMagicBits = 0x4b400000u;  // 1.5 * 2^23
 constexpr float kTcMagic = 12582912.0f;
 // A plane count above which the cells hold 0/1 instead of 0/2^r, so that an
@@ -78,7 +91,7 @@ constexpr int kTcSmallP = 256;
 
 struct TcPlanHeader {
   int P;       // union planes of the group
-  int nchunk;  // ceil(P / 32)
+  int nks;     // max(1, ceil(P / 32)): K-steps of 32 planes with a B block
   int pad0, pad1;
   float K[4];  // C_h
   float D[4];  // Delta_h (a power of two)
@@ -88,7 +101,7 @@ static_assert(sizeof(TcPlanHeader) == 64, "header size");
 
 struct TcPlanLayout {
   int off_rows;  // uint16 [4 d]: c * 4 + j of every union plane, channel-major
-  int off_b;     // int8 [ceil(4 d / 16)][1024]
+  int off_b;     // int8 [ceil(4 d / 32)][512]: B of every K-step
   int bytes;
 };
 
@@ -96,14 +109,15 @@ __host__ __device__ inline TcPlanLayout tc_plan_layout(int d) {
   TcPlanLayout L;
   L.off_rows = (int)sizeof(TcPlanHeader);
   L.off_b = align16(L.off_rows + 2 * 4 * d);
-  L.bytes = L.off_b + ((4 * d + 15) / 16) * kTcKStepBytes;
+  L.bytes = L.off_b + ((4 * d + kTcKStep - 1) / kTcKStep) * kTcBChunkBytes;
   return L;
 }
 
 int tc_plan_bytes(int d) { return tc_plan_layout(d).bytes; }
 
 static int tc_smem_bytes(int d, int S) {
-  int b = 128 + kTcNumStages * kTcStageBytes + tc_plan_layout(d).bytes + 4 * (S + 1);
+  int b = 128 + 2 * kTcStageBytes + tc_plan_layout(d).bytes + 4 * (S + 1) +
+          kTcEpiWarps * 4 * kTcCandBuf * 8;
   // more than half an SM's shared memory: one block per SM, so that the
   // block's 512 tensor-memory columns never wait for another block
   return b < 120 * 1024 ? 120 * 1024 : b;
@@ -113,12 +127,6 @@ static int tc_smem_bytes(int d, int S) {
 
 __device__ __forceinline__ uint32_t tc_smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void tc_cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
 }
 
 __device__ __forceinline__ uint64_t tc_smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -142,35 +150,34 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
       "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n" ::"r"(bar)
       : "memory");
 }
-// Arrives on bar once all of this thread's earlier cp.async copies are done.
-__device__ __forceinline__ void mbar_arrive_cp_async(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
-}
 
 // Waits for the completion of the phase of bar with the given parity, giving
-// up after about a second (2^31 cycles).  Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// up after about a second (2^31 cycles).  Returns false on timeout.  Each
+// try_wait may suspend the thread for up to 0.1 ms until the phase completes,
+// so a waiting warp takes no issue slots from the working ones.
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, P;\n\t}\n"
       : "=r"(done)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(100000u)
       : "memory");
-  if (done) return true;
+  return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    asm volatile(
-        "{\n\t.reg .pred P;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
-        "selp.b32 %0, 1, 0, P;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (done) return true;
+    if (mbar_try(bar, parity)) return true;
     if (clock64() - t0 > (1ll << 31)) return false;
   }
+}
+
+// Named barrier among the `count` threads of the build warps.
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc) {
@@ -196,13 +203,16 @@ __device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&v)[8]) {
       : "memory");
 }
 
-// Writes the value x into 32 consecutive columns of this warp's lanes.
-__device__ __forceinline__ void tc_st32_fill(uint32_t taddr, uint32_t x) {
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};\n" ::"r"(
-          taddr),
-      "r"(x)
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};\n" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 
@@ -309,10 +319,10 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   if (threadIdx.x == blockDim.x - 1) s_P = incl;
   __syncthreads();
   const int P = s_P;
-  const int nks = (P + 15) / 16;
-  // B of every used K-step starts at zero (padding planes, heads that do not
-  // read a plane, and the other key of every cell contribute nothing)
-  for (int i = threadIdx.x; i < nks * kTcKStepBytes / 16; i += blockDim.x)
+  const int nks = P > 0 ? (P + kTcKStep - 1) / kTcKStep : 1;
+  // B of every used K-step starts at zero (padding planes and heads that do
+  // not read a plane contribute nothing)
+  for (int i = threadIdx.x; i < nks * kTcBChunkBytes / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(bmat)[i] = make_uint4(0, 0, 0, 0);
   double delta[4];
   for (int hh = 0; hh < 4; ++hh) {
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   }
   if (threadIdx.x == 0) {
     hdr->P = P;
-    hdr->nchunk = (P + kTcChunkPlanes - 1) / kTcChunkPlanes;
+    hdr->nks = nks;
     hdr->pad0 = hdr->pad1 = 0;
     const int nw = (blockDim.x + 31) >> 5;
     for (int hh = 0; hh < 4; ++hh) {
@@ -340,19 +350,16 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   for (int j = 0; j < tstar; ++j) {
     const int pl = off + j;
     rows[pl] = (uint16_t)(c * 4 + j);
-    int8_t *bk = bmat + (size_t)(pl >> 4) * kTcKStepBytes;
-    const int col = (pl & 15) >> 1, pp = pl & 1;
+    int8_t *bk = bmat + (size_t)(pl / kTcKStep) * kTcBChunkBytes;
+    const int k = pl % kTcKStep;
     for (int hh = 0; hh < G; ++hh) {
       if (j >= t[hh]) continue;
       long long x = llrint(ldexp(w[hh], 3 - j) / delta[hh]);
       for (int dg = 0; dg < 4; ++dg) {
         const long long v = dg < 3 ? ((x + 128) & 255) - 128 : x;
         x = (x - v) >> 8;
-        for (int kq = 0; kq < 2; ++kq) {
-          const int n = kq * 16 + hh * 4 + dg;
-          const int k = 4 * col + 2 * pp + kq;
-          bk[(n >> 3) * kTcSBO + (k >> 4) * kTcLBO + (n & 7) * 16 + (k & 15)] = (int8_t)v;
-        }
+        const int n = hh * 4 + dg;
+        bk[(n >> 3) * kTcSBO + (k >> 4) * kTcLBO + (n & 7) * 16 + (k & 15)] = (int8_t)v;
       }
     }
   }
@@ -395,6 +402,56 @@ __device__ __forceinline__ TcLoc tc_locate(const ScanParams &p, const int *s_tpr
   return L;
 }
 
+// Writes the n buffered candidates of one head to the candidate buffer: one
+// global atomic reserves their places.  All lanes of the warp call it.  Out
+// of line: it runs about once per 64 candidates, and the scoring loop keeps
+// its registers and schedule.
+__device__ __noinline__ void tc_flush(const ScanParams &p, int64_t head,
+                                      const unsigned long long *buf, unsigned n) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  unsigned base = 0;
+  if (lane == 0) base = atomicAdd(&p.counts[head], n);
+  base = __shfl_sync(0xffffffffu, base, 0);
+  unsigned long long *dst = p.cand + head * p.cap;
+  for (unsigned i = lane; i < n; i += 32) {
+    const int64_t pos = (int64_t)base + i;
+    if (pos < p.cap) dst[pos] = buf[i];
+  }
+  __syncwarp();
+}
+
+// Appends this warp's candidates among keys tk, tk + 1 (bit 2 h + k of cm:
+// key tk + k clears head h's threshold, score s[2 h + k]) to the warp's
+// per-head buffers (fill[h] entries used), flushing a buffer before it
+// overflows.  All lanes call it; out of line, since it is the rare path.
+__device__ __noinline__ void tc_append(const ScanParams &p, int64_t head0, int G,
+                                       unsigned long long *cbuf, unsigned *fill, uint32_t cm,
+                                       int tk, float s0, float s1, float s2, float s3, float s4,
+                                       float s5, float s6, float s7) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  const float sv[8] = {s0, s1, s2, s3, s4, s5, s6, s7};
+  for (int h = 0; h < G; ++h) {
+    const bool t0 = (cm >> (2 * h)) & 1u, t1 = (cm >> (2 * h + 1)) & 1u;
+    const unsigned b0 = __ballot_sync(0xffffffffu, t0);
+    const unsigned b1 = __ballot_sync(0xffffffffu, t1);
+    if (!(b0 | b1)) continue;
+    const unsigned nn = (unsigned)(__popc(b0) + __popc(b1));
+    unsigned f = fill[h];
+    unsigned long long *cb = cbuf + h * kTcCandBuf;
+    if (f + nn > (unsigned)kTcCandBuf) {
+      tc_flush(p, head0 + h, cb, f);
+      f = 0u;
+    }
+    if (t0) cb[f + __popc(b0 & lt)] = composite(sv[2 * h], (uint32_t)tk);
+    if (t1) cb[f + __popc(b0) + __popc(b1 & lt)] = composite(sv[2 * h + 1], (uint32_t)(tk + 1));
+    __syncwarp();
+    if (lane == 0) fill[h] = f + nn;
+    __syncwarp();
+  }
+}
+
 template <int G, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -404,23 +461,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const int d = p.d;
   const TcPlanLayout PL = tc_plan_layout(d);
   unsigned char *sStage = smem;
-  unsigned char *sPlan = smem + kTcNumStages * kTcStageBytes;
+  unsigned char *sPlan = smem + 2 * kTcStageBytes;
+  unsigned long long *sCand = reinterpret_cast<unsigned long long *>(sPlan + PL.bytes);
+  int *s_tprefix = reinterpret_cast<int *>(sCand + kTcEpiWarps * 4 * kTcCandBuf);
   const TcPlanHeader *sHdr = reinterpret_cast<const TcPlanHeader *>(sPlan);
   const uint16_t *sRows = reinterpret_cast<const uint16_t *>(sPlan + PL.off_rows);
-  int *s_tprefix = reinterpret_cast<int *>(sPlan + PL.bytes);
-  __shared__ __align__(8) unsigned long long s_bar[2 * kTcNumStages + 2 * kTcNumABuf + 4];
+  __shared__ __align__(8) unsigned long long s_bar[6];
   __shared__ uint32_t s_tmem;
   __shared__ int s_tmp[32];
   __shared__ volatile int s_fault;
+  __shared__ unsigned s_fill[kTcEpiWarps][4];  // candidates buffered per epilogue warp and head
 
   const uint32_t bar0 = tc_smem_u32(&s_bar[0]);
-  auto stage_full = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  auto stage_empty = [&](int i) { return bar0 + 8u * (uint32_t)(kTcNumStages + i); };
-  auto a_full = [&](int i) { return bar0 + 8u * (uint32_t)(2 * kTcNumStages + i); };
-  auto a_empty = [&](int i) { return bar0 + 8u * (uint32_t)(2 * kTcNumStages + kTcNumABuf + i); };
-  auto acc_full = [&](int i) { return bar0 + 8u * (uint32_t)(2 * kTcNumStages + 2 * kTcNumABuf + i); };
-  auto acc_empty = [&](int i) {
-    return bar0 + 8u * (uint32_t)(2 * kTcNumStages + 2 * kTcNumABuf + 2 + i);
+  auto a_empty = [=](int i) { return bar0 + 8u * (uint32_t)i; };
+  auto acc_full = [=](int i) { return bar0 + 8u * (uint32_t)(2 + i); };
+  auto acc_empty = [=](int i) { return bar0 + 8u * (uint32_t)(4 + i); };
+  // A wait that gives up records a fault; the caller carries on (never
+  // leaving its warp's named barriers), so that the block still finishes.
+  auto wait_or_fault = [&](uint32_t bar, uint32_t parity) {
+    if (!s_fault && !mbar_wait(bar, parity)) s_fault = 1;
   };
 
   // ---- tile space: every (session, KV head) contributes its tiles --------
@@ -449,17 +508,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < kTcNumStages; ++i) {
-      mbar_init(stage_full(i), 32);             // every producer lane, after its copies
-      mbar_init(stage_empty(i), kTcBuildWarps);
-    }
-    for (int i = 0; i < kTcNumABuf; ++i) {
-      mbar_init(a_full(i), kTcBuildWarps);
-      mbar_init(a_empty(i), 1);                 // tcgen05.commit
-    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), kTcBuildWarps);
+      mbar_init(a_empty(i), kTcBuildWarps);    // every build warp commits its MMAs
+      mbar_init(acc_full(i), kTcBuildWarps);   // every build warp commits at a tile's end
+      mbar_init(acc_empty(i), kTcEpiWarps);    // every epilogue warp
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     s_fault = 0;
@@ -470,21 +522,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const uint32_t tmem = s_tmem;
   const int quarter = warp & 3;
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-  if (warp < kTcBuildWarps) {
-    // warps q and q + 4 preset one half each of the two accumulator sets
-    const int half = warp >> 2;
-    for (int i = 0; i < 4; ++i)
-      tc_st32_fill(tmem + lane_base + (uint32_t)(half * kTcAccCols + 32 * i), kTcMagicBits);
+  uint32_t mg[32];  // the accumulator preset, kept in registers by the epilogue warps
+#pragma unroll
+  for (int i = 0; i < 32; ++i) mg[i] = kTcMagicBits;
+  if (warp >= kTcEpiWarp0) {
+#pragma unroll
+    for (int i = 0; i < 2 * kTcAccCols / 32; ++i) tc_st32(tmem + lane_base + (uint32_t)(32 * i), mg);
     tc_wait_st();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
-  // pipeline counters: chunk items and tiles since the start of the kernel,
-  // and (MMA thread) the last item and tile whose completion was committed
+  // chunks and tiles since the start of the kernel
   uint32_t it = 0, tj = 0;
-  int last_item = -1, last_tile = -1;
 
   // ---- segments: runs of tiles that share one (session, KV head) ---------
   int t = t_begin;
@@ -498,269 +549,254 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     {
       const int gid = L0.s * p.h_kv + L0.g;
       const unsigned char *gplan = p.plans + (size_t)gid * PL.bytes;
-      const int P = reinterpret_cast<const TcPlanHeader *>(gplan)->P;
-      const int used = PL.off_b + ((P + 15) / 16) * kTcKStepBytes;
+      const int nk = reinterpret_cast<const TcPlanHeader *>(gplan)->nks;
+      const int used = PL.off_b + nk * kTcBChunkBytes;
       for (int i = tid; i < used / 16; i += kTcThreads)
         reinterpret_cast<uint4 *>(sPlan)[i] = reinterpret_cast<const uint4 *>(gplan)[i];
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // B is read by the MMAs
     }
     __syncthreads();
     const int P = sHdr->P;
-    const int nch = sHdr->nchunk > 0 ? sHdr->nchunk : 1;  // a plane-less group still has tiles
-    const bool big = P > kTcSmallP;                        // 0/1 cells instead of 0/2^r
+    const int nks = sHdr->nks;
+    const int nch = (nks + 1) / 2;   // chunks of 64 planes per tile
+    const bool big = P > kTcSmallP;  // 0/1 cells instead of 0/2^r
     const int64_t head0 = (int64_t)L0.s * p.h_q + L0.g * G;
+    const int nchunks = ntiles * nch;
 
-    if (warp == kTcProducerWarp) {
-      // ---------------------------------------------------------- producer --
+    if (warp < kTcBuildWarps) {
+      // --------------------------------------------- load, build and MMA --
+      const int hf = warp >> 2;  // plane groups 8 hf .. 8 hf + 7 of a chunk
+      const uint32_t sel = (uint32_t)quarter | ((uint32_t)(4 + quarter) << 4);  // byte q of a, of b
       const uint32_t *gbase = L0.planes + (int64_t)L0.g * d * 4 * L0.W;
       const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
-      uint32_t i = it;
-      for (int j = 0; j < ntiles && !s_fault; ++j) {
-        const int ti = ti0 + j;
-        for (int c = 0; c < nch; ++c, ++i) {
-          const int st = (int)(i % kTcNumStages);
-          if (i >= (uint32_t)kTcNumStages &&
-              !mbar_wait(stage_empty(st), ((i / kTcNumStages) - 1) & 1)) {
-            s_fault = 1;
-            break;
-          }
-          const int nrows = min(kTcChunkPlanes, P - c * kTcChunkPlanes);
-          const uint32_t dst0 = tc_smem_u32(sStage + st * kTcStageBytes);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int id = lane + 32 * k;  // row id / 8, 16-byte piece id % 8
-            const int row = id >> 3, piece = id & 7;
-            if (row < nrows) {
-              const uint32_t *src = gbase + (int64_t)sRows[c * kTcChunkPlanes + row] * L0.W;
-              int64_t gw;
-              bool ok;
-              if (MODE == kModeSample) {
-                const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (piece >> 1);
-                gw = sj * kSampleStride * kSectorWords + (piece & 1) * 4;
-                ok = sj < nsamp && gw < L0.W;
-              } else {
-                gw = (int64_t)ti * kTcTileWords + piece * 4;
-                ok = gw < L0.W;
-              }
-              tc_cp_async16(dst0 + (uint32_t)(row * 128 + piece * 16),
-                            ok ? (const void *)(src + gw) : (const void *)src, ok ? 16u : 0u);
-            }
-          }
-          mbar_arrive_cp_async(stage_full(st));
+      const int piece = lane & 7;
+      const int myrow = 8 * warp + (lane >> 3);  // and myrow + 4
+      // this warp's two 16-byte pieces of chunk u (segment-relative), 0 past the end
+      auto load = [&](int u, uint4 &va, uint4 &vb) {
+        va = make_uint4(0u, 0u, 0u, 0u);
+        vb = va;
+        if (u >= nchunks) return;
+        const int ti = ti0 + u / nch, c = u - (u / nch) * nch;
+        const int rbase = c * kTcChunkPlanes;
+        const int nrows = min(kTcChunkPlanes, P - rbase);
+        int64_t gw;
+        bool ok;
+        if (MODE == kModeSample) {
+          const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (piece >> 1);
+          gw = sj * kSampleStride * kSectorWords + (piece & 1) * 4;
+          ok = sj < nsamp && gw < L0.W;
+        } else {
+          gw = (int64_t)ti * kTcTileWords + piece * 4;
+          ok = gw < L0.W;
         }
-        if (s_fault) break;
-      }
-      asm volatile("cp.async.wait_all;\n" ::: "memory");
-    } else if (warp == kTcMmaWarp) {
-      // --------------------------------------------------------------- MMA --
-      if (lane == 0) {
-        const uint32_t b_addr = tc_smem_u32(sPlan + PL.off_b);
-        uint32_t i = it, tt = tj;
-        bool ok = true;
-        for (int j = 0; j < ntiles && ok; ++j, ++tt) {
+        if (ok && myrow < nrows)
+          va = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)sRows[rbase + myrow] * L0.W + gw));
+        if (ok && myrow + 4 < nrows)
+          vb = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)sRows[rbase + myrow + 4] * L0.W + gw));
+      };
+      uint4 ring[kTcLoadAhead][2];
+#pragma unroll
+      for (int j = 0; j < kTcLoadAhead; ++j) load(j, ring[j][0], ring[j][1]);
+      const uint32_t b_addr = tc_smem_u32(sPlan + PL.off_b);
+      for (int u0 = 0; u0 < nchunks; u0 += kTcLoadAhead) {
+#pragma unroll
+        for (int jj = 0; jj < kTcLoadAhead; ++jj) {
+          const int u = u0 + jj;
+          if (u >= nchunks) break;
+          const uint32_t ug = it + (uint32_t)u;  // chunk index since the kernel start
+          const int tl = u / nch, c = u - tl * nch;
+          const uint32_t tt = tj + (uint32_t)tl;
           const int ab = (int)(tt & 1);
-          if (tt >= 2 && (s_fault || !mbar_wait(acc_empty(ab), ((tt >> 1) - 1) & 1))) {
-            ok = false;
-            break;
+          const int sb = (int)(ug & 1);
+          // 1. stage this warp's rows of chunk u, and load chunk u + ahead
+          uint4 *st = reinterpret_cast<uint4 *>(sStage + sb * kTcStageBytes);
+          st[myrow * 8 + piece] = ring[jj][0];
+          st[(myrow + 4) * 8 + piece] = ring[jj][1];
+          load(u + kTcLoadAhead, ring[jj][0], ring[jj][1]);
+          // 2. the A buffer of chunk u - 2 must be consumed
+          if (warp == 0 && ug >= 2) {
+            if (lane == 0) wait_or_fault(a_empty(sb), ((ug >> 1) - 1) & 1);
+            __syncwarp();
           }
-          tc_fence_after();
-          const uint32_t dcol = tmem + (uint32_t)(ab * kTcAccCols);
-          for (int c = 0; c < nch; ++c, ++i) {
-            const int b = (int)(i % kTcNumABuf);
-            if (s_fault || !mbar_wait(a_full(b), (i / kTcNumABuf) & 1)) {
-              ok = false;
-              break;
+          named_sync(1, kTcBuildWarps * 32);
+          // 3. gather byte q of four plane words per plane group
+          const uint32_t *srow = reinterpret_cast<const uint32_t *>(sStage + sb * kTcStageBytes) + lane;
+          uint32_t T[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r0 = 4 * (8 * hf + i);
+            const uint32_t x0 = srow[(r0 + 0) * kTcTileWords];
+            const uint32_t x1 = srow[(r0 + 1) * kTcTileWords];
+            const uint32_t x2 = srow[(r0 + 2) * kTcTileWords];
+            const uint32_t x3 = srow[(r0 + 3) * kTcTileWords];
+            T[i] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
+          }
+          // 4. cells of M-blocks r = 0..7: columns 64 hf + 8 r .. + 7 of the A buffer
+          //    (this warp's K-step), written 32 columns at a time
+          const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + sb * kTcABufCols + 64 * hf);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t cell[32];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              const int r = 4 * h2 + rr;
+              if (!big) {
+                const uint32_t m = 0x01010101u << r;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cell[8 * rr + i] = T[i] & m;
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cell[8 * rr + i] = (T[i] >> r) & 0x01010101u;
+              }
             }
-            tc_fence_after();
-            const uint32_t acol = tmem + (uint32_t)(kTcAColBase + b * kTcABufCols);
+            tc_st32(acol + (uint32_t)(32 * h2), cell);
+          }
+          tc_wait_st();
+          tc_fence_before();
+          // 5. a tile's first MMAs need its accumulators free
+          if (warp == 0 && c == 0 && tt >= 2) {
+            if (lane == 0) wait_or_fault(acc_empty(ab), ((tt >> 1) - 1) & 1);
+            __syncwarp();
+          }
+          named_sync(2, kTcBuildWarps * 32);
+          tc_fence_after();
+          // 6. the MMAs of M-block `warp`
+          if (lane == 0) {
+            const uint32_t dcol = tmem + (uint32_t)(ab * kTcAccCols + kTcN * warp);
+            const uint32_t acl = tmem + (uint32_t)(kTcAColBase + sb * kTcABufCols + 8 * warp);
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
-              if (c * kTcChunkPlanes + 16 * ks < P) {
-                const uint64_t bdesc = tc_smem_desc(
-                    b_addr + (uint32_t)((2 * c + ks) * kTcKStepBytes), kTcLBO, kTcSBO);
-#pragma unroll
-                for (int mb = 0; mb < 4; ++mb)
-                  tc_mma(dcol + (uint32_t)(32 * mb), acol + (uint32_t)(16 * mb + 8 * ks), bdesc);
-              }
+              const int kidx = 2 * c + ks;
+              if (kidx < nks)
+                tc_mma(dcol, acl + (uint32_t)(64 * ks),
+                       tc_smem_desc(b_addr + (uint32_t)(kidx * kTcBChunkBytes), kTcLBO, kTcSBO));
             }
-            tc_commit(a_empty(b));
-            last_item = (int)i;
-            if (c == nch - 1) {
-              tc_commit(acc_full(ab));
-              last_tile = (int)tt;
-            }
+            tc_commit(a_empty(sb));
+            if (c == nch - 1) tc_commit(acc_full(ab));
           }
+          __syncwarp();
         }
-        if (!ok) s_fault = 1;
       }
     } else {
-      // ----------------------------------------------- build and epilogue --
-      const int half = warp >> 2;  // which K-step of a chunk; which kk pair in the epilogue
-      const uint32_t m0 = 0x01010101u << quarter;        // r = q
-      const uint32_t m1 = 0x01010101u << (quarter + 4);  // r = q + 4
-      float Kh[G], Dh[G][2], tau[G];
+      // ---------------------------------------------------------- epilogue --
+      // s = K + Delta 2^-r sum_m 256^m (f_m - M), f_m the accumulator of digit
+      // m read as a float (the two low digits combined before M is removed)
+      const int ew = warp - kTcEpiWarp0;
+      unsigned long long *cbuf = sCand + (size_t)ew * 4 * kTcCandBuf;
+      unsigned *fill = s_fill[ew];
+      if (lane < 4) fill[lane] = 0u;
+      __syncwarp();
+      float Kh[G], Dh[G], tau[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         Kh[h] = sHdr->K[h];
-        Dh[h][0] = big ? sHdr->D[h] : ldexpf(sHdr->D[h], -quarter);
-        Dh[h][1] = big ? sHdr->D[h] : ldexpf(sHdr->D[h], -(quarter + 4));
+        Dh[h] = sHdr->D[h];
         tau[h] = -INFINITY;
         if (MODE == kModeFilter) {
           const uint32_t key = p.tau[head0 + h];
           tau[h] = key == 0u ? -INFINITY : key_float(key);
         }
       }
-      const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
-
-      auto epilogue = [&](int ti, uint32_t tt) -> bool {
+      const int nsamp = MODE == kModeSample ? (int)sampled_sectors(L0.n) : 0;
+      const int nkeys = (int)L0.n;
+      for (int tl = 0; tl < ntiles; ++tl) {
+        const uint32_t tt = tj + (uint32_t)tl;
+        const int ti = ti0 + tl;
         const int ab = (int)(tt & 1);
-        if (s_fault || !mbar_wait(acc_full(ab), (tt >> 1) & 1)) return false;
+        if (lane == 0) wait_or_fault(acc_full(ab), (tt >> 1) & 1);
+        __syncwarp();
         tc_fence_after();
+        // key of (lane, quarter, r): 32 lane + 8 quarter + r of the tile
+        int tok0, slot0 = 0;
+        bool live = true;
+        if (MODE == kModeSample) {
+          const int sj = ti * kTcSampleSectorsPerTile + (lane >> 3);
+          live = sj < nsamp;
+          tok0 = (sj * kSampleStride * kSectorWords + (lane & 7)) * 32 + 8 * quarter;
+          slot0 = sj * 256 + (lane & 7) * 32 + 8 * quarter;
+        } else {
+          tok0 = (ti * kTcTileWords + lane) * 32 + 8 * quarter;
+        }
+        const uint32_t abase = tmem + lane_base + (uint32_t)(ab * kTcAccCols);
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const uint32_t taddr = tmem + lane_base + (uint32_t)(ab * kTcAccCols + 32 * (2 * hr + half));
+        for (int rp = 0; rp < kTcMBlocks / 2; ++rp) {
+          // M-blocks r = 2 rp, 2 rp + 1: keys tok0 + r
           uint32_t v[32];
-          tc_ld32(taddr, v);
-          tc_st32_fill(taddr, kTcMagicBits);
-          const int r = quarter + 4 * hr;
+          tc_ld32(abase + (uint32_t)(32 * rp), v);
+          tc_st32(abase + (uint32_t)(32 * rp), mg);
+          float sc[2][4];
 #pragma unroll
-          for (int kq = 0; kq < 2; ++kq) {
-            const int bit = 8 * (2 * half + kq) + r;  // key bit within the word
-            float sc[G];
+          for (int hr = 0; hr < 2; ++hr) {
+            const float scale = big ? 1.0f : 1.0f / (float)(1 << (2 * rp + hr));
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const uint32_t *a = v + 16 * kq + 4 * h;
-              float x = __uint_as_float(a[3]) - kTcMagic;
-              x = fmaf(x, 256.0f, __uint_as_float(a[2]) - kTcMagic);
-              x = fmaf(x, 256.0f, __uint_as_float(a[1]) - kTcMagic);
-              x = fmaf(x, 256.0f, __uint_as_float(a[0]) - kTcMagic);
-              sc[h] = fmaf(x, Dh[h][hr], Kh[h]);
+            for (int h = 0; h < 4; ++h) {
+              if (h < G) {
+                const uint32_t *a = v + 16 * hr + 4 * h;
+                const float hi = fmaf(__uint_as_float(a[3]) - kTcMagic, 256.0f,
+                                      __uint_as_float(a[2]) - kTcMagic);
+                const float lo = fmaf(__uint_as_float(a[1]), 256.0f,
+                                      __uint_as_float(a[0]) - 257.0f * kTcMagic);
+                sc[hr][h] = fmaf(fmaf(hi, 65536.0f, lo), Dh[h] * scale, Kh[h]);
+              } else {
+                sc[hr][h] = 0.0f;
+              }
             }
-            if (MODE == kModeSample) {
-              const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (lane >> 3);
-              if (sj < nsamp) {
-                const int64_t tok = (sj * kSampleStride * kSectorWords + (lane & 7)) * 32 + bit;
-                const int64_t sl = sj * 256 + (lane & 7) * 32 + bit;
-#pragma unroll
-                for (int h = 0; h < G; ++h)
-                  p.sample[(head0 + h) * p.m_max + sl] = tok < L0.n ? float_key(sc[h]) : 0u;
-              }
-            } else {
-              const int64_t tok = ((int64_t)ti * kTcTileWords + lane) * 32 + bit;
-              const bool valid = tok < L0.n;
-              if (p.debug_scores && valid) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) p.debug_scores[(head0 + h) * L0.n + tok] = sc[h];
-              }
-              bool take[G], any = false;
+          }
+          const int tk = tok0 + 2 * rp;
+          if (MODE == kModeSample) {
+            if (live) {
 #pragma unroll
               for (int h = 0; h < G; ++h) {
-                take[h] = valid && sc[h] >= tau[h];
-                any |= take[h];
-              }
-              if (__any_sync(0xffffffffu, any)) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                  const unsigned ballot = __ballot_sync(0xffffffffu, take[h]);
-                  if (ballot) {
-                    unsigned base = 0;
-                    if (lane == 0) base = atomicAdd(&p.counts[head0 + h], (unsigned)__popc(ballot));
-                    base = __shfl_sync(0xffffffffu, base, 0);
-                    if (take[h]) {
-                      const unsigned pos = base + __popc(ballot & ((1u << lane) - 1u));
-                      if ((int64_t)pos < p.cap)
-                        p.cand[(head0 + h) * p.cap + pos] = composite(sc[h], (uint32_t)tok);
-                    }
-                  }
-                }
+                uint32_t *dst = p.sample + (head0 + h) * p.m_max + slot0 + 2 * rp;
+                dst[0] = tk < nkeys ? float_key(sc[0][h]) : 0u;
+                dst[1] = tk + 1 < nkeys ? float_key(sc[1][h]) : 0u;
               }
             }
+          } else {
+            if (p.debug_scores) {
+#pragma unroll
+              for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr)
+                  if (tk + hr < nkeys)
+                    p.debug_scores[(head0 + h) * (int64_t)nkeys + tk + hr] = sc[hr][h];
+            }
+            uint32_t cm = 0u;  // bit 2 h + k: key tk + k clears head h's threshold
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              cm |= (tk < nkeys && sc[0][h] >= tau[h] ? 1u : 0u) << (2 * h);
+              cm |= (tk + 1 < nkeys && sc[1][h] >= tau[h] ? 1u : 0u) << (2 * h + 1);
+            }
+            if (__any_sync(0xffffffffu, cm != 0u))
+              tc_append(p, head0, G, cbuf, fill, cm, tk, sc[0][0], sc[1][0], sc[0][1], sc[1][1],
+                        sc[0][2], sc[1][2], sc[0][3], sc[1][3]);
           }
         }
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty(ab));
-        return true;
-      };
-
-      uint32_t i = it, tt = tj;
-      bool ok = true;
-      for (int j = 0; j < ntiles && ok; ++j, ++tt) {
-        const int ti = ti0 + j;
-        for (int c = 0; c < nch; ++c, ++i) {
-          const int st = (int)(i % kTcNumStages);
-          const int b = (int)(i % kTcNumABuf);
-          if (s_fault || !mbar_wait(stage_full(st), (i / kTcNumStages) & 1)) {
-            ok = false;
-            break;
-          }
-          if (i >= (uint32_t)kTcNumABuf &&
-              (s_fault || !mbar_wait(a_empty(b), ((i / kTcNumABuf) - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int p0 = c * kTcChunkPlanes + 16 * half;  // first plane of this warp's K-step
-          if (p0 < P) {
-            const uint32_t *srow =
-                reinterpret_cast<const uint32_t *>(sStage + st * kTcStageBytes) + 16 * half * 32 + lane;
-            uint32_t cell[4][8];
-            if (!big) {
-#pragma unroll
-              for (int pr = 0; pr < 8; ++pr) {
-                const uint32_t x0 = srow[(2 * pr) * 32];
-                const uint32_t x1 = srow[(2 * pr + 1) * 32];
-                const uint32_t c0 = __byte_perm(x0, x1, 0x5410);  // keys kk = 0, 1
-                const uint32_t c1 = __byte_perm(x0, x1, 0x7632);  // keys kk = 2, 3
-                cell[0][pr] = c0 & m0;
-                cell[1][pr] = c1 & m0;
-                cell[2][pr] = c0 & m1;
-                cell[3][pr] = c1 & m1;
-              }
-            } else {
-#pragma unroll
-              for (int pr = 0; pr < 8; ++pr) {
-                const uint32_t x0 = srow[(2 * pr) * 32];
-                const uint32_t x1 = srow[(2 * pr + 1) * 32];
-                const uint32_t c0 = __byte_perm(x0, x1, 0x5410);
-                const uint32_t c1 = __byte_perm(x0, x1, 0x7632);
-                cell[0][pr] = (c0 >> quarter) & 0x01010101u;
-                cell[1][pr] = (c1 >> quarter) & 0x01010101u;
-                cell[2][pr] = (c0 >> (quarter + 4)) & 0x01010101u;
-                cell[3][pr] = (c1 >> (quarter + 4)) & 0x01010101u;
-              }
-            }
-            const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + b * kTcABufCols + 8 * half);
-#pragma unroll
-            for (int mb = 0; mb < 4; ++mb) tc_st8(acol + (uint32_t)(16 * mb), cell[mb]);
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(stage_empty(st));
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(a_full(b));
-        }
-        if (!ok) break;
-        // the previous tile's MMAs ran while this tile was being built
-        if (j > 0 && !epilogue(ti - 1, tt - 1)) ok = false;
       }
-      if (ok && !epilogue(ti0 + ntiles - 1, tj + ntiles - 1)) ok = false;
-      if (!ok) s_fault = 1;
+      if (MODE == kModeFilter) {
+        for (int h = 0; h < G; ++h) {
+          const unsigned f = fill[h];
+          if (f) tc_flush(p, head0 + h, cbuf + h * kTcCandBuf, f);
+        }
+      }
     }
-    it += (uint32_t)(ntiles * nch);
+    it += (uint32_t)nchunks;
     tj += (uint32_t)ntiles;
     t = seg_end;
   }
 
   // ---- teardown ------------------------------------------------------------
-  // every commit must have landed before the block's barriers and tensor
-  // memory go away (on the normal path they have; after a fault, wait)
-  if (warp == kTcMmaWarp && lane == 0) {
-    if (last_item >= 0)
-      mbar_wait(a_empty(last_item % kTcNumABuf), ((uint32_t)last_item / kTcNumABuf) & 1);
-    if (last_tile >= 0) mbar_wait(acc_full(last_tile & 1), ((uint32_t)last_tile >> 1) & 1);
+  // The epilogue has seen every tile's accumulators, so every MMA is done;
+  // wait for the arrivals of the last two chunks' commits before the
+  // barriers and tensor memory go away.
+  __syncthreads();
+  if (tid == 0) {
+    if (it >= 1) mbar_wait(a_empty((it - 1) & 1), ((it - 1) >> 1) & 1);
+    if (it >= 2) mbar_wait(a_empty((it - 2) & 1), ((it - 2) >> 1) & 1);
   }
   __syncthreads();
   if (s_fault && tid == 0) atomicAdd(&p.status->device_faults, 1u);
