@@ -54,8 +54,8 @@ def parse(argv=None):
     ap.add_argument("--config", default="decode_1m")
     ap.add_argument("--budget", type=int, default=92)
     ap.add_argument("--k", type=int, default=None)
-    ap.add_argument("--tensor-cores", action="store_true",
-                    help="run the scan on the tcgen05 kernel instead of the CUDA-core kernel")
+    ap.add_argument("--cuda-cores", action="store_true",
+                    help="run the scan on the CUDA-core kernel instead of the tcgen05 kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -342,7 +342,7 @@ def run_native(args):
     k = args.k or cfg["k"]
     B = args.budget
     h_kv, h_q, d = cfg["h_kv"], cfg["h_q"], cfg["d"]
-    flags = F.FLAG_TENSOR_CORES if args.tensor_cores else 0
+    flags = F.FLAG_CUDA_CORES if args.cuda_cores else 0
     ragged = cfg["name"] == "ragged_32_sessions"
     host = cfg["name"] == "host_resident_1m"
     ws = F.Workspace(device)
@@ -499,7 +499,7 @@ def run_native(args):
                     "channels, 4-bit min-max codes)",
             "config": {"workload": workload_desc(cfg, B, k), "sessions_per_rank": S,
                        "keys_per_rank": n_total, "h_kv": h_kv, "h_q": h_q, "d": d,
-                       "budget_bits": B, "k": k, "scan_kernel": "tcgen05" if flags else "cuda-core",
+                       "budget_bits": B, "k": k, "scan_kernel": "cuda-core" if flags else "tcgen05",
                        "l2": "flushed between steps (256 MiB write, outside the events)"},
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": None,

@@ -1232,7 +1232,7 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
   int sms = 0;
   cudaError_t e = num_sms(&sms);
   if (e != cudaSuccess) return e;
-  const bool tc = (p.flags & FATHOM_FLAG_TENSOR_CORES) != 0;
+  const bool tc = (p.flags & FATHOM_FLAG_CUDA_CORES) == 0;
   if (tc) {
     e = launch_tc_plan(p, stream);
   } else {

@@ -31,7 +31,7 @@ PLANES_DEVICE = 0
 PLANES_HOST_MAPPED = 1
 FLAG_NO_SAMPLING = 1
 FLAG_FORCE_FALLBACK = 2
-FLAG_TENSOR_CORES = 4
+FLAG_CUDA_CORES = 4
 
 EXPORTED = [
     "fathom_last_error", "fathom_plane_words", "fathom_planes_bytes", "fathom_pack_planes",

@@ -75,9 +75,10 @@ typedef enum fathom_planes_location {
 /* Test knobs for fathom_scan_args.flags (0 in normal use). */
 #define FATHOM_FLAG_NO_SAMPLING 1u     /* skip the threshold sample: every key is a candidate */
 #define FATHOM_FLAG_FORCE_FALLBACK 2u  /* take the exact single-block fallback for every head */
-/* Run the scan on the tcgen05 tensor-core kernel (int8 MMA into tensor memory)
- * instead of the CUDA-core kernel.  Same results; slower at the measured sizes. */
-#define FATHOM_FLAG_TENSOR_CORES 4u
+/* Run the scan on the CUDA-core kernel (fp32 FMAs on per-channel prefix codes)
+ * instead of the default tcgen05 tensor-core kernel (int8 MMAs into tensor
+ * memory).  Same results; kept as a second, independent implementation. */
+#define FATHOM_FLAG_CUDA_CORES 4u
 
 /* Last error message of the calling thread ("" if none). */
 FATHOM_API const char *fathom_last_error(void);
@@ -136,7 +137,10 @@ FATHOM_API fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, co
  *   s_h(i) = sum_c q_c * deq_{t_c}(v_{t_c}(i, c)),
  * v_t the value of the first t planes of channel c and
  * deq_t(v) = m_c + s_c (2^(4-t) v + (2^(4-t) - 1) / 2), the centre of the
- * t-bit cell (t = 0: the constant m_c + 7.5 s_c).  Scores accumulate in fp32.
+ * t-bit cell (t = 0: the constant m_c + 7.5 s_c).  Scores are formed in
+ * fp32: the tensor-core kernel sums the plane bits against 30-bit fixed-point
+ * weights exactly in int32 and converts once, the CUDA-core kernel
+ * accumulates fp32 FMAs.
  * Output per head: the k keys with the largest s_h, ordered by score
  * descending then index ascending; if k > n the tail is index -1, score -inf.
  * Per KV head the scan reads, for each channel, the longest prefix any of its

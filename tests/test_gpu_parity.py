@@ -227,19 +227,27 @@ def test_fallback_with_compaction():
                    "fallback head %d" % h)
 
 
-# ------------------------------------------------ tensor-core scan kernel --
+# --------------------------------------------------- CUDA-core scan kernel --
+# (the default scan is the tcgen05 kernel; the CUDA-core kernel is the
+# second implementation behind FLAG_CUDA_CORES)
 
 @pytest.mark.parametrize("n,G,B,k", [(4096, 1, 92, 64), (4097, 4, 92, 7), (12345, 2, 17, 100),
                                      (40000, 4, 136, 64), (3000, 4, 0, 50), (3000, 4, 512, 50)])
-def test_tensor_core_scan(n, G, B, k):
-    """The tcgen05 (int8 MMA) form of the scan gives the oracle's answer."""
+def test_cuda_core_scan(n, G, B, k):
+    """The CUDA-core (fp32 FMA) form of the scan gives the oracle's answer."""
     case = synthkv.make_case(seed=300 + n + G, n=n, h_kv=2, h_q=2 * G, d=128, q_dtype="bf16")
-    _full_check(case, B, k, flags=F.FLAG_TENSOR_CORES, what="tc n=%d G=%d B=%d" % (n, G, B))
+    _full_check(case, B, k, flags=F.FLAG_CUDA_CORES, what="cc n=%d G=%d B=%d" % (n, G, B))
 
 
-def test_tensor_core_scan_layer_131k(layer_131k):
-    _check_config(layer_131k, 92, 2048, heads_full={0, 13, 26, 31}, what="tc 131k",
-                  flags=F.FLAG_TENSOR_CORES)
+@pytest.mark.parametrize("d", [32, 256])
+def test_cuda_core_scan_widths(d):
+    case = synthkv.make_case(seed=d + 1, n=5000, h_kv=1, h_q=4, d=d, q_dtype="bf16")
+    _full_check(case, d // 2, 33, flags=F.FLAG_CUDA_CORES, what="cc d=%d" % d)
+
+
+def test_cuda_core_scan_layer_131k(layer_131k):
+    _check_config(layer_131k, 92, 2048, heads_full={0, 13, 26, 31}, what="cc 131k",
+                  flags=F.FLAG_CUDA_CORES)
 
 
 # ------------------------------------------------------ full-size configs --
@@ -293,10 +301,10 @@ def test_decode_1m(decode_1m, B):
     assert rep.fallback_heads == 0
 
 
-def test_decode_1m_tensor_cores(decode_1m):
-    """The tcgen05 scan on the 1M-token step (the benchmarked launch set)."""
-    _check_config(decode_1m, 92, 2048, heads_full={0, 21}, what="tc 1M",
-                  flags=F.FLAG_TENSOR_CORES)
+def test_decode_1m_cuda_cores(decode_1m):
+    """The CUDA-core scan on the 1M-token step."""
+    _check_config(decode_1m, 92, 2048, heads_full={0, 21}, what="cc 1M",
+                  flags=F.FLAG_CUDA_CORES)
     rep = F.read_report()
     assert rep.fallback_heads == 0
     assert rep.device_faults == 0
@@ -314,17 +322,17 @@ def test_host_resident_1m_budget_sweep():
         _, _, (idx_d, sc_d) = run_gpu(case, B, 2048)
         np.testing.assert_array_equal(idx_h, _np(idx_d))
         np.testing.assert_array_equal(sc_h, _np(sc_d))
-    # the tcgen05 scan reads host-resident planes too
-    idx_h, sc_h = _check_config(case, 92, 2048, heads_full={3}, what="tc host B=92",
-                                host_mapped=True, flags=F.FLAG_TENSOR_CORES)
-    _, _, (idx_d, sc_d) = run_gpu(case, 92, 2048, flags=F.FLAG_TENSOR_CORES)
+    # the CUDA-core scan reads host-resident planes too
+    idx_h, sc_h = _check_config(case, 92, 2048, heads_full={3}, what="cc host B=92",
+                                host_mapped=True, flags=F.FLAG_CUDA_CORES)
+    _, _, (idx_d, sc_d) = run_gpu(case, 92, 2048, flags=F.FLAG_CUDA_CORES)
     np.testing.assert_array_equal(idx_h, _np(idx_d))
     np.testing.assert_array_equal(sc_h, _np(sc_d))
 
 
-@pytest.mark.parametrize("tc", [False, True])
-def test_ragged_32_sessions_batched(tc):
-    flags = F.FLAG_TENSOR_CORES if tc else 0
+@pytest.mark.parametrize("cuda_cores", [False, True])
+def test_ragged_32_sessions_batched(cuda_cores):
+    flags = F.FLAG_CUDA_CORES if cuda_cores else 0
     c = synthkv.CONFIGS["ragged_32_sessions"]
     sessions = synthkv.make_ragged(c["seed"], c["sessions"], c["n_lo"], c["n_hi"], c["h_kv"],
                                    c["h_q"], c["d"], c["q_dtype"], device="cuda")
