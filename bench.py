@@ -29,6 +29,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -212,6 +213,32 @@ def get_cfg(name):
     cfg["name"] = name
     return cfg
 
+
+
+def profiled_traffic(workload, kernel_source):
+    """DRAM bytes (read + write) per launch of the filtering scan, from the ncu
+    summaries under profiles/ -- only while the kernel source hashes to the one
+    the counters were taken on and the workload matches; else None."""
+    import glob
+    import hashlib
+    src = os.path.join(ROOT, kernel_source)
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                m = re.match(r"^(traffic_bytes_per_launch|kernel_source|kernel_source_sha256|workload): (\S+)$",
+                             line.strip())
+                if m:
+                    fields[m.group(1)] = m.group(2)
+        if (fields.get("kernel_source") == kernel_source and fields.get("workload") == workload
+                and fields.get("kernel_source_sha256") == digest
+                and "traffic_bytes_per_launch" in fields):
+            return int(fields["traffic_bytes_per_launch"])
+    return None
 
 def workload_desc(cfg, budget, k):
     if cfg["name"] == "ragged_32_sessions":
@@ -491,6 +518,10 @@ def run_native(args):
                          "of all %d keys, brute-force top-%d; single thread, %.1f s" % (c.n, k, secs)}
 
     if rank == 0:
+        traffic = None
+        if not ragged and not host:
+            traffic = profiled_traffic(cfg["name"], "bit_plane_kv_scan_b200/csrc/scan.cu"
+                                       if flags else "bit_plane_kv_scan_b200/csrc/scan_tc.cu")
         res = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": True,
@@ -502,7 +533,7 @@ def run_native(args):
                        "budget_bits": B, "k": k, "scan_kernel": "cuda-core" if flags else "tcgen05",
                        "l2": "flushed between steps (256 MiB write, outside the events)"},
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
-                         "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_kind": peak_kind, "kernel": "filtering scan",
                          "kernel_ms": t_kern, "algorithmic_bytes": alg_bytes,
                          "union_planes": int(rep.union_planes)},
