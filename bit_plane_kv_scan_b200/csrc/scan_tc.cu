@@ -26,21 +26,28 @@
 // Every key has its own row and B has N = 16 columns (head, digit).
 //
 // Work split (measured on B200: one thread issues a tcgen05.mma only every
-// ~46 cycles, an mbarrier round trip costs 100-200 cycles, and bulk copies of
-// 128-byte row pieces are limited by their per-copy cost):
-//  * A chunk is 64 plane rows of a tile.  The eight build warps load it
-//    themselves with 16-byte global loads (warp w: rows 8 w .. 8 w + 7),
-//    eight chunks ahead in registers, stage it in shared memory, and
-//    synchronise with named barriers only.
-//  * Warp w (lane quarter w % 4, plane groups 8 (w / 4) .. + 7, i.e. K-step
-//    w / 4 of the chunk) writes its 64 cells per lane to tensor memory in two
-//    32-column stores (A buffer columns: K-step, then M-block, then group);
-//    after a barrier, warp w issues the two MMAs of
-//    M-block w (two K-steps of 32 planes) and commits them: eight issuers,
-//    and every accumulator region always fed by the same thread.
-//  * Warps 8-11 read a finished tile's accumulators back, score, and collect
-//    the keys above the head's threshold in shared memory, flushing them to
-//    the candidate buffer with one global atomic per flush.
+// ~46 cycles, a tcgen05.commit reaches its mbarrier ~800 cycles after issue,
+// and bulk copies of 128-byte row pieces are limited by their per-copy cost).
+// The K-steps (32 union planes of one tile) of a run of tiles are taken two at
+// a time as a chunk, so only a tile's last K-step can be part padding.
+//  * Load warps 0-3: thread (plane group i, word quad m) loads four plane rows
+//    of the chunk with 16-byte global loads (three chunks ahead in
+//    registers, more prefetched into L2), transposes the bytes so that
+//    T = [x0.q, x1.q, x2.q, x3.q] for each lane quarter q, and stores them in
+//    a four-stage shared-memory ring, where a build warp reads its T values
+//    conflict-free.
+//  * Build warps 4-11 (lane quarter w % 4, group g = M-blocks 4 g .. 4 g + 3)
+//    write the cells of their M-blocks for both K-steps to tensor memory (two
+//    32-column stores).  The four warps of a group meet at a named barrier
+//    one chunk later, after reading the next stage, and each then issues
+//    the two MMAs of its own M-block: eight issuers, every accumulator
+//    region always fed by the same thread.
+//  * Epilogue warps 12-19 (lane quarter, half: four M-blocks each) read a
+//    finished tile's accumulators back, score, and collect the keys above
+//    the head's threshold in shared memory, flushing them to the candidate
+//    buffer with one global atomic per flush.
+// Stages, A buffers (two) and accumulators (two) are handed over with
+// mbarriers.
 // Accumulators are preset to the bits of 1.5 * 2^23, so that an accumulator
 // read back as a float is 1.5 * 2^23 + acc exactly (|acc| <= 2^22).  When
 // P > 256 the cells hold 0/1 instead of 0/2^r so that acc stays within 2^22.
@@ -55,11 +62,15 @@ constexpr int kTcTileWords = 32;                        // 1024 keys per tile
 constexpr int kTcChunkPlanes = 64;                      // plane rows per chunk
 constexpr int kTcKStep = 32;                            // planes per MMA (K = 32 int8)
 constexpr int kTcStageBytes = kTcChunkPlanes * kTcTileWords * 4;  // 8 KiB
+constexpr int kTcLoadWarps = 4;                         // warps 0-3
+constexpr int kTcBuildWarp0 = 4;                        // warps 4-11
 constexpr int kTcBuildWarps = 8;
-constexpr int kTcEpiWarp0 = 8;                          // warps 8-11
-constexpr int kTcEpiWarps = 4;
-constexpr int kTcThreads = (kTcBuildWarps + kTcEpiWarps) * 32;
-constexpr int kTcLoadAhead = 8;                         // chunks in flight per build warp
+constexpr int kTcEpiWarp0 = 12;                         // warps 12-19
+constexpr int kTcEpiWarps = 8;                          // two per lane quarter
+constexpr int kTcThreads = (kTcLoadWarps + kTcBuildWarps + kTcEpiWarps) * 32;
+constexpr int kTcStages = 4;                            // staged chunks in shared memory
+constexpr int kTcRing = 3;                              // chunks a load thread holds in registers
+constexpr int kTcPrefetch = 8;                          // chunks beyond those prefetched into L2
 constexpr int kTcMBlocks = 8;                           // one per bit position r
 constexpr int kTcN = 16;                                // (head, digit) columns
 constexpr int kTcAccCols = kTcMBlocks * kTcN;           // 128: one tile's accumulators
@@ -116,7 +127,7 @@ __host__ __device__ inline TcPlanLayout tc_plan_layout(int d) {
 int tc_plan_bytes(int d) { return tc_plan_layout(d).bytes; }
 
 static int tc_smem_bytes(int d, int S) {
-  int b = 128 + 2 * kTcStageBytes + tc_plan_layout(d).bytes + 4 * (S + 1) +
+  int b = 128 + kTcStages * kTcStageBytes + tc_plan_layout(d).bytes + 4 * (S + 1) +
           kTcEpiWarps * 4 * kTcCandBuf * 8;
   // more than half an SM's shared memory: one block per SM, so that the
   // block's 512 tensor-memory columns never wait for another block
@@ -153,16 +164,16 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 
 // Waits for the completion of the phase of bar with the given parity, giving
 // up after about a second (2^31 cycles).  Returns false on timeout.  Each
-// try_wait may suspend the thread for up to 0.1 ms until the phase completes,
-// so a waiting warp takes no issue slots from the working ones.
+// try_wait may suspend the thread for a system-dependent time until the phase
+// completes (an explicit suspend-time hint measured slower on B200).
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
       "selp.b32 %0, 1, 0, P;\n\t}\n"
       : "=r"(done)
-      : "r"(bar), "r"(parity), "r"(100000u)
+      : "r"(bar), "r"(parity)
       : "memory");
   return done != 0;
 }
@@ -461,25 +472,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const int d = p.d;
   const TcPlanLayout PL = tc_plan_layout(d);
   unsigned char *sStage = smem;
-  unsigned char *sPlan = smem + 2 * kTcStageBytes;
+  unsigned char *sPlan = smem + kTcStages * kTcStageBytes;
   unsigned long long *sCand = reinterpret_cast<unsigned long long *>(sPlan + PL.bytes);
   int *s_tprefix = reinterpret_cast<int *>(sCand + kTcEpiWarps * 4 * kTcCandBuf);
   const TcPlanHeader *sHdr = reinterpret_cast<const TcPlanHeader *>(sPlan);
   const uint16_t *sRows = reinterpret_cast<const uint16_t *>(sPlan + PL.off_rows);
-  __shared__ __align__(8) unsigned long long s_bar[6];
+  __shared__ __align__(8) unsigned long long s_bar[16];
   __shared__ uint32_t s_tmem;
   __shared__ int s_tmp[32];
   __shared__ volatile int s_fault;
   __shared__ unsigned s_fill[kTcEpiWarps][4];  // candidates buffered per epilogue warp and head
 
   const uint32_t bar0 = tc_smem_u32(&s_bar[0]);
-  auto a_empty = [=](int i) { return bar0 + 8u * (uint32_t)i; };
-  auto acc_full = [=](int i) { return bar0 + 8u * (uint32_t)(2 + i); };
-  auto acc_empty = [=](int i) { return bar0 + 8u * (uint32_t)(4 + i); };
+  auto stage_full = [=](int s) { return bar0 + 8u * (uint32_t)s; };
+  auto stage_empty = [=](int s) { return bar0 + 8u * (uint32_t)(kTcStages + s); };
+  auto a_empty = [=](int g, int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 2 * g + b); };
+  auto acc_full = [=](int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 4 + b); };
+  auto acc_empty = [=](int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 6 + b); };
   // A wait that gives up records a fault; the caller carries on (never
   // leaving its warp's named barriers), so that the block still finishes.
   auto wait_or_fault = [&](uint32_t bar, uint32_t parity) {
     if (!s_fault && !mbar_wait(bar, parity)) s_fault = 1;
+  };
+  // one lane waits, the warp follows
+  auto warp_wait = [&](uint32_t bar, uint32_t parity) {
+    if (lane == 0) wait_or_fault(bar, parity);
+    __syncwarp();
+  };
+  auto warp_arrive = [&](uint32_t bar) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
   };
 
   // ---- tile space: every (session, KV head) contributes its tiles --------
@@ -508,10 +530,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   if (tid == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(stage_full(s), kTcLoadWarps);    // every load warp
+      mbar_init(stage_empty(s), kTcBuildWarps);  // every build warp
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(a_empty(i), kTcBuildWarps);    // every build warp commits its MMAs
-      mbar_init(acc_full(i), kTcBuildWarps);   // every build warp commits at a tile's end
-      mbar_init(acc_empty(i), kTcEpiWarps);    // every epilogue warp
+      mbar_init(a_empty(0, i), kTcBuildWarps / 2);  // the MMA commits of a build group
+      mbar_init(a_empty(1, i), kTcBuildWarps / 2);
+      mbar_init(acc_full(i), kTcBuildWarps);        // every build warp commits at a tile's end
+      mbar_init(acc_empty(i), kTcEpiWarps);         // every epilogue warp
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     s_fault = 0;
@@ -522,12 +549,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const uint32_t tmem = s_tmem;
   const int quarter = warp & 3;
   const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-  uint32_t mg[32];  // the accumulator preset, kept in registers by the epilogue warps
+  uint32_t mg[8];  // the accumulator preset, stored eight columns at a time
 #pragma unroll
-  for (int i = 0; i < 32; ++i) mg[i] = kTcMagicBits;
+  for (int i = 0; i < 8; ++i) mg[i] = kTcMagicBits;
   if (warp >= kTcEpiWarp0) {
+    // epilogue warp (quarter, half eh) owns M-blocks 4 eh .. 4 eh + 3: columns 64 eh .. + 63
+    const int eh = (warp - kTcEpiWarp0) >> 2;
 #pragma unroll
-    for (int i = 0; i < 2 * kTcAccCols / 32; ++i) tc_st32(tmem + lane_base + (uint32_t)(32 * i), mg);
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        tc_st8(tmem + lane_base + (uint32_t)(b * kTcAccCols + 64 * eh + 8 * i), mg);
     tc_wait_st();
   }
   tc_fence_before();
@@ -558,130 +590,202 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     __syncthreads();
     const int P = sHdr->P;
     const int nks = sHdr->nks;
-    const int nch = (nks + 1) / 2;   // chunks of 64 planes per tile
     const bool big = P > kTcSmallP;  // 0/1 cells instead of 0/2^r
     const int64_t head0 = (int64_t)L0.s * p.h_q + L0.g * G;
-    const int nchunks = ntiles * nch;
+    // The segment's K-steps (tile tl, plane block kidx), tile by tile, are
+    // taken two at a time: chunk u holds K-steps 2 u and 2 u + 1, which may
+    // belong to two tiles.  Only a tile's last K-step is ever partly padding.
+    const int nksteps = ntiles * nks;
+    const int nchunks = (nksteps + 1) / 2;
 
-    if (warp < kTcBuildWarps) {
-      // --------------------------------------------- load, build and MMA --
-      const int hf = warp >> 2;  // plane groups 8 hf .. 8 hf + 7 of a chunk
-      const uint32_t sel = (uint32_t)quarter | ((uint32_t)(4 + quarter) << 4);  // byte q of a, of b
+    if (warp < kTcLoadWarps) {
+      // --------------------------------------------------------------- load --
+      // Thread (group i, quad m) loads words 4 m .. 4 m + 3 of the tile from
+      // the four plane rows 4 i .. 4 i + 3 of a chunk, and stores byte q of
+      // the four rows' words as T = [x0.q, x1.q, x2.q, x3.q] at
+      // stage[i][q][word]: a build warp of quarter q reads its T of plane
+      // group i for word `lane` with one conflict-free load.
+      const int m = tid & 7;
+      const int grp = tid >> 3;  // 0 .. 15
       const uint32_t *gbase = L0.planes + (int64_t)L0.g * d * 4 * L0.W;
       const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
-      const int piece = lane & 7;
-      const int myrow = 8 * warp + (lane >> 3);  // and myrow + 4
-      // this warp's two 16-byte pieces of chunk u (segment-relative), 0 past the end
-      auto load = [&](int u, uint4 &va, uint4 &vb) {
-        va = make_uint4(0u, 0u, 0u, 0u);
-        vb = va;
-        if (u >= nchunks) return;
-        const int ti = ti0 + u / nch, c = u - (u / nch) * nch;
-        const int rbase = c * kTcChunkPlanes;
-        const int nrows = min(kTcChunkPlanes, P - rbase);
+      const bool pf = !p.planes_host;
+      // word offset of this thread's quad in tile ti, or -1 past the data
+      auto quad_word = [&](int ti) -> int64_t {
         int64_t gw;
-        bool ok;
         if (MODE == kModeSample) {
-          const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (piece >> 1);
-          gw = sj * kSampleStride * kSectorWords + (piece & 1) * 4;
-          ok = sj < nsamp && gw < L0.W;
+          const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (m >> 1);
+          gw = sj * kSampleStride * kSectorWords + (m & 1) * 4;
+          if (sj >= nsamp) return -1;
         } else {
-          gw = (int64_t)ti * kTcTileWords + piece * 4;
-          ok = gw < L0.W;
+          gw = (int64_t)ti * kTcTileWords + m * 4;
         }
-        if (ok && myrow < nrows)
-          va = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)sRows[rbase + myrow] * L0.W + gw));
-        if (ok && myrow + 4 < nrows)
-          vb = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)sRows[rbase + myrow + 4] * L0.W + gw));
+        return gw < L0.W ? gw : -1;
       };
-      uint4 ring[kTcLoadAhead][2];
+      // this thread's K-step of a chunk is its half (grp >> 3); a cursor
+      // (tile, kidx) walks the K-steps of that half, two K-steps per chunk
+      const int half = grp >> 3;
+      const int rgrp = 4 * (grp & 7);  // first of its four rows in the K-step
+      auto cursor0 = [&](int &tl, int &kx) {
+        tl = 0;
+        kx = half;
+        if (kx >= nks) { kx -= nks; ++tl; }
+      };
+      auto advance = [&](int &tl, int &kx) {
+        kx += 2;
+        while (kx >= nks) { kx -= nks; ++tl; }
+      };
+      int ltl, lk;  // next K-step to load
+      cursor0(ltl, lk);
+      auto load_next = [&](uint4 (&v)[4]) {
 #pragma unroll
-      for (int j = 0; j < kTcLoadAhead; ++j) load(j, ring[j][0], ring[j][1]);
-      const uint32_t b_addr = tc_smem_u32(sPlan + PL.off_b);
-      for (int u0 = 0; u0 < nchunks; u0 += kTcLoadAhead) {
+        for (int k = 0; k < 4; ++k) v[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (ltl < ntiles) {
+          const int64_t gw = quad_word(ti0 + ltl);
+          const int r0 = lk * kTcKStep + rgrp;
+          if (gw >= 0) {
 #pragma unroll
-        for (int jj = 0; jj < kTcLoadAhead; ++jj) {
+            for (int k = 0; k < 4; ++k)
+              if (r0 + k < P)
+                v[k] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)sRows[r0 + k] * L0.W + gw));
+          }
+        }
+        advance(ltl, lk);
+      };
+      int ftl, fk;  // next K-step to prefetch into L2
+      cursor0(ftl, fk);
+      auto prefetch_next = [&]() {
+        if (ftl < ntiles && pf && m == 0) {
+          const int64_t gw = quad_word(ti0 + ftl);
+          const int r0 = fk * kTcKStep + rgrp;
+          if (gw >= 0) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (r0 + k < P)
+                asm volatile("prefetch.global.L2 [%0];\n" ::"l"(gbase + (int64_t)sRows[r0 + k] * L0.W + gw));
+          }
+        }
+        advance(ftl, fk);
+      };
+      for (int j = 0; j < kTcRing + kTcPrefetch; ++j) prefetch_next();
+      uint4 ring[kTcRing][4];
+#pragma unroll
+      for (int j = 0; j < kTcRing; ++j) load_next(ring[j]);
+      for (int u0 = 0; u0 < nchunks; u0 += kTcRing) {
+#pragma unroll
+        for (int jj = 0; jj < kTcRing; ++jj) {
           const int u = u0 + jj;
           if (u >= nchunks) break;
-          const uint32_t ug = it + (uint32_t)u;  // chunk index since the kernel start
-          const int tl = u / nch, c = u - tl * nch;
-          const uint32_t tt = tj + (uint32_t)tl;
-          const int ab = (int)(tt & 1);
-          const int sb = (int)(ug & 1);
-          // 1. stage this warp's rows of chunk u, and load chunk u + ahead
-          uint4 *st = reinterpret_cast<uint4 *>(sStage + sb * kTcStageBytes);
-          st[myrow * 8 + piece] = ring[jj][0];
-          st[(myrow + 4) * 8 + piece] = ring[jj][1];
-          load(u + kTcLoadAhead, ring[jj][0], ring[jj][1]);
-          // 2. the A buffer of chunk u - 2 must be consumed
-          if (warp == 0 && ug >= 2) {
-            if (lane == 0) wait_or_fault(a_empty(sb), ((ug >> 1) - 1) & 1);
-            __syncwarp();
+          const uint32_t ug = it + (uint32_t)u;
+          const int s = (int)(ug % kTcStages);
+          if (ug >= (uint32_t)kTcStages) warp_wait(stage_empty(s), ((ug / kTcStages) - 1) & 1);
+          uint32_t *dst = reinterpret_cast<uint32_t *>(sStage + s * kTcStageBytes) + grp * 4 * kTcTileWords + 4 * m;
+          uint32_t Tq[4][4];  // [quarter][word]
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t x0 = (&ring[jj][0].x)[w], x1 = (&ring[jj][1].x)[w];
+            const uint32_t x2 = (&ring[jj][2].x)[w], x3 = (&ring[jj][3].x)[w];
+            const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
+            const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
+            Tq[0][w] = __byte_perm(a_lo, b_lo, 0x5410);
+            Tq[1][w] = __byte_perm(a_lo, b_lo, 0x7632);
+            Tq[2][w] = __byte_perm(a_hi, b_hi, 0x5410);
+            Tq[3][w] = __byte_perm(a_hi, b_hi, 0x7632);
           }
-          named_sync(1, kTcBuildWarps * 32);
-          // 3. gather byte q of four plane words per plane group
-          const uint32_t *srow = reinterpret_cast<const uint32_t *>(sStage + sb * kTcStageBytes) + lane;
-          uint32_t T[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r0 = 4 * (8 * hf + i);
-            const uint32_t x0 = srow[(r0 + 0) * kTcTileWords];
-            const uint32_t x1 = srow[(r0 + 1) * kTcTileWords];
-            const uint32_t x2 = srow[(r0 + 2) * kTcTileWords];
-            const uint32_t x3 = srow[(r0 + 3) * kTcTileWords];
-            T[i] = __byte_perm(__byte_perm(x0, x1, sel), __byte_perm(x2, x3, sel), 0x5410);
-          }
-          // 4. cells of M-blocks r = 0..7: columns 64 hf + 8 r .. + 7 of the A buffer
-          //    (this warp's K-step), written 32 columns at a time
-          const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + sb * kTcABufCols + 64 * hf);
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t cell[32];
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-              const int r = 4 * h2 + rr;
-              if (!big) {
-                const uint32_t m = 0x01010101u << r;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) cell[8 * rr + i] = T[i] & m;
-              } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) cell[8 * rr + i] = (T[i] >> r) & 0x01010101u;
-              }
-            }
-            tc_st32(acol + (uint32_t)(32 * h2), cell);
-          }
-          tc_wait_st();
-          tc_fence_before();
-          // 5. a tile's first MMAs need its accumulators free
-          if (warp == 0 && c == 0 && tt >= 2) {
-            if (lane == 0) wait_or_fault(acc_empty(ab), ((tt >> 1) - 1) & 1);
-            __syncwarp();
-          }
-          named_sync(2, kTcBuildWarps * 32);
-          tc_fence_after();
-          // 6. the MMAs of M-block `warp`
-          if (lane == 0) {
-            const uint32_t dcol = tmem + (uint32_t)(ab * kTcAccCols + kTcN * warp);
-            const uint32_t acl = tmem + (uint32_t)(kTcAColBase + sb * kTcABufCols + 8 * warp);
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-              const int kidx = 2 * c + ks;
-              if (kidx < nks)
-                tc_mma(dcol, acl + (uint32_t)(64 * ks),
-                       tc_smem_desc(b_addr + (uint32_t)(kidx * kTcBChunkBytes), kTcLBO, kTcSBO));
-            }
-            tc_commit(a_empty(sb));
-            if (c == nch - 1) tc_commit(acc_full(ab));
-          }
-          __syncwarp();
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(dst + q * kTcTileWords) = make_uint4(Tq[q][0], Tq[q][1], Tq[q][2], Tq[q][3]);
+          warp_arrive(stage_full(s));
+          load_next(ring[jj]);
+          prefetch_next();
         }
       }
+    } else if (warp < kTcEpiWarp0) {
+      // -------------------------------------------------------- build + MMA --
+      // Build warp (quarter q, group g) writes the cells of M-blocks
+      // 4 g .. 4 g + 3 for its lane quarter, both K-steps of a chunk; after
+      // the four warps of its group have stored, it issues the two MMAs of
+      // M-block 4 g + q.  A chunk's MMAs are issued one chunk late, after the
+      // next chunk's stage has been read, so that the tensor memory stores
+      // have that long to complete.
+      const int g = (warp - kTcBuildWarp0) >> 2;
+      const int mrow = 4 * g + quarter;  // the M-block this warp issues
+      // B of K-step kx: the descriptor's address field counts 16-byte units
+      const uint64_t b_desc0 = tc_smem_desc(tc_smem_u32(sPlan + PL.off_b), kTcLBO, kTcSBO);
+      // the MMAs of chunk up, whose first K-step is (tile tl, block kx)
+      auto complete = [&](int up, int tl, int kx) {
+        const uint32_t ug = it + (uint32_t)up;
+        const int sb = (int)(ug & 1);
+        tc_wait_st();
+        tc_fence_before();
+        named_sync(1 + g, 4 * 32);
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t acl = tmem + (uint32_t)(kTcAColBase + sb * kTcABufCols + 8 * mrow);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            if (2 * up + ks < nksteps) {
+              const uint32_t tt = tj + (uint32_t)tl;
+              const int ab = (int)(tt & 1);
+              // a tile's first MMA needs its accumulators read out
+              if (kx == 0 && tt >= 2) wait_or_fault(acc_empty(ab), ((tt >> 1) - 1) & 1);
+              tc_mma(tmem + (uint32_t)(ab * kTcAccCols + kTcN * mrow), acl + (uint32_t)(64 * ks),
+                     b_desc0 + (uint64_t)(kx * (kTcBChunkBytes >> 4)));
+              if (kx == nks - 1) tc_commit(acc_full(ab));
+            }
+            if (++kx == nks) { kx = 0; ++tl; }
+          }
+          tc_commit(a_empty(g, sb));
+        }
+        __syncwarp();
+      };
+      int btl = 0, bk = 0;  // chunk u's first K-step
+      int ptl = 0, pk = 0;  // chunk u - 1's
+      for (int u = 0; u < nchunks; ++u) {
+        const uint32_t ug = it + (uint32_t)u;
+        const int s = (int)(ug % kTcStages);
+        const int sb = (int)(ug & 1);
+        warp_wait(stage_full(s), (ug / kTcStages) & 1);
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(sStage + s * kTcStageBytes) + quarter * kTcTileWords + lane;
+        uint32_t T[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) T[i] = src[i * 4 * kTcTileWords];
+        warp_arrive(stage_empty(s));
+        if (u > 0) complete(u - 1, ptl, pk);
+        // chunk u's A buffer was last read by the MMAs of chunk u - 2
+        if (ug >= 2) warp_wait(a_empty(g, sb), ((ug >> 1) - 1) & 1);
+        const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + sb * kTcABufCols + 32 * g);
+        const int nk_here = 2 * u + 1 < nksteps ? 2 : 1;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          if (ks >= nk_here) break;
+          uint32_t cell[32];
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            const int r = 4 * g + rr;
+            if (!big) {
+              const uint32_t msk = 0x01010101u << r;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) cell[8 * rr + i] = T[8 * ks + i] & msk;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) cell[8 * rr + i] = (T[8 * ks + i] >> r) & 0x01010101u;
+            }
+          }
+          tc_st32(acol + (uint32_t)(64 * ks), cell);
+        }
+        ptl = btl;
+        pk = bk;
+        bk += 2;
+        while (bk >= nks) { bk -= nks; ++btl; }
+      }
+      complete(nchunks - 1, ptl, pk);
     } else {
       // ---------------------------------------------------------- epilogue --
       // s = K + Delta 2^-r sum_m 256^m (f_m - M), f_m the accumulator of digit
       // m read as a float (the two low digits combined before M is removed)
       const int ew = warp - kTcEpiWarp0;
+      const int eh = ew >> 2;  // M-blocks 4 eh .. 4 eh + 3
       unsigned long long *cbuf = sCand + (size_t)ew * 4 * kTcCandBuf;
       unsigned *fill = s_fill[ew];
       if (lane < 4) fill[lane] = 0u;
@@ -703,8 +807,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
         const uint32_t tt = tj + (uint32_t)tl;
         const int ti = ti0 + tl;
         const int ab = (int)(tt & 1);
-        if (lane == 0) wait_or_fault(acc_full(ab), (tt >> 1) & 1);
-        __syncwarp();
+        warp_wait(acc_full(ab), (tt >> 1) & 1);
         tc_fence_after();
         // key of (lane, quarter, r): 32 lane + 8 quarter + r of the tile
         int tok0, slot0 = 0;
@@ -719,15 +822,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
         }
         const uint32_t abase = tmem + lane_base + (uint32_t)(ab * kTcAccCols);
 #pragma unroll
-        for (int rp = 0; rp < kTcMBlocks / 2; ++rp) {
+        for (int rr = 0; rr < 2; ++rr) {
           // M-blocks r = 2 rp, 2 rp + 1: keys tok0 + r
+          const int rp = 2 * eh + rr;
           uint32_t v[32];
           tc_ld32(abase + (uint32_t)(32 * rp), v);
-          tc_st32(abase + (uint32_t)(32 * rp), mg);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tc_st8(abase + (uint32_t)(32 * rp + 8 * i), mg);
           float sc[2][4];
 #pragma unroll
           for (int hr = 0; hr < 2; ++hr) {
-            const float scale = big ? 1.0f : 1.0f / (float)(1 << (2 * rp + hr));
+            const float scale = big ? 1.0f : __int_as_float((127 - (2 * rp + hr)) << 23);  // 2^-r
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               if (h < G) {
@@ -774,8 +879,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
         }
         tc_wait_st();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty(ab));
+        warp_arrive(acc_empty(ab));
       }
       if (MODE == kModeFilter) {
         for (int h = 0; h < G; ++h) {
@@ -795,8 +899,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   // barriers and tensor memory go away.
   __syncthreads();
   if (tid == 0) {
-    if (it >= 1) mbar_wait(a_empty((it - 1) & 1), ((it - 1) >> 1) & 1);
-    if (it >= 2) mbar_wait(a_empty((it - 2) & 1), ((it - 2) >> 1) & 1);
+    for (int back = 1; back <= 2; ++back) {
+      if (it < (uint32_t)back) break;
+      const uint32_t ug = it - (uint32_t)back;
+      mbar_wait(a_empty(0, (int)(ug & 1)), (ug >> 1) & 1);
+      mbar_wait(a_empty(1, (int)(ug & 1)), (ug >> 1) & 1);
+    }
   }
   __syncthreads();
   if (s_fault && tid == 0) atomicAdd(&p.status->device_faults, 1u);
