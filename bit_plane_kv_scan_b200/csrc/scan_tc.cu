@@ -32,16 +32,16 @@
 // a time as a chunk, so only a tile's last K-step can be part padding.
 //  * Load warps 0-3: thread (plane group i, word quad m) loads four plane rows
 //    of the chunk with 16-byte global loads (three chunks ahead in
-//    registers, more prefetched into L2), transposes the bytes so that
-//    T = [x0.q, x1.q, x2.q, x3.q] for each lane quarter q, and stores them in
-//    a four-stage shared-memory ring, where a build warp reads its T values
-//    conflict-free.
+//    registers; row addresses from a per-segment offset table), transposes
+//    the bytes so that T = [x0.q, x1.q, x2.q, x3.q] for each lane quarter q,
+//    and stores them in a four-stage shared-memory ring, where a build warp
+//    reads its T values conflict-free.  Lane 0 of load warp l also issues
+//    the MMAs of M-blocks 2 l and 2 l + 1, five chunks behind its loads:
+//    four issuers, every accumulator region always fed by the same thread.
 //  * Build warps 4-11 (lane quarter w % 4, group g = M-blocks 4 g .. 4 g + 3)
 //    write the cells of their M-blocks for both K-steps to tensor memory (two
-//    32-column stores).  The four warps of a group meet at a named barrier
-//    one chunk later, after reading the next stage, and each then issues
-//    the two MMAs of its own M-block: eight issuers, every accumulator
-//    region always fed by the same thread.
+//    32-column stores) and signal them one chunk later, after reading the
+//    next stage, so that the stores have that long to land.
 //  * Epilogue warps 12-19 (lane quarter, half: four M-blocks each) read a
 //    finished tile's accumulators back, score, and collect the keys above
 //    the head's threshold in shared memory, flushing them to the candidate
@@ -70,7 +70,6 @@ constexpr int kTcEpiWarps = 8;                          // two per lane quarter
 constexpr int kTcThreads = (kTcLoadWarps + kTcBuildWarps + kTcEpiWarps) * 32;
 constexpr int kTcStages = 4;                            // staged chunks in shared memory
 constexpr int kTcRing = 3;                              // chunks a load thread holds in registers
-constexpr int kTcPrefetch = 8;                          // chunks beyond those prefetched into L2
 constexpr int kTcMBlocks = 8;                           // one per bit position r
 constexpr int kTcN = 16;                                // (head, digit) columns
 constexpr int kTcAccCols = kTcMBlocks * kTcN;           // 128: one tile's accumulators
@@ -126,9 +125,14 @@ __host__ __device__ inline TcPlanLayout tc_plan_layout(int d) {
 
 int tc_plan_bytes(int d) { return tc_plan_layout(d).bytes; }
 
+// Row offset table: one entry per union plane row, padded to whole K-steps.
+__host__ __device__ inline int tc_off_bytes(int d) {
+  return align16(4 * (((4 * d + kTcKStep - 1) / kTcKStep) * kTcKStep));
+}
+
 static int tc_smem_bytes(int d, int S) {
-  int b = 128 + kTcStages * kTcStageBytes + tc_plan_layout(d).bytes + 4 * (S + 1) +
-          kTcEpiWarps * 4 * kTcCandBuf * 8;
+  int b = 128 + kTcStages * kTcStageBytes + tc_off_bytes(d) + tc_plan_layout(d).bytes +
+          4 * (S + 1) + kTcEpiWarps * 4 * kTcCandBuf * 8;
   // more than half an SM's shared memory: one block per SM, so that the
   // block's 512 tensor-memory columns never wait for another block
   return b < 120 * 1024 ? 120 * 1024 : b;
@@ -166,6 +170,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // up after about a second (2^31 cycles).  Returns false on timeout.  Each
 // try_wait may suspend the thread for a system-dependent time until the phase
 // completes (an explicit suspend-time hint measured slower on B200).
+// Non-blocking probe of the phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
@@ -472,12 +488,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const int d = p.d;
   const TcPlanLayout PL = tc_plan_layout(d);
   unsigned char *sStage = smem;
-  unsigned char *sPlan = smem + kTcStages * kTcStageBytes;
+  uint32_t *sOff = reinterpret_cast<uint32_t *>(smem + kTcStages * kTcStageBytes);
+  unsigned char *sPlan = smem + kTcStages * kTcStageBytes + tc_off_bytes(d);
   unsigned long long *sCand = reinterpret_cast<unsigned long long *>(sPlan + PL.bytes);
   int *s_tprefix = reinterpret_cast<int *>(sCand + kTcEpiWarps * 4 * kTcCandBuf);
   const TcPlanHeader *sHdr = reinterpret_cast<const TcPlanHeader *>(sPlan);
   const uint16_t *sRows = reinterpret_cast<const uint16_t *>(sPlan + PL.off_rows);
-  __shared__ __align__(8) unsigned long long s_bar[16];
+  __shared__ __align__(8) unsigned long long s_bar[2 * kTcStages + 12];
   __shared__ uint32_t s_tmem;
   __shared__ int s_tmp[32];
   __shared__ volatile int s_fault;
@@ -489,15 +506,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   auto a_empty = [=](int g, int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 2 * g + b); };
   auto acc_full = [=](int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 4 + b); };
   auto acc_empty = [=](int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 6 + b); };
+  auto a_full = [=](int g, int b) { return bar0 + 8u * (uint32_t)(2 * kTcStages + 8 + 2 * g + b); };
   // A wait that gives up records a fault; the caller carries on (never
   // leaving its warp's named barriers), so that the block still finishes.
   auto wait_or_fault = [&](uint32_t bar, uint32_t parity) {
     if (!s_fault && !mbar_wait(bar, parity)) s_fault = 1;
   };
   // one lane waits, the warp follows
+  // every lane probes (one shared-memory word, so all see the same phase);
+  // only a phase still open sends lane 0 into the bounded wait
   auto warp_wait = [&](uint32_t bar, uint32_t parity) {
-    if (lane == 0) wait_or_fault(bar, parity);
-    __syncwarp();
+    if (!__all_sync(0xffffffffu, mbar_test(bar, parity))) {
+      if (lane == 0) wait_or_fault(bar, parity);
+      __syncwarp();
+    }
   };
   auto warp_arrive = [&](uint32_t bar) {
     __syncwarp();
@@ -535,9 +557,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
       mbar_init(stage_empty(s), kTcBuildWarps);  // every build warp
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(a_empty(0, i), kTcBuildWarps / 2);  // the MMA commits of a build group
-      mbar_init(a_empty(1, i), kTcBuildWarps / 2);
-      mbar_init(acc_full(i), kTcBuildWarps);        // every build warp commits at a tile's end
+      for (int g = 0; g < 2; ++g) {
+        mbar_init(a_full(g, i), kTcBuildWarps / 2);   // the build warps of group g
+        mbar_init(a_empty(g, i), kTcLoadWarps / 2);   // the MMA commits for group g
+      }
+      mbar_init(acc_full(i), kTcLoadWarps);         // every MMA issuer commits at a tile's end
       mbar_init(acc_empty(i), kTcEpiWarps);         // every epilogue warp
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -591,6 +615,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     const int P = sHdr->P;
     const int nks = sHdr->nks;
     const bool big = P > kTcSmallP;  // 0/1 cells instead of 0/2^r
+    // word offset / 4 of every union row within the KV head's planes; the
+    // padding rows of the last K-step repeat its first row (their B weights
+    // are zero, and the repeated row is already on its way from memory)
+    for (int r = tid; r < nks * kTcKStep; r += kTcThreads)
+      sOff[r] = (uint32_t)((int64_t)sRows[r < P ? r : (r & ~(kTcKStep - 1))] * (L0.W >> 2));
+    __syncthreads();
     const int64_t head0 = (int64_t)L0.s * p.h_q + L0.g * G;
     // The segment's K-steps (tile tl, plane block kidx), tile by tile, are
     // taken two at a time: chunk u holds K-steps 2 u and 2 u + 1, which may
@@ -609,18 +639,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
       const int grp = tid >> 3;  // 0 .. 15
       const uint32_t *gbase = L0.planes + (int64_t)L0.g * d * 4 * L0.W;
       const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
-      const bool pf = !p.planes_host;
-      // word offset of this thread's quad in tile ti, or -1 past the data
+      // word offset of this thread's quad in tile ti, clamped into the row:
+      // words past the data hold keys that the epilogue never reports
+      const int64_t wmax = L0.W - 4;
       auto quad_word = [&](int ti) -> int64_t {
         int64_t gw;
         if (MODE == kModeSample) {
           const int64_t sj = (int64_t)ti * kTcSampleSectorsPerTile + (m >> 1);
           gw = sj * kSampleStride * kSectorWords + (m & 1) * 4;
-          if (sj >= nsamp) return -1;
+          if (sj >= nsamp) gw = wmax;
         } else {
           gw = (int64_t)ti * kTcTileWords + m * 4;
         }
-        return gw < L0.W ? gw : -1;
+        return gw < wmax ? gw : wmax;
       };
       // this thread's K-step of a chunk is its half (grp >> 3); a cursor
       // (tile, kidx) walks the K-steps of that half, two K-steps per chunk
@@ -638,36 +669,57 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
       int ltl, lk;  // next K-step to load
       cursor0(ltl, lk);
       auto load_next = [&](uint4 (&v)[4]) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = make_uint4(0u, 0u, 0u, 0u);
         if (ltl < ntiles) {
           const int64_t gw = quad_word(ti0 + ltl);
-          const int r0 = lk * kTcKStep + rgrp;
-          if (gw >= 0) {
+          const uint4 o = *reinterpret_cast<const uint4 *>(sOff + lk * kTcKStep + rgrp);
+          v[0] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.x * 4 + gw));
+          v[1] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.y * 4 + gw));
+          v[2] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.z * 4 + gw));
+          v[3] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.w * 4 + gw));
+        } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              if (r0 + k < P)
-                v[k] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)sRows[r0 + k] * L0.W + gw));
-          }
+          for (int k = 0; k < 4; ++k) v[k] = make_uint4(0u, 0u, 0u, 0u);
         }
         advance(ltl, lk);
       };
-      int ftl, fk;  // next K-step to prefetch into L2
-      cursor0(ftl, fk);
-      auto prefetch_next = [&]() {
-        if (ftl < ntiles && pf && m == 0) {
-          const int64_t gw = quad_word(ti0 + ftl);
-          const int r0 = fk * kTcKStep + rgrp;
-          if (gw >= 0) {
+      // MMA issue: lane 0 of load warp l feeds M-blocks 2 l and 2 l + 1 (build
+      // group l / 2), NS + 1 chunks behind its loads: by the time it has
+      // waited for stage u - NS to be read, the build warps have stored and
+      // signalled chunk u - NS - 1.
+      const int ig = warp >> 1;
+      const uint64_t b_desc0 = tc_smem_desc(tc_smem_u32(sPlan + PL.off_b), kTcLBO, kTcSBO);
+      int itl = 0, ik = 0;  // first K-step of the next chunk to issue
+      auto issue = [&](int v) {
+        const uint32_t ugv = it + (uint32_t)v;
+        const int sbv = (int)(ugv & 1);
+        warp_wait(a_full(ig, sbv), (ugv >> 1) & 1);
+        tc_fence_after();
+        if (lane == 0) {
+          int tl = itl, kx = ik;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              if (r0 + k < P)
-                asm volatile("prefetch.global.L2 [%0];\n" ::"l"(gbase + (int64_t)sRows[r0 + k] * L0.W + gw));
+          for (int ks = 0; ks < 2; ++ks) {
+            if (2 * v + ks < nksteps) {
+              const uint32_t tt = tj + (uint32_t)tl;
+              const int ab = (int)(tt & 1);
+              // a tile's first MMA needs its accumulators read out
+              if (kx == 0 && tt >= 2) wait_or_fault(acc_empty(ab), ((tt >> 1) - 1) & 1);
+              const uint64_t bd = b_desc0 + (uint64_t)(kx * (kTcBChunkBytes >> 4));
+#pragma unroll
+              for (int mb = 0; mb < 2; ++mb) {
+                const int r = 2 * warp + mb;
+                tc_mma(tmem + (uint32_t)(ab * kTcAccCols + kTcN * r),
+                       tmem + (uint32_t)(kTcAColBase + sbv * kTcABufCols + 8 * r + 64 * ks), bd);
+              }
+              if (kx == nks - 1) tc_commit(acc_full(ab));
+            }
+            if (++kx == nks) { kx = 0; ++tl; }
           }
+          tc_commit(a_empty(ig, sbv));
         }
-        advance(ftl, fk);
+        __syncwarp();
+        ik += 2;
+        while (ik >= nks) { ik -= nks; ++itl; }
       };
-      for (int j = 0; j < kTcRing + kTcPrefetch; ++j) prefetch_next();
       uint4 ring[kTcRing][4];
 #pragma unroll
       for (int j = 0; j < kTcRing; ++j) load_next(ring[j]);
@@ -679,6 +731,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
           const uint32_t ug = it + (uint32_t)u;
           const int s = (int)(ug % kTcStages);
           if (ug >= (uint32_t)kTcStages) warp_wait(stage_empty(s), ((ug / kTcStages) - 1) & 1);
+          if (u > kTcStages) issue(u - kTcStages - 1);
           uint32_t *dst = reinterpret_cast<uint32_t *>(sStage + s * kTcStageBytes) + grp * 4 * kTcTileWords + 4 * m;
           uint32_t Tq[4][4];  // [quarter][word]
 #pragma unroll
@@ -697,50 +750,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
             *reinterpret_cast<uint4 *>(dst + q * kTcTileWords) = make_uint4(Tq[q][0], Tq[q][1], Tq[q][2], Tq[q][3]);
           warp_arrive(stage_full(s));
           load_next(ring[jj]);
-          prefetch_next();
         }
       }
+      for (int v = max(0, nchunks - kTcStages - 1); v < nchunks; ++v) issue(v);
     } else if (warp < kTcEpiWarp0) {
-      // -------------------------------------------------------- build + MMA --
+      // ------------------------------------------------------------ build --
       // Build warp (quarter q, group g) writes the cells of M-blocks
-      // 4 g .. 4 g + 3 for its lane quarter, both K-steps of a chunk; after
-      // the four warps of its group have stored, it issues the two MMAs of
-      // M-block 4 g + q.  A chunk's MMAs are issued one chunk late, after the
-      // next chunk's stage has been read, so that the tensor memory stores
-      // have that long to complete.
+      // 4 g .. 4 g + 3 for its lane quarter, both K-steps of a chunk.  It
+      // signals chunk u - 1 (its stores complete) after reading stage u, so
+      // that the tensor memory stores have that long to land.
       const int g = (warp - kTcBuildWarp0) >> 2;
-      const int mrow = 4 * g + quarter;  // the M-block this warp issues
-      // B of K-step kx: the descriptor's address field counts 16-byte units
-      const uint64_t b_desc0 = tc_smem_desc(tc_smem_u32(sPlan + PL.off_b), kTcLBO, kTcSBO);
-      // the MMAs of chunk up, whose first K-step is (tile tl, block kx)
-      auto complete = [&](int up, int tl, int kx) {
-        const uint32_t ug = it + (uint32_t)up;
-        const int sb = (int)(ug & 1);
+      auto signal = [&](int up) {
         tc_wait_st();
         tc_fence_before();
-        named_sync(1 + g, 4 * 32);
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t acl = tmem + (uint32_t)(kTcAColBase + sb * kTcABufCols + 8 * mrow);
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            if (2 * up + ks < nksteps) {
-              const uint32_t tt = tj + (uint32_t)tl;
-              const int ab = (int)(tt & 1);
-              // a tile's first MMA needs its accumulators read out
-              if (kx == 0 && tt >= 2) wait_or_fault(acc_empty(ab), ((tt >> 1) - 1) & 1);
-              tc_mma(tmem + (uint32_t)(ab * kTcAccCols + kTcN * mrow), acl + (uint32_t)(64 * ks),
-                     b_desc0 + (uint64_t)(kx * (kTcBChunkBytes >> 4)));
-              if (kx == nks - 1) tc_commit(acc_full(ab));
-            }
-            if (++kx == nks) { kx = 0; ++tl; }
-          }
-          tc_commit(a_empty(g, sb));
-        }
-        __syncwarp();
+        warp_arrive(a_full(g, (int)((it + (uint32_t)up) & 1)));
       };
-      int btl = 0, bk = 0;  // chunk u's first K-step
-      int ptl = 0, pk = 0;  // chunk u - 1's
       for (int u = 0; u < nchunks; ++u) {
         const uint32_t ug = it + (uint32_t)u;
         const int s = (int)(ug % kTcStages);
@@ -751,7 +775,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) T[i] = src[i * 4 * kTcTileWords];
         warp_arrive(stage_empty(s));
-        if (u > 0) complete(u - 1, ptl, pk);
+        if (u > 0) signal(u - 1);
         // chunk u's A buffer was last read by the MMAs of chunk u - 2
         if (ug >= 2) warp_wait(a_empty(g, sb), ((ug >> 1) - 1) & 1);
         const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + sb * kTcABufCols + 32 * g);
@@ -774,12 +798,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
           }
           tc_st32(acol + (uint32_t)(64 * ks), cell);
         }
-        ptl = btl;
-        pk = bk;
-        bk += 2;
-        while (bk >= nks) { bk -= nks; ++btl; }
       }
-      complete(nchunks - 1, ptl, pk);
+      signal(nchunks - 1);
     } else {
       // ---------------------------------------------------------- epilogue --
       // s = K + Delta 2^-r sum_m 256^m (f_m - M), f_m the accumulator of digit
