@@ -216,6 +216,17 @@ __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint32_t tmem_a, uint64_
       : "memory");
 }
 
+// One lane of the (converged) warp: the lowest.
+__device__ __forceinline__ bool tc_elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t.reg .b32 R;\n\t"
+      "elect.sync R|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
@@ -692,27 +703,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
       auto issue = [&](int v) {
         const uint32_t ugv = it + (uint32_t)v;
         const int sbv = (int)(ugv & 1);
+        // the chunk's two K-steps: (tile, block) and accumulator buffers,
+        // all warp-uniform, worked out before the one elected lane issues
+        const int tl0 = itl, kx0 = ik;
+        const int tl1 = kx0 + 1 == nks ? tl0 + 1 : tl0;
+        const int kx1 = kx0 + 1 == nks ? 0 : kx0 + 1;
+        const bool two = 2 * v + 1 < nksteps;
+        const uint32_t tt0 = tj + (uint32_t)tl0, tt1 = tj + (uint32_t)tl1;
+        // a tile's first MMA needs its accumulators read out
+        if (kx0 == 0 && tt0 >= 2) warp_wait(acc_empty((int)(tt0 & 1)), ((tt0 >> 1) - 1) & 1);
+        if (two && kx1 == 0 && tt1 >= 2) warp_wait(acc_empty((int)(tt1 & 1)), ((tt1 >> 1) - 1) & 1);
         warp_wait(a_full(ig, sbv), (ugv >> 1) & 1);
         tc_fence_after();
-        if (lane == 0) {
-          int tl = itl, kx = ik;
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            if (2 * v + ks < nksteps) {
-              const uint32_t tt = tj + (uint32_t)tl;
-              const int ab = (int)(tt & 1);
-              // a tile's first MMA needs its accumulators read out
-              if (kx == 0 && tt >= 2) wait_or_fault(acc_empty(ab), ((tt >> 1) - 1) & 1);
-              const uint64_t bd = b_desc0 + (uint64_t)(kx * (kTcBChunkBytes >> 4));
-#pragma unroll
-              for (int mb = 0; mb < 2; ++mb) {
-                const int r = 2 * warp + mb;
-                tc_mma(tmem + (uint32_t)(ab * kTcAccCols + kTcN * r),
-                       tmem + (uint32_t)(kTcAColBase + sbv * kTcABufCols + 8 * r + 64 * ks), bd);
-              }
-              if (kx == nks - 1) tc_commit(acc_full(ab));
-            }
-            if (++kx == nks) { kx = 0; ++tl; }
+        const uint32_t acl = tmem + (uint32_t)(kTcAColBase + sbv * kTcABufCols + 16 * warp);
+        const uint32_t d0 = tmem + (uint32_t)((tt0 & 1) * kTcAccCols + 2 * kTcN * warp);
+        const uint32_t d1 = tmem + (uint32_t)((tt1 & 1) * kTcAccCols + 2 * kTcN * warp);
+        const uint64_t bd0 = b_desc0 + (uint64_t)(kx0 * (kTcBChunkBytes >> 4));
+        const uint64_t bd1 = b_desc0 + (uint64_t)(kx1 * (kTcBChunkBytes >> 4));
+        if (tc_elect_one()) {
+          // M-blocks 2 l and 2 l + 1: A columns 8 r (+ 64 for the second K-step)
+          tc_mma(d0, acl, bd0);
+          tc_mma(d0 + kTcN, acl + 8u, bd0);
+          if (kx0 == nks - 1) tc_commit(acc_full((int)(tt0 & 1)));
+          if (two) {
+            tc_mma(d1, acl + 64u, bd1);
+            tc_mma(d1 + kTcN, acl + 72u, bd1);
+            if (kx1 == nks - 1) tc_commit(acc_full((int)(tt1 & 1)));
           }
           tc_commit(a_empty(ig, sbv));
         }
