@@ -174,4 +174,33 @@ __device__ __forceinline__ float load_q(const void *q, int q_bf16, int64_t i) {
   return reinterpret_cast<const float *>(q)[i];
 }
 
+// ------------------------------------------------------- dependent launch --
+// The step's kernels run back to back on one stream.  Each is launched with
+// programmatic stream serialisation: it may be scheduled while its
+// predecessor finishes, and waits (grid_dependency_wait) before it touches
+// anything the predecessor wrote.  Each lets its successor launch early
+// (allow_dependent_launch) as soon as it starts.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace fathom

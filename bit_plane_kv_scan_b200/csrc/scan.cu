@@ -102,6 +102,8 @@ __device__ __forceinline__ void hist_add(unsigned *hist, int digit) {
 // ------------------------------------------------------------ plan kernel --
 
 __global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   const int gid = blockIdx.x;
   const int s = gid / p.h_kv;
   const int g = gid - s * p.h_kv;
@@ -319,6 +321,8 @@ __device__ __forceinline__ void scan_entry(const uint32_t *src, int tstar, int n
 
 template <int G, int MODE>
 __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   extern __shared__ __align__(16) unsigned char smem[];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -798,6 +802,8 @@ __device__ __forceinline__ void find_bin_from_top(const unsigned *hist, unsigned
 // registers (the common case); larger samples are read from memory.
 constexpr int kThrKeys = 16;
 __global__ void __launch_bounds__(1024) threshold_kernel(ScanParams p) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   const int64_t h = blockIdx.x;
   const int s = (int)(h / p.h_q);
   const int64_t n = session_of(p, s).n;
@@ -998,6 +1004,8 @@ constexpr int kMergeKeys = 8;
 constexpr int kBinSortMax = 256;
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int kpow2,
                                                               int sort_cap) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   // [sort_cap] placed candidates, then [sort_cap] ranked (sort_cap = 8 blockDim >= kpow2)
   extern __shared__ unsigned long long s_out[];
   unsigned long long *s_rank = s_out + sort_cap;
@@ -1243,8 +1251,7 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
   if (any_sampling) {
     e = tc ? launch_tc_scan(p, kModeSample, sms, stream) : launch_scan_m<kModeSample>(p, stream);
     if (e != cudaSuccess) return e;
-    threshold_kernel<<<heads, 1024, 0, stream>>>(p);
-    e = cudaGetLastError();
+    e = launch_dependent(threshold_kernel, dim3(heads), dim3(1024), 0, stream, p);
     if (e != cudaSuccess) return e;
   }
   if (p.prof_begin) {
@@ -1265,8 +1272,8 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
   const int msmem = 2 * sort_cap * 8;
   e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
   if (e != cudaSuccess) return e;
-  merge_kernel<<<heads, kMergeThreads, msmem, stream>>>(p, kpow2, sort_cap);
-  return cudaGetLastError();
+  return launch_dependent(merge_kernel, dim3(heads), dim3(kMergeThreads), (size_t)msmem, stream, p,
+                          kpow2, sort_cap);
 }
 
 }  // namespace fathom

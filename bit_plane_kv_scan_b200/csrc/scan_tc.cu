@@ -301,6 +301,8 @@ __device__ int tc_block_scan(int v, int *s_tmp) {
 
 // One block of 256 threads per (session, KV head); thread c is channel c.
 __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   const int gid = blockIdx.x;
   const int s = gid / p.h_kv;
   const int g = gid - s * p.h_kv;
@@ -325,7 +327,10 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   if (c < d) {
     const double m = se.qmin[(int64_t)g * d + c];
     const double sc = se.qscale[(int64_t)g * d + c];
-    for (int hh = 0; hh < G; ++hh) {
+    // fixed trip count, so that t, w and kpart stay in registers
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+      if (hh >= G) break;
       const int64_t hq = (int64_t)(g * G + hh) * d + c;
       t[hh] = se.alloc[hq];
       const double qv = load_q(se.q, p.q_bf16, hq);
@@ -362,13 +367,15 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   // not read a plane contribute nothing)
   for (int i = threadIdx.x; i < nks * kTcBChunkBytes / 16; i += blockDim.x)
     reinterpret_cast<uint4 *>(bmat)[i] = make_uint4(0, 0, 0, 0);
-  double delta[4];
+  double delta[4], inv_delta[4];
+#pragma unroll
   for (int hh = 0; hh < 4; ++hh) {
     // the largest plane weight is 8 max_c |q_c s_c|; W / Delta < 2^30
     const double wmax = 8.0 * __longlong_as_double((long long)s_wmax[hh]);
     int ex = 0;
     frexp(wmax, &ex);  // wmax < 2^ex
     delta[hh] = wmax > 0.0 ? ldexp(1.0, ex - 30) : 1.0;
+    inv_delta[hh] = wmax > 0.0 ? ldexp(1.0, 30 - ex) : 1.0;  // exact: a power of two
   }
   if (threadIdx.x == 0) {
     hdr->P = P;
@@ -390,9 +397,13 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
     rows[pl] = (uint16_t)(c * 4 + j);
     int8_t *bk = bmat + (size_t)(pl / kTcKStep) * kTcBChunkBytes;
     const int k = pl % kTcKStep;
-    for (int hh = 0; hh < G; ++hh) {
-      if (j >= t[hh]) continue;
-      long long x = llrint(ldexp(w[hh], 3 - j) / delta[hh]);
+    const double pj = (double)(1 << (3 - j));  // 2^(3 - j), j <= 3
+#pragma unroll
+    for (int hh = 0; hh < 4; ++hh) {
+      if (hh >= G || j >= t[hh]) continue;
+      // W / Delta scaled by powers of two only: exact, then rounded once
+      long long x = __double2ll_rn(w[hh] * pj * inv_delta[hh]);
+#pragma unroll
       for (int dg = 0; dg < 4; ++dg) {
         const long long v = dg < 3 ? ((x + 128) & 255) - 128 : x;
         x = (x - v) >> 8;
@@ -492,6 +503,8 @@ __device__ __noinline__ void tc_append(const ScanParams &p, int64_t head0, int G
 
 template <int G, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -962,8 +975,7 @@ static cudaError_t launch_tc_gm(const ScanParams &p, int sms, cudaStream_t strea
   cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<G, MODE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  tc_scan_kernel<G, MODE><<<sms, kTcThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(tc_scan_kernel<G, MODE>, dim3(sms), dim3(kTcThreads), (size_t)smem, stream, p);
 }
 
 cudaError_t launch_tc_plan(const ScanParams &p, cudaStream_t stream) {
