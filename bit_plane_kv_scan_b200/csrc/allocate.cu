@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(1024) allocate_kernel(const void *__restrict__
                                                         const float *__restrict__ sigma, int G,
                                                         int d, int budget,
                                                         uint8_t *__restrict__ alloc) {
+  grid_dependency_wait();
+  allow_dependent_launch();
   const int h = blockIdx.x;
   const int slot = threadIdx.x;  // 4 c + tau, slot < 4 d = blockDim.x
   const int c = slot >> 2, tau = slot & 3;
@@ -104,8 +106,8 @@ __global__ void __launch_bounds__(1024) allocate_kernel(const void *__restrict__
 cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
                             int budget, uint8_t *alloc, cudaStream_t stream) {
   const int G = h_q / h_kv;
-  allocate_kernel<<<h_q, 4 * d, 0, stream>>>(q, q_bf16, sigma, G, d, budget, alloc);
-  return cudaGetLastError();
+  return launch_dependent(allocate_kernel, dim3(h_q), dim3(4 * d), 0, stream, q, q_bf16, sigma,
+                          G, d, budget, alloc);
 }
 
 }  // namespace fathom

@@ -120,6 +120,9 @@ WsLayout ws_layout(int S, int64_t n_max, int d, int h_q, int h_kv, int k, uint32
 
 void fill_ws(ScanParams &p, const WsLayout &L, void *ws) {
   unsigned char *b = static_cast<unsigned char *>(ws);
+  p.zero = reinterpret_cast<uint32_t *>(b);
+  p.zero_words = (int)(L.zero_bytes / 4);
+  p.plan_stride = (p.flags & FATHOM_FLAG_CUDA_CORES) ? plan_layout(p.d).bytes : tc_plan_bytes(p.d);
   p.status = reinterpret_cast<WsStatus *>(b);
   p.counts = reinterpret_cast<uint32_t *>(b + L.off_counts);
   p.tau = reinterpret_cast<uint32_t *>(b + L.off_tau);
@@ -266,9 +269,8 @@ fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_by
   p.prof_begin = g_prof_begin;
   p.prof_end = g_prof_end;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
-  e = launch_scan_pipeline(p, sampling_on(a->n, L.sample_rank, a->flags), s);
+  // the plan kernel clears the workspace's status, counters and thresholds
+  cudaError_t e = launch_scan_pipeline(p, sampling_on(a->n, L.sample_rank, a->flags), s);
   if (e != cudaSuccess) return cuda_fail(e, "scan launch");
   return ok();
 }
@@ -320,9 +322,7 @@ fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, s
   p.prof_begin = g_prof_begin;
   p.prof_end = g_prof_end;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
-  e = launch_scan_pipeline(p, L.m_max > 0, s);
+  cudaError_t e = launch_scan_pipeline(p, L.m_max > 0, s);
   if (e != cudaSuccess) return cuda_fail(e, "scan launch");
   return ok();
 }

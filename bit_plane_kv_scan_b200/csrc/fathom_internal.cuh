@@ -113,6 +113,9 @@ struct ScanParams {
   int64_t cap;      // candidate capacity per query head
   int64_t m_max;    // sample slots per query head
   // workspace
+  uint32_t *zero;    // prefix of the workspace the plan kernel clears (status, counts, tau)
+  int zero_words;
+  int plan_stride;   // bytes between consecutive plans
   WsStatus *status;
   uint32_t *counts;  // [S * h_q] candidate counts
   uint32_t *tau;     // [S * h_q] threshold keys (0 = keep every key)

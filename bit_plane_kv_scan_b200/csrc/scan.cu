@@ -104,6 +104,10 @@ __device__ __forceinline__ void hist_add(unsigned *hist, int digit) {
 __global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
   grid_dependency_wait();
   allow_dependent_launch();
+  // clear the workspace's status, counters and thresholds (read by the
+  // kernels after this one)
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_words; i += gridDim.x * blockDim.x)
+    p.zero[i] = 0u;
   const int gid = blockIdx.x;
   const int s = gid / p.h_kv;
   const int g = gid - s * p.h_kv;
@@ -210,7 +214,6 @@ __global__ void __launch_bounds__(256) plan_kernel(ScanParams p) {
       hdr->K[hh] = (float)sum;
       hdr->tau[hh] = -INFINITY;
     }
-    atomicAdd(&p.status->union_planes, (uint32_t)nplanes);
   }
 }
 
@@ -1006,6 +1009,26 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
                                                               int sort_cap) {
   grid_dependency_wait();
   allow_dependent_launch();
+  if (blockIdx.x == 0) {
+    // union planes of every (session, KV head), from the plan headers
+    __shared__ unsigned s_up[32];
+    unsigned v = 0;
+    for (int gid = threadIdx.x; gid < p.S * p.h_kv; gid += blockDim.x) {
+      const unsigned char *plan = p.plans + (size_t)gid * p.plan_stride;
+      v += (p.flags & FATHOM_FLAG_CUDA_CORES)
+               ? (unsigned)reinterpret_cast<const PlanHeader *>(plan)->union_planes
+               : (unsigned)*reinterpret_cast<const int *>(plan);  // the tc plan's P
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0) s_up[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned t = 0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += s_up[w];
+      p.status->union_planes = t;
+    }
+  }
   // [sort_cap] placed candidates, then [sort_cap] ranked (sort_cap = 8 blockDim >= kpow2)
   extern __shared__ unsigned long long s_out[];
   unsigned long long *s_rank = s_out + sort_cap;
@@ -1244,8 +1267,7 @@ cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStr
   if (tc) {
     e = launch_tc_plan(p, stream);
   } else {
-    plan_kernel<<<p.S * p.h_kv, 256, 0, stream>>>(p);
-    e = cudaGetLastError();
+    e = launch_dependent(plan_kernel, dim3(p.S * p.h_kv), dim3(256), 0, stream, p);
   }
   if (e != cudaSuccess) return e;
   if (any_sampling) {

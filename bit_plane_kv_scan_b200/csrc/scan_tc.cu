@@ -303,6 +303,10 @@ __device__ int tc_block_scan(int v, int *s_tmp) {
 __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   grid_dependency_wait();
   allow_dependent_launch();
+  // clear the workspace's status, counters and thresholds (read by the
+  // kernels after this one)
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_words; i += gridDim.x * blockDim.x)
+    p.zero[i] = 0u;
   const int gid = blockIdx.x;
   const int s = gid / p.h_kv;
   const int g = gid - s * p.h_kv;
@@ -389,7 +393,6 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
       hdr->D[hh] = (float)delta[hh];
       hdr->pad2[hh] = 0.0f;
     }
-    atomicAdd(&p.status->union_planes, (uint32_t)P);
   }
   __syncthreads();
   for (int j = 0; j < tstar; ++j) {
@@ -503,7 +506,9 @@ __device__ __noinline__ void tc_append(const ScanParams &p, int64_t head0, int G
 
 template <int G, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
-  grid_dependency_wait();
+  // the prologue below (tile space, tensor memory, barriers) reads only the
+  // call's inputs, so it overlaps the previous kernel; the plans, thresholds
+  // and counters that kernel writes are read after grid_dependency_wait
   allow_dependent_launch();
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x;
@@ -613,6 +618,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+
+  grid_dependency_wait();
 
   // chunks and tiles since the start of the kernel
   uint32_t it = 0, tj = 0;
@@ -979,8 +986,7 @@ static cudaError_t launch_tc_gm(const ScanParams &p, int sms, cudaStream_t strea
 }
 
 cudaError_t launch_tc_plan(const ScanParams &p, cudaStream_t stream) {
-  tc_plan_kernel<<<p.S * p.h_kv, 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(tc_plan_kernel, dim3(p.S * p.h_kv), dim3(256), 0, stream, p);
 }
 
 cudaError_t launch_tc_scan(const ScanParams &p, int mode, int sms, cudaStream_t stream) {
