@@ -13,7 +13,9 @@ One step = fathom_allocate + fathom_scan_topk (plan, sample scan, threshold,
 filtering scan, merge).  Device time per step comes from CUDA events on the
 launching stream; L2 is flushed (256 MiB write) between steps, outside the
 events.  The dominant kernel (the filtering scan) is timed alone with events
-the library records around it.
+the library records around it, in K further steps: an event between two
+kernels breaks their programmatic dependent launch, so the step time is
+taken without them.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
                     [--config NAME] [--budget B]
@@ -440,10 +442,18 @@ def run_native(args):
     sampler.start()
     for i in range(K):
         flush.zero_()
-        F.profile_scan_kernel(kb[i], ke[i])
         sb[i].record(stream)
         step()
         se[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    # The filtering scan alone, timed with events the library records around
+    # it in K more steps: events between two kernels break their dependent
+    # launch, so the step time above is taken without them.
+    for i in range(K):
+        flush.zero_()
+        F.profile_scan_kernel(kb[i], ke[i])
+        step()
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()

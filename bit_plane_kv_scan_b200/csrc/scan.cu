@@ -996,9 +996,9 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
 // One block per head (kMergeThreads = 1024 threads).  Usually the
 // candidates fit in registers (kMergeKeys a thread): they are binned by score
 // (kSelBins equal bins between their min and max, monotone in the score) and
-// the bin b holding the k-th best is found; the candidates from b up are
-// binned again over their own, narrower range, so that a bin holds a handful
-// of keys.  They are placed bin by bin from the top (a counting sort); then
+// the bin b holding the k-th best is found.  Candidates sit near the
+// threshold, whose upper tail thins out fast, so a bin at or above b holds a
+// handful of keys.  They are placed bin by bin from the top (a counting sort); then
 // each candidate's place inside its bin is its rank there (the count of
 // larger composites in the bin: descending composite = score desc, index
 // asc).  The first k are the answer.  Crowded bins fall back to a register
@@ -1098,27 +1098,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
     }
     __syncthreads();
     int bstar = block_hist_find(hist, (unsigned)k, s_wsum, &s_bin, &s_above);
-    // second level: rebin the candidates of bins >= bstar over [their min, hi]
-    {
-      float lo2 = INFINITY, hi2 = -INFINITY;
+    // candidates below the k-th best's bin take no further part
 #pragma unroll
-      for (int j = 0; j < kMergeKeys; ++j)
-        if (bin[j] >= bstar) lo2 = fminf(lo2, key_float((uint32_t)(c[j] >> 32)));
-      for (int i = tid; i < kSelBins; i += nthr) hist[i] = 0u;
-      block_minmax(lo2, hi2, s_mm);
-      const float scale2 = hi > lo2 ? (float)kSelBins / (hi - lo2) : 0.0f;
-#pragma unroll
-      for (int j = 0; j < kMergeKeys; ++j) {
-        if (bin[j] >= bstar) {
-          bin[j] = sel_bin(key_float((uint32_t)(c[j] >> 32)), lo2, scale2);
-          atomicAdd(&hist[bin[j]], 1u);
-        } else {
-          bin[j] = -1;
-        }
-      }
-      __syncthreads();
-      bstar = block_hist_find(hist, (unsigned)k, s_wsum, &s_bin, &s_above);
-    }
+    for (int j = 0; j < kMergeKeys; ++j)
+      if (bin[j] < bstar) bin[j] = -1;
     // exclusive offsets of the bins in top order: thread t owns top-order
     // positions 4 t .. 4 t + 3 (bins kSelBins - 1 - 4 t - q)
     {
