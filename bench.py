@@ -217,27 +217,38 @@ def get_cfg(name):
 
 
 
+def code_digest(path):
+    """sha256 of a C++/CUDA source with its comments and blank lines removed,
+    so that an edit to comments alone keeps a profile's counters valid."""
+    import hashlib
+    with open(path) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.split("\n")]
+    code = "\n".join(ln for ln in lines if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()
+
+
 def profiled_traffic(workload, kernel_source):
     """DRAM bytes (read + write) per launch of the filtering scan, from the ncu
-    summaries under profiles/ -- only while the kernel source hashes to the one
-    the counters were taken on and the workload matches; else None."""
+    summaries under profiles/ -- only while the kernel source (comments aside)
+    hashes to the one the counters were taken on and the workload matches;
+    else None."""
     import glob
-    import hashlib
     src = os.path.join(ROOT, kernel_source)
     if not os.path.exists(src):
         return None
-    with open(src, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
+    digest = code_digest(src)
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         fields = {}
         with open(path) as f:
             for line in f:
-                m = re.match(r"^(traffic_bytes_per_launch|kernel_source|kernel_source_sha256|workload): (\S+)$",
+                m = re.match(r"^(traffic_bytes_per_launch|kernel_source|kernel_code_sha256|workload): (\S+)$",
                              line.strip())
                 if m:
                     fields[m.group(1)] = m.group(2)
         if (fields.get("kernel_source") == kernel_source and fields.get("workload") == workload
-                and fields.get("kernel_source_sha256") == digest
+                and fields.get("kernel_code_sha256") == digest
                 and "traffic_bytes_per_launch" in fields):
             return int(fields["traffic_bytes_per_launch"])
     return None

@@ -18,10 +18,9 @@
 // Layout (B200 design).  A tile is 1024 keys of one KV head: 32 plane words
 // per plane.  Tensor-memory lane (quarter q, lane l) of M-block r (r < 8)
 // stands for key 32 l + 8 q + r of the tile: word l, byte q, bit r.  Plane
-// rows are taken four at a time; the warp of lane quarter q gathers byte q
-// of the four words of its lane with three byte permutes,
-//   T = [x0.byte q, x1.byte q, x2.byte q, x3.byte q],
-// and M-block r receives the 32-bit cell T & (0x01010101 << r): four int8 K
+// rows are taken four at a time, and byte q of the four rows' word l forms
+//   T = [x0.byte q, x1.byte q, x2.byte q, x3.byte q];
+// M-block r receives the 32-bit cell T & (0x01010101 << r): four int8 K
 // elements, one per plane, each 0 or 2^r (undone by the epilogue's scale).
 // Every key has its own row and B has N = 16 columns (head, digit).
 //
@@ -35,9 +34,10 @@
 //    registers; row addresses from a per-segment offset table), transposes
 //    the bytes so that T = [x0.q, x1.q, x2.q, x3.q] for each lane quarter q,
 //    and stores them in a four-stage shared-memory ring, where a build warp
-//    reads its T values conflict-free.  Lane 0 of load warp l also issues
-//    the MMAs of M-blocks 2 l and 2 l + 1, five chunks behind its loads:
-//    four issuers, every accumulator region always fed by the same thread.
+//    reads its T values conflict-free.  One elected lane of load warp l also
+//    issues the MMAs of M-blocks 2 l and 2 l + 1, five chunks behind its
+//    loads: four issuers, every accumulator region always fed by the same
+//    thread.
 //  * Build warps 4-11 (lane quarter w % 4, group g = M-blocks 4 g .. 4 g + 3)
 //    write the cells of their M-blocks for both K-steps to tensor memory (two
 //    32-column stores) and signal them one chunk later, after reading the

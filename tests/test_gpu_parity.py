@@ -196,6 +196,26 @@ def test_k_larger_than_n_and_empty():
     assert (_np(idx) == -1).all() and np.isneginf(_np(sc)).all()
 
 
+@pytest.mark.parametrize("cuda_cores", [False, True])
+def test_report_counts_and_workspace_reuse(cuda_cores):
+    """The report's union-plane count is the sum over KV heads of every
+    channel's largest prefix in its query-head group (the bytes the scan
+    reads, in plane rows), and a second scan on the same workspace reports
+    its own counts: the status, counters and thresholds are cleared by the
+    scan itself, with no memset."""
+    case = synthkv.make_case(seed=23, n=40000, h_kv=2, h_q=8, d=128, q_dtype="bf16")
+    G = case.h_q // case.h_kv
+    base = F.FLAG_CUDA_CORES if cuda_cores else 0
+    for budget, extra in ((92, F.FLAG_FORCE_FALLBACK), (136, 0), (92, 0)):
+        _, alloc, (idx, sc) = run_gpu(case, budget, 64, flags=base | extra)
+        rep = F.read_report()
+        t = _np(alloc).astype(np.int64).reshape(case.h_kv, G, case.d)
+        assert rep.union_planes == int(t.max(axis=1).sum())
+        assert rep.fallback_heads == (case.h_q if extra else 0)
+        assert rep.device_faults == 0
+        assert 64 <= rep.max_candidates
+
+
 def test_sampled_threshold_path_and_fallbacks():
     """n large enough that the sampled threshold is used (k=64 samples from
     n >= 8192); the forced fallback and the no-sampling path must give the
