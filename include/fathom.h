@@ -27,7 +27,10 @@
  *     prefixes across the host link.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     stream-ordered and asynchronous: none synchronises the host except
- *     fathom_scan_read_report.
+ *     fathom_scan_read_report.  Kernels are launched with programmatic
+ *     stream serialisation: one may be scheduled while the stream's previous
+ *     kernel finishes, but waits for that kernel to complete before it reads
+ *     or writes anything; ordering with the caller's own work is unchanged.
  *   - Every call validates its arguments on the host before any launch and
  *     returns a status; on error nothing is launched and
  *     fathom_last_error() holds a message.  No C++ exception crosses the ABI.
@@ -230,7 +233,9 @@ FATHOM_API fathom_status fathom_scan_topk_noalloc(const fathom_scan_args *args, 
  * records `begin` (a cudaEvent_t) on its stream just before the filtering scan
  * kernel -- the kernel that streams the union plane prefixes -- and `end`
  * just after it, so a caller can time that kernel alone with
- * cudaEventElapsedTime.  Pass NULL, NULL to clear.  Never synchronises. */
+ * cudaEventElapsedTime.  Pass NULL, NULL to clear.  Never synchronises.
+ * The two events stop the kernels around the filtering scan from overlapping
+ * it, so time whole steps without them. */
 FATHOM_API void fathom_profile_scan_kernel(void *begin, void *end);
 
 /* What the last scan on a workspace recorded.  Synchronises `stream`. */
