@@ -4,58 +4,93 @@
 // "a prefix of t planes is exactly the channel's t-bit quantizer").
 //
 // One block turns 1024 tokens (32 plane words) of one KV head into every
-// plane row of those words.  Warp w owns word w: lane b loads token 32w+b's
-// d/2 code bytes with 16-byte loads, and one warp vote per (channel, plane)
-// yields the plane word directly.  The words are staged in shared memory
-// and written out as 128-byte row segments.  Integer and bit-exact; the
-// transpose reads and writes each byte of the store once (HBM-bound).
+// plane row of those words.  Thread (token group tg, code word cw) loads the
+// 32-bit code word cw (channels 8 cw .. 8 cw + 7) of the 32 tokens of group
+// tg, one coalesced 4-byte load each, and transposes that 32 x 32 bit matrix
+// in registers (byte permutes for the 16- and 8-bit block swaps, masked
+// shift-xor swaps below that).  Afterwards register i holds bit i of the
+// code word for all 32 tokens: the plane word of (channel, plane) that bit i
+// encodes.  The words are staged in shared memory and written out as
+// 128-byte row segments.  Integer and bit-exact; each byte of the store is
+// read and written once (HBM-bound).
 #include "fathom_internal.cuh"
 
 namespace fathom {
 
-template <int D>
-__global__ void __launch_bounds__(1024) pack_kernel(const uint8_t *__restrict__ codes, int64_t n,
-                                                    uint32_t *__restrict__ planes, int64_t W) {
-  extern __shared__ uint32_t sm_words[];  // [D * 4 rows][32 words]
-  constexpr int kVec = D / 32;            // 16-byte vectors per token (D/2 bytes)
-  const int g = blockIdx.y;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int64_t w0 = (int64_t)blockIdx.x * 32;
-  const int64_t tok = (w0 + warp) * 32 + lane;
-
-  uint32_t v[kVec * 4];
-  if (tok < n) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(codes + ((int64_t)g * n + tok) * (D / 2));
-#pragma unroll
-    for (int i = 0; i < kVec; ++i) {
-      uint4 x = __ldg(src + i);
-      v[4 * i + 0] = x.x;
-      v[4 * i + 1] = x.y;
-      v[4 * i + 2] = x.z;
-      v[4 * i + 3] = x.w;
-    }
+// Swaps the off-diagonal halves of the 2 x 2 blocks of width J in the bit
+// matrix rows a (upper) and b (lower): the bits of a at positions with bit J
+// set trade places with the bits of b at positions J lower.
+template <int J>
+__device__ __forceinline__ void swap_blocks(uint32_t &a, uint32_t &b) {
+  if (J == 16) {
+    const uint32_t na = __byte_perm(a, b, 0x5410), nb = __byte_perm(a, b, 0x7632);
+    a = na;
+    b = nb;
+  } else if (J == 8) {
+    const uint32_t na = __byte_perm(a, b, 0x6240), nb = __byte_perm(a, b, 0x7351);
+    a = na;
+    b = nb;
   } else {
-#pragma unroll
-    for (int i = 0; i < kVec * 4; ++i) v[i] = 0u;
+    constexpr uint32_t m = J == 4 ? 0x0F0F0F0Fu : J == 2 ? 0x33333333u : 0x55555555u;
+    const uint32_t t = ((a >> J) ^ b) & m;
+    b ^= t;
+    a ^= t << J;
   }
+}
 
+template <int J>
+__device__ __forceinline__ void transpose_stage(uint32_t (&x)[32]) {
 #pragma unroll
-  for (int c = 0; c < D; ++c) {
-    // channel c is nibble c % 8 of 32-bit word c / 8 (low nibble = even channel)
-    const uint32_t u = (v[c >> 3] >> (4 * (c & 7))) & 15u;
+  for (int t = 0; t < 32; ++t)
+    if ((t & J) == 0) swap_blocks<J>(x[t], x[t + J]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(D * 4) pack_kernel(const uint8_t *__restrict__ codes, int64_t n,
+                                                   uint32_t *__restrict__ planes, int64_t W) {
+  constexpr int kWordsPerToken = D / 8;        // 32-bit code words (8 channels each)
+  constexpr int kThreads = 32 * kWordsPerToken;
+  constexpr int kRows = 4 * D;                 // plane rows c * 4 + j of one KV head
+  // shared-memory column rotation per code word, so that the 32 lanes of a
+  // warp store into 32 different banks
+  constexpr int kRot = kWordsPerToken >= 32 ? 1 : 32 / kWordsPerToken;
+  extern __shared__ uint32_t sm_words[];  // [kRows][32], row r rotated by kRot * (r / 32)
+  const int g = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int tg = tid / kWordsPerToken;
+  const int cw = tid - tg * kWordsPerToken;
+  const int64_t w0 = (int64_t)blockIdx.x * 32;
+  const int64_t tok0 = (w0 + tg) * 32;
+  const uint32_t *src = reinterpret_cast<const uint32_t *>(codes + (int64_t)g * n * (D / 2)) + cw;
+
+  uint32_t x[32];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t word = __ballot_sync(0xffffffffu, (u >> (3 - j)) & 1u);
-      if (lane == 0) sm_words[(c * 4 + j) * 32 + warp] = word;
-    }
+  for (int t = 0; t < 32; ++t) {
+    const int64_t tok = tok0 + t;
+    x[t] = tok < n ? __ldg(src + tok * kWordsPerToken) : 0u;
+  }
+  transpose_stage<16>(x);
+  transpose_stage<8>(x);
+  transpose_stage<4>(x);
+  transpose_stage<2>(x);
+  transpose_stage<1>(x);
+
+  // bit i of code word cw is bit i % 4 of nibble (i / 4) % 2 of byte i / 8:
+  // channel 8 cw + 2 (i / 8) + (i / 4) % 2, plane 3 - i % 4
+  const int col = (tg + kRot * cw) & 31;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int row = 32 * cw + 4 * (2 * (i >> 3) + ((i >> 2) & 1)) + 3 - (i & 3);
+    sm_words[row * 32 + col] = x[i];
   }
   __syncthreads();
 
-  for (int idx = threadIdx.x; idx < D * 4 * 32; idx += 1024) {
-    const int row = idx >> 5;
-    const int64_t w = w0 + (idx & 31);
-    if (w < W) planes[((int64_t)g * D * 4 + row) * W + w] = sm_words[idx];
+  const int lane = tid & 31;
+  const int64_t w = w0 + lane;
+  if (w < W) {
+    uint32_t *dst = planes + (int64_t)g * kRows * W + w;
+    for (int row = tid >> 5; row < kRows; row += kThreads / 32)
+      dst[(int64_t)row * W] = sm_words[row * 32 + ((lane + kRot * (row >> 5)) & 31)];
   }
 }
 
@@ -72,7 +107,7 @@ static cudaError_t launch_pack_d(const uint8_t *codes, int64_t n, int h_kv, uint
     configured = true;
   }
   dim3 grid((unsigned)((W + 31) / 32), (unsigned)h_kv);
-  pack_kernel<D><<<grid, 1024, smem, stream>>>(codes, n, planes, W);
+  pack_kernel<D><<<grid, D * 4, smem, stream>>>(codes, n, planes, W);
   return cudaGetLastError();
 }
 

@@ -75,7 +75,8 @@ def case_np(case):
 # ------------------------------------------------------------------ pack --
 
 @pytest.mark.parametrize("n,d,h_kv", [(1, 32, 1), (31, 64, 2), (4096, 128, 1), (4097, 128, 2),
-                                      (33333, 256, 1), (100000, 96, 3)])
+                                      (33333, 256, 1), (100000, 96, 3), (5000, 160, 2),
+                                      (1025, 192, 1), (70000, 224, 1)])
 def test_pack_bit_exact(n, d, h_kv):
     rng = np.random.default_rng(n + d)
     codes = rng.integers(0, 256, size=(h_kv, n, d // 2), dtype=np.uint8)
