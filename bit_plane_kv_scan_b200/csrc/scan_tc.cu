@@ -454,6 +454,43 @@ __device__ __forceinline__ TcLoc tc_locate(const ScanParams &p, const int *s_tpr
   return L;
 }
 
+// A block whose tiles span two (session, KV head) groups drains its pipeline
+// between them (measured: about 2.5 tiles of work).  The filtering pass
+// splits the tiles over the blocks on a cost line on which every group is
+// preceded by that overhead, so that a block that crosses a group boundary
+// takes correspondingly fewer tiles.  Costs are in half tiles.
+constexpr int kTcSwitchHalfTiles = 5;
+
+// Cost position of global tile k: 2 k + sw (groups up to and including k's).
+template <int MODE>
+__device__ __forceinline__ int64_t tc_cost_pos(const ScanParams &p, const int *s_tprefix, int k,
+                                               int64_t sw) {
+  int lo = 0, hi = p.S;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_tprefix[mid] <= k) lo = mid; else hi = mid;
+  }
+  const int per = (int)tc_tiles_per_group<MODE>(session_of(p, lo).n, p);
+  const int64_t group = (int64_t)lo * p.h_kv + (k - s_tprefix[lo]) / per;
+  return 2 * (int64_t)k + sw * (group + 1);
+}
+
+// First tile of block b (b = nblocks gives the tile count): the first tile
+// whose cost position is at or past b / nblocks of the cost line.
+template <int MODE>
+__device__ int tc_split_point(const ScanParams &p, const int *s_tprefix, int b, int nblocks) {
+  const int total = s_tprefix[p.S];
+  const int64_t sw = MODE == kModeFilter ? kTcSwitchHalfTiles : 0;
+  const int64_t cost_total = 2 * (int64_t)total + sw * p.S * p.h_kv;
+  const int64_t c = cost_total * b / nblocks;
+  int lo = 0, hi = total;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (tc_cost_pos<MODE>(p, s_tprefix, mid, sw) < c) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
 // Writes the n buffered candidates of one head to the candidate buffer: one
 // global atomic reserves their places.  All lanes of the warp call it.  Out
 // of line: it runs about once per 64 candidates, and the scoring loop keeps
@@ -567,9 +604,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     if (base == 0 && tid == 0) s_tprefix[0] = 0;
     __syncthreads();
   }
-  const int total = s_tprefix[p.S];
-  const int t_begin = (int)(((int64_t)blockIdx.x * total) / gridDim.x);
-  const int t_end = (int)(((int64_t)(blockIdx.x + 1) * total) / gridDim.x);
+  if (tid < 2) s_tmp[tid] = tc_split_point<MODE>(p, s_tprefix, (int)blockIdx.x + tid, (int)gridDim.x);
+  __syncthreads();
+  const int t_begin = s_tmp[0];
+  const int t_end = s_tmp[1];
   if (t_begin >= t_end) return;
 
   // ---- tensor memory, barriers, preset accumulators ----------------------
