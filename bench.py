@@ -64,6 +64,9 @@ def parse(argv=None):
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--cuda-cores", action="store_true",
                     help="run the scan on the CUDA-core kernel instead of the tcgen05 kernel")
+    ap.add_argument("--uniform", action="store_true",
+                    help="allocate the budget query-independently (the same depth in every "
+                         "channel, fathom_allocate_uniform) instead of by water-filling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -258,17 +261,19 @@ def profiled_traffic(workload, kernel_source):
             return int(fields["traffic_bytes_per_launch"])
     return None
 
-def workload_desc(cfg, budget, k):
+def workload_desc(cfg, budget, k, uniform=False):
+    how = (", uniform allocation (the same depth in every channel for every query head)"
+           if uniform else "")
     if cfg["name"] == "ragged_32_sessions":
         return ("ragged_32_sessions: 32 sessions, n ~ U[%d, %d] keys each, %d KV heads x d=%d, "
-                "%d %s query heads (GQA %d), B=%d bits/key, top-k=%d, one batched launch set" % (
+                "%d %s query heads (GQA %d), B=%d bits/key%s, top-k=%d, one batched launch set" % (
                     cfg["n_lo"], cfg["n_hi"], cfg["h_kv"], cfg["d"], cfg["h_q"], cfg["q_dtype"],
-                    cfg["h_q"] // cfg["h_kv"], budget, k))
+                    cfg["h_q"] // cfg["h_kv"], budget, how, k))
     where = " in pinned host memory" if cfg["name"] == "host_resident_1m" else ""
     return ("%s: n=%d keys, %d KV heads x d=%d (4-bit channel-major bit planes%s), %d %s query "
-            "heads (GQA %d), B=%d bits/key, top-k=%d" % (
+            "heads (GQA %d), B=%d bits/key%s, top-k=%d" % (
                 cfg["name"], cfg["n"], cfg["h_kv"], cfg["d"], where, cfg["h_q"], cfg["q_dtype"],
-                cfg["h_q"] // cfg["h_kv"], budget, k))
+                cfg["h_q"] // cfg["h_kv"], budget, how, k))
 
 
 def union_plane_bytes(alloc, n, h_kv, words):
@@ -283,15 +288,19 @@ def union_plane_bytes(alloc, n, h_kv, words):
 
 # ------------------------------------------------------------ CPU oracle --
 
-def oracle_sample(case_np, budget, k, heads):
+def oracle_sample(case_np, budget, k, heads, uniform=False):
     """Oracle allocation + scores + top-k for the listed query heads; returns seconds."""
     import oracle
     codes, qmin, qscale, q, sigma = case_np
     G = q.shape[0] // codes.shape[0]
+    d = q.shape[1]
     t0 = time.perf_counter()
     for h in heads:
         g = h // G
-        t = oracle.allocate(q[h], sigma[g], budget)
+        if uniform:
+            t = oracle.allocate_uniform(1, d, budget)[0]
+        else:
+            t = oracle.allocate(q[h], sigma[g], budget)
         s = oracle.scores_from_codes(codes[g], qmin[g], qscale[g], q[h], t)
         oracle.topk(s, k)
     return time.perf_counter() - t0
@@ -322,8 +331,8 @@ def run_reference(args):
                                  cfg["q_dtype"], device=dev, keep_keys=False)
     cn = case_numpy(case)
     for i in range(args.warmup):
-        oracle_sample(cn, args.budget, k, [i % cfg["h_q"]])
-    secs = [oracle_sample(cn, args.budget, k, [(args.warmup + i) % cfg["h_q"]])
+        oracle_sample(cn, args.budget, k, [i % cfg["h_q"]], args.uniform)
+    secs = [oracle_sample(cn, args.budget, k, [(args.warmup + i) % cfg["h_q"]], args.uniform)
             for i in range(args.steps)]
     t = float(np.mean(secs))
     value = case.n / t / 1e9
@@ -334,7 +343,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, synthkv)",
-        "config": {"workload": workload_desc(cfg, args.budget, k), "budget_bits": args.budget,
+        "config": {"workload": workload_desc(cfg, args.budget, k, args.uniform),
+                   "budget_bits": args.budget,
                    "k": k, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
@@ -419,6 +429,12 @@ def run_native(args):
     n_total = sum(c.n for c in cases)
     n_max_cfg = max(c.n for c in cases)
 
+    def allocate(q_src):
+        if args.uniform:
+            F.allocate_uniform(S * h_q, d, B, out=alloc_all)
+        else:
+            F.allocate(q_src, sigma_all, B, out=alloc_all)
+
     def make_step(q_src):
         if ragged:
             descs = [dict(planes=planes[i], qmin=cases[i].qmin, qscale=cases[i].qscale,
@@ -429,13 +445,13 @@ def run_native(args):
                                  device=device)
 
             def step():
-                F.allocate(q_src, sigma_all, B, out=alloc_all)
+                allocate(q_src)
                 scan(ws)
         else:
             c = cases[0]
 
             def step():
-                F.allocate(q_src, sigma_all, B, out=alloc_all)
+                allocate(q_src)
                 F.scan_topk(planes[0], c.qmin, c.qscale, q_src, alloc_all, k, c.n,
                             host_mapped=host, flags=flags, workspace=ws, out=outs[0])
         return step
@@ -539,7 +555,7 @@ def run_native(args):
                                     device=device, keep_keys=False).codes
         cn = case_numpy(c)
         heads = list(range(8))
-        secs = oracle_sample(cn, B, k, heads)
+        secs = oracle_sample(cn, B, k, heads, args.uniform)
         cpu = {"value": len(heads) * c.n / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "query heads 0-7 (KV heads 0-1) of this step: allocation, fp64 scores "
                          "of all %d keys, brute-force top-%d; single thread, %.1f s" % (c.n, k, secs)}
@@ -547,7 +563,8 @@ def run_native(args):
     if rank == 0:
         traffic = None
         if not ragged and not host:
-            traffic = profiled_traffic(cfg["name"], "bit_plane_kv_scan_b200/csrc/scan.cu"
+            traffic = profiled_traffic(cfg["name"] + ("_uniform" if args.uniform else ""),
+                                       "bit_plane_kv_scan_b200/csrc/scan.cu"
                                        if flags else "bit_plane_kv_scan_b200/csrc/scan_tc.cu")
         res = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -555,9 +572,10 @@ def run_native(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded, synthkv: Qwen3-8B-shaped GQA keys with outlier "
                     "channels, 4-bit min-max codes)",
-            "config": {"workload": workload_desc(cfg, B, k), "sessions_per_rank": S,
+            "config": {"workload": workload_desc(cfg, B, k, args.uniform), "sessions_per_rank": S,
                        "keys_per_rank": n_total, "h_kv": h_kv, "h_q": h_q, "d": d,
                        "budget_bits": B, "k": k, "scan_kernel": "cuda-core" if flags else "tcgen05",
+                       "allocation": "uniform" if args.uniform else "water-filling",
                        "l2": "flushed between steps (256 MiB write, outside the events)"},
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,

@@ -110,4 +110,27 @@ cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h
                           G, d, budget, alloc);
 }
 
+// Query-independent read of `budget` bits per key: every channel takes
+// budget / d planes and channels c < budget % d one more.  This is the
+// water-filling rule above with every channel equally important (its slot
+// order takes all channels' first slots, lower channels first, then all
+// second slots, ...), so every query head reads the same prefixes and a GQA
+// group's union is one head's read.  One thread per (head, channel).
+__global__ void __launch_bounds__(256) allocate_uniform_kernel(int n_entries, int d, int budget,
+                                                               uint8_t *__restrict__ alloc) {
+  grid_dependency_wait();
+  allow_dependent_launch();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_entries) return;
+  const int c = i % d;
+  alloc[i] = (uint8_t)(budget / d + (c < budget % d ? 1 : 0));
+}
+
+cudaError_t launch_allocate_uniform(int h_q, int d, int budget, uint8_t *alloc,
+                                    cudaStream_t stream) {
+  const int n_entries = h_q * d;
+  return launch_dependent(allocate_uniform_kernel, dim3((n_entries + 255) / 256), dim3(256), 0,
+                          stream, n_entries, d, budget, alloc);
+}
+
 }  // namespace fathom

@@ -11,6 +11,8 @@
 namespace fathom {
 cudaError_t launch_pack(const uint8_t *codes, int64_t n, int d, int h_kv, uint32_t *planes,
                         cudaStream_t stream);
+cudaError_t launch_allocate_uniform(int h_q, int d, int budget, uint8_t *alloc,
+                                    cudaStream_t stream);
 cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
                             int budget, uint8_t *alloc, cudaStream_t stream);
 cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream);
@@ -199,6 +201,19 @@ fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, const float *
   cudaError_t e = launch_allocate(q, q_dtype == FATHOM_BF16, sigma, h_q, h_kv, d, budget_bits,
                                   alloc, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "allocate launch");
+  return ok();
+}
+
+fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits, uint8_t *alloc,
+                                      void *stream) {
+  fathom_status st = check_shape(d, h_q, 1);
+  if (st != FATHOM_OK) return st;
+  REQUIRE((int64_t)h_q * d < ((int64_t)1 << 30), "h_q=%d too large", h_q);
+  REQUIRE(budget_bits >= 0 && budget_bits <= 4 * d, "budget_bits=%d out of range [0, 4d=%d]",
+          budget_bits, 4 * d);
+  REQUIRE_DEV(alloc, "alloc");
+  cudaError_t e = launch_allocate_uniform(h_q, d, budget_bits, alloc, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "allocate_uniform launch");
   return ok();
 }
 

@@ -35,7 +35,8 @@ FLAG_CUDA_CORES = 4
 
 EXPORTED = [
     "fathom_last_error", "fathom_plane_words", "fathom_planes_bytes", "fathom_pack_planes",
-    "fathom_allocate", "fathom_scan_topk_workspace_size", "fathom_scan_topk",
+    "fathom_allocate", "fathom_allocate_uniform", "fathom_scan_topk_workspace_size",
+    "fathom_scan_topk",
     "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
     "fathom_scan_read_report", "fathom_profile_scan_kernel", "fathom_scan_topk_noalloc",
 ]
@@ -105,6 +106,8 @@ def lib() -> ctypes.CDLL:
         L.fathom_pack_planes.argtypes = [vp, i64, ci, ci, vp, vp]
         L.fathom_allocate.restype = ci
         L.fathom_allocate.argtypes = [vp, ci, vp, ci, ci, ci, ci, vp, vp]
+        L.fathom_allocate_uniform.restype = ci
+        L.fathom_allocate_uniform.argtypes = [ci, ci, ci, vp, vp]
         L.fathom_scan_topk_workspace_size.restype = sz
         L.fathom_scan_topk_workspace_size.argtypes = [ctypes.POINTER(ScanArgs)]
         L.fathom_scan_topk.restype = ci
@@ -170,6 +173,16 @@ def allocate(q: torch.Tensor, sigma: torch.Tensor, budget: int, stream=None,
         out = torch.empty((h_q, d), dtype=torch.uint8, device=q.device)
     _check(lib().fathom_allocate(_ptr(q.contiguous()), _dtype_code(q), _ptr(sigma.contiguous()),
                                  h_q, h_kv, d, int(budget), _ptr(out), _stream(stream)))
+    return out
+
+
+def allocate_uniform(h_q: int, d: int, budget: int, device=None, stream=None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The query-independent allocation of `budget` bits: uint8 [h_q, d] on `device`."""
+    if out is None:
+        out = torch.empty((h_q, d), dtype=torch.uint8, device=torch.device(device or "cuda"))
+    _check(lib().fathom_allocate_uniform(int(h_q), int(d), int(budget), _ptr(out),
+                                         _stream(stream)))
     return out
 
 

@@ -14,6 +14,9 @@
  *   fathom_pack_planes   4-bit codes -> bit planes (once per cache, off the
  *                        per-step path);
  *   fathom_allocate      per query head, bits per channel (the allocation);
+ *   fathom_allocate_uniform   the same B bits per key for every query head,
+ *                        spread evenly over the channels (the fixed-depth
+ *                        read that the adaptive allocation is compared with);
  *   fathom_scan_topk     scores of all n keys from the allocated prefixes and
  *                        the per-head top-k (one session);
  *   fathom_scan_topk_batched   the same for many sessions in one launch set.
@@ -130,6 +133,22 @@ FATHOM_API fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int
  */
 FATHOM_API fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, const float *sigma, int h_q,
                               int h_kv, int d, int budget_bits, uint8_t *alloc, void *stream);
+
+/* fathom_allocate_uniform -- a query-independent allocation of the same
+ * budget: the fixed-depth read that the pages' measurements set the
+ * adaptive read against (findings: "1.67x faster GPU time than 136-bit
+ * scans"; abstract: "at equal bytes").
+ *   alloc   [h_q][d] uint8 out: t_c = budget_bits / d for every channel,
+ *           plus one for channels c < budget_bits % d; the same row for
+ *           every head, so sum_c t_c = budget_bits.
+ * This is fathom_allocate's rule with every channel equally important (its
+ * tie-break takes lower channels first), so a GQA group's union prefix is
+ * one head's read.  The result feeds fathom_scan_topk unchanged.
+ * Requires d a multiple of 32 in [32, 256], h_q >= 1 and
+ * 0 <= budget_bits <= 4d.
+ */
+FATHOM_API fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits, uint8_t *alloc,
+                                      void *stream);
 
 /* fathom_scan_topk -- score all n keys of one session from the allocated
  * plane prefixes and return each query head's top-k (method paragraph 1:

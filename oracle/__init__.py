@@ -128,6 +128,17 @@ def allocate_heads(q, sigma, budget: int) -> np.ndarray:
     return np.stack([allocate(q[h], sigma[h // G], budget) for h in range(q.shape[0])])
 
 
+def allocate_uniform(h_q: int, d: int, budget: int) -> np.ndarray:
+    """The query-independent read of `budget` bits per key (the fixed-depth
+    read the pages compare the adaptive one with): every channel takes
+    budget // d planes and the first budget % d channels one more; the same
+    row for every head.  uint8 [h_q, d]."""
+    base, extra = divmod(int(budget), int(d))
+    row = np.full(int(d), base, dtype=np.uint8)
+    row[:extra] += 1
+    return np.tile(row, (int(h_q), 1))
+
+
 def dequant_prefix(m: float, s: float, t: int, v: int) -> float:
     return float(_load().oracle_dequant_prefix(float(m), float(s), int(t), int(v)))
 

@@ -88,6 +88,15 @@ def _args(**kw):
     return F.ScanArgs(**a)
 
 
+def test_allocate_uniform_rejects_bad_arguments(L):
+    assert L.fathom_allocate_uniform(32, 100, 92, None, None) == F.ERR_UNSUPPORTED
+    assert L.fathom_allocate_uniform(0, 128, 92, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate_uniform(32, 128, 513, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate_uniform(32, 128, -1, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_allocate_uniform(32, 128, 136, None, None) == F.ERR_INVALID_ARGUMENT
+    assert b"alloc" in L.fathom_last_error()
+
+
 def test_scan_workspace_size_and_limits(L):
     ws = L.fathom_scan_topk_workspace_size(ctypes.byref(_args()))
     assert ws > 0 and ws % 256 == 0

@@ -42,7 +42,7 @@ def _planes_np(planes):
     return _np(planes).view(np.uint32)
 
 
-def run_gpu(case, budget, k, flags=0, debug=False, host_mapped=False):
+def run_gpu(case, budget, k, flags=0, debug=False, host_mapped=False, uniform=False):
     dev = torch.device("cuda")
     codes = case.codes.to(dev)
     planes = F.pack_planes(codes)
@@ -54,7 +54,10 @@ def run_gpu(case, budget, k, flags=0, debug=False, host_mapped=False):
         planes_used = planes
     q = case.q_storage().to(dev)
     sigma = case.sigma.to(dev)
-    alloc = F.allocate(q, sigma, budget)
+    if uniform:
+        alloc = F.allocate_uniform(case.h_q, case.d, budget, device=dev)
+    else:
+        alloc = F.allocate(q, sigma, budget)
     out = F.scan_topk(planes_used, case.qmin.to(dev), case.qscale.to(dev), q, alloc, k, case.n,
                       debug_scores=debug, flags=flags, host_mapped=host_mapped)
     torch.cuda.synchronize()
@@ -136,10 +139,17 @@ def test_allocate_bit_exact(name, q, sigma, dtype):
 
 # ------------------------------------------------------------ small scans --
 
-def _full_check(case, budget, k, flags=0, what=""):
-    planes, alloc, (idx, sc, dbg) = run_gpu(case, budget, k, flags=flags, debug=True)
+def _want_alloc(case, cn, budget, uniform):
+    if uniform:
+        return oracle.allocate_uniform(case.h_q, case.d, budget)
+    return oracle.allocate_heads(cn[3], _np(case.sigma), budget)
+
+
+def _full_check(case, budget, k, flags=0, what="", uniform=False):
+    planes, alloc, (idx, sc, dbg) = run_gpu(case, budget, k, flags=flags, debug=True,
+                                            uniform=uniform)
     cn = case_np(case)
-    want_alloc = oracle.allocate_heads(cn[3], _np(case.sigma), budget)
+    want_alloc = _want_alloc(case, cn, budget, uniform)
     np.testing.assert_array_equal(_np(alloc), want_alloc)
     np.testing.assert_array_equal(_planes_np(planes), oracle.pack_planes(cn[0]))
     G = case.group
@@ -150,6 +160,24 @@ def _full_check(case, budget, k, flags=0, what=""):
         scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
         check_dense(dbg[h], ref, scale, "%s head %d" % (what, h))
         check_topk(idx[h], sc[h], ref, k, scale, "%s head %d" % (what, h))
+
+
+@pytest.mark.parametrize("h_q,d,B", [(1, 32, 0), (4, 64, 100), (32, 128, 92), (32, 128, 136),
+                                     (3, 96, 200), (7, 256, 1024)])
+def test_allocate_uniform_bit_exact(h_q, d, B):
+    got = F.allocate_uniform(h_q, d, B)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(_np(got), oracle.allocate_uniform(h_q, d, B))
+
+
+@pytest.mark.parametrize("B", [68, 136])
+@pytest.mark.parametrize("cuda_cores", [False, True])
+def test_uniform_read_scan(B, cuda_cores):
+    """The scan over a query-independent allocation, dense scores and top-k
+    against the oracle (both scan kernels)."""
+    case = synthkv.make_case(seed=11 + B, n=20000, h_kv=2, h_q=8, d=128, q_dtype="bf16")
+    _full_check(case, B, 64, flags=F.FLAG_CUDA_CORES if cuda_cores else 0,
+                what="uniform B=%d cc=%d" % (B, cuda_cores), uniform=True)
 
 
 def test_tiny_4k_config():
@@ -273,10 +301,11 @@ def test_cuda_core_scan_layer_131k(layer_131k):
 
 # ------------------------------------------------------ full-size configs --
 
-def _check_config(case, budget, k, heads_full, what, host_mapped=False, flags=0):
-    _, alloc, (idx, sc) = run_gpu(case, budget, k, host_mapped=host_mapped, flags=flags)
+def _check_config(case, budget, k, heads_full, what, host_mapped=False, flags=0, uniform=False):
+    _, alloc, (idx, sc) = run_gpu(case, budget, k, host_mapped=host_mapped, flags=flags,
+                                  uniform=uniform)
     cn = case_np(case)
-    want_alloc = oracle.allocate_heads(cn[3], _np(case.sigma), budget)
+    want_alloc = _want_alloc(case, cn, budget, uniform)
     got_alloc = _np(alloc)
     np.testing.assert_array_equal(got_alloc, want_alloc)
     idx, sc = _np(idx), _np(sc)
@@ -320,6 +349,15 @@ def test_decode_1m(decode_1m, B):
                   what="1M B=%d" % B)
     rep = F.read_report()
     assert rep.fallback_heads == 0
+
+
+def test_decode_1m_uniform_136(decode_1m):
+    """The fixed-depth comparison read: 136 bits per key, the same for every
+    query head, on the 1M-token step."""
+    _check_config(decode_1m, 136, 2048, heads_full={0, 31}, what="1M uniform 136", uniform=True)
+    rep = F.read_report()
+    assert rep.fallback_heads == 0
+    assert rep.union_planes == 8 * 136  # a GQA group's union is one head's read
 
 
 def test_decode_1m_cuda_cores(decode_1m):

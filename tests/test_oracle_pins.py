@@ -226,6 +226,25 @@ def test_allocation_matches_closed_form_water_filling(B):
 
 # ------------------------------------------------------------------ scores --
 
+@pytest.mark.parametrize("d", [8, 32, 128])
+def test_uniform_allocation_is_water_filling_with_equal_importance(d):
+    """The fixed-depth read: for every budget it equals the C oracle's
+    water-filling allocation when every channel has the same importance
+    (the slot order then takes every channel's first slot, lower channels
+    first, then every second slot, ...), sums to B and varies by at most one
+    plane between channels."""
+    ones = np.ones(d)
+    budgets = range(0, 4 * d + 1) if d <= 32 else [0, 1, 68, 92, 127, 128, 129, 136, 300, 511, 512]
+    for B in budgets:
+        t = oracle.allocate_uniform(3, d, B)
+        assert t.shape == (3, d) and t.dtype == np.uint8
+        assert (t == t[0]).all()
+        np.testing.assert_array_equal(t[0], oracle.allocate(ones, ones, B))
+        assert int(t[0].sum()) == B
+        assert int(t[0].max()) - int(t[0].min()) <= 1
+        assert t[0].max() <= 4
+
+
 def test_hand_example_scores_and_topk(golden):
     ex = golden["scan"]
     codes = np.array(ex["codes_bytes"], dtype=np.uint8).reshape(ex["n"], 1)
