@@ -67,6 +67,9 @@ def parse(argv=None):
     ap.add_argument("--uniform", action="store_true",
                     help="allocate the budget query-independently (the same depth in every "
                          "channel, fathom_allocate_uniform) instead of by water-filling")
+    ap.add_argument("--attention", action="store_true",
+                    help="also time the sparse attention over each head's top-k (the step after "
+                         "the scan; random bf16 K/V rows of the workload's shape), outside the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
@@ -546,6 +549,39 @@ def run_native(args):
     h2d = q_host.numel() * q_host.element_size()
     d2h = S * h_q * k * 8
 
+    attention = None
+    if args.attention and not ragged:
+        # the step after the scan, timed on its own: each head's attention over
+        # the top-k rows this step selected (random bf16 keys and values)
+        gen = torch.Generator(device=device).manual_seed(1234 + rank)
+        n1 = cases[0].n
+        k_rows = torch.randn((h_kv, n1, d), generator=gen, device=device).to(torch.bfloat16)
+        v_rows = torch.randn((h_kv, n1, d), generator=gen, device=device).to(torch.bfloat16)
+        idx = outs[0][0]
+        a_out = torch.empty((h_q, d), dtype=torch.float32, device=device)
+        a_lse = torch.empty((h_q,), dtype=torch.float32, device=device)
+        for _ in range(3):
+            F.sparse_attention(q_all, k_rows, v_rows, idx, out=a_out, lse=a_lse)
+        ab = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ae = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            ab[i].record(stream)
+            F.sparse_attention(q_all, k_rows, v_rows, idx, out=a_out, lse=a_lse)
+            ae[i].record(stream)
+        torch.cuda.synchronize()
+        a_ms = float(np.mean([x.elapsed_time(y) for x, y in zip(ab, ae)]))
+        rows = int(((idx >= 0) & (idx < n1)).sum().item())
+        a_bytes = rows * d * 2 * 2 + idx.numel() * 4 + q_all.numel() * q_all.element_size() + \
+            a_out.numel() * 4 + a_lse.numel() * 4
+        a_peak, a_kind = load_peaks()
+        a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
+        attention = {"kernel": "attention_kernel", "ms": a_ms, "rows": rows,
+                     "algorithmic_bytes": a_bytes, "achieved": a_gbs, "peak": a_peak,
+                     "unit": "GB/s", "frac": a_gbs / a_peak, "peak_kind": a_kind,
+                     "l2": "flushed before each launch"}
+        del k_rows, v_rows
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not ragged:
         import oracle
@@ -592,6 +628,8 @@ def run_native(args):
         }
         if cpu is not None:
             res["cpu_baseline"] = cpu
+        if attention is not None:
+            res["attention"] = attention
         print(json.dumps(res))
     if world > 1:
         import torch.distributed as dist

@@ -11,4 +11,5 @@ from .fathom import (  # noqa: F401
     PLANES_HOST_MAPPED, BatchedScan, FathomError, Workspace, allocate, allocate_uniform, lib,
     pack_planes,
     plane_words, profile_scan_kernel, read_report, scan_topk, scan_topk_batched,
+    sparse_attention,
 )

@@ -6,6 +6,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <cmath>
+
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -13,6 +15,10 @@ cudaError_t launch_pack(const uint8_t *codes, int64_t n, int d, int h_kv, uint32
                         cudaStream_t stream);
 cudaError_t launch_allocate_uniform(int h_q, int d, int budget, uint8_t *alloc,
                                     cudaStream_t stream);
+cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
+                             const uint16_t *v_rows, const int32_t *idx, int64_t n, int d,
+                             int h_q, int h_kv, int k, float scale, float *out, float *lse,
+                             cudaStream_t stream);
 cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
                             int budget, uint8_t *alloc, cudaStream_t stream);
 cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream);
@@ -214,6 +220,32 @@ fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits, uint8_t *
   REQUIRE_DEV(alloc, "alloc");
   cudaError_t e = launch_allocate_uniform(h_q, d, budget_bits, alloc, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "allocate_uniform launch");
+  return ok();
+}
+
+fathom_status fathom_sparse_attention(const fathom_attention_args *a, void *stream) {
+  REQUIRE(a != nullptr, "args is NULL");
+  fathom_status st = check_shape(a->d, a->h_q, a->h_kv);
+  if (st != FATHOM_OK) return st;
+  REQUIRE(a->q_dtype == FATHOM_F32 || a->q_dtype == FATHOM_BF16, "q_dtype=%d unknown",
+          (int)a->q_dtype);
+  REQUIRE(a->n >= 0 && a->n < ((int64_t)1 << 31), "n=%lld out of range [0, 2^31)",
+          (long long)a->n);
+  REQUIRE(a->k >= 0, "k=%d is negative", a->k);
+  REQUIRE(std::isfinite(a->softmax_scale), "softmax_scale is not finite");
+  REQUIRE_DEV(a->q, "q");
+  if (a->k > 0) REQUIRE_DEV(a->idx, "idx");
+  REQUIRE_DEV(a->out, "out");
+  if (a->lse) REQUIRE_DEV(a->lse, "lse");
+  if (a->n > 0 && a->k > 0) {
+    REQUIRE_DEV(a->k_rows, "k_rows");
+    REQUIRE_DEV(a->v_rows, "v_rows");
+    REQUIRE(aligned(a->k_rows, 16) && aligned(a->v_rows, 16), "k_rows/v_rows not 16-byte aligned");
+  }
+  cudaError_t e = launch_attention(a->q, a->q_dtype == FATHOM_BF16, a->k_rows, a->v_rows, a->idx,
+                                   a->n, a->d, a->h_q, a->h_kv, a->k, a->softmax_scale, a->out,
+                                   a->lse, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();
 }
 

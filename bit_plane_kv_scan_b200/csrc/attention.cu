@@ -1,0 +1,192 @@
+// Sparse attention over the selected keys: the step after the scan ("Fathom
+// Makes KV-Cache Scans Query-Adaptive for Long-Context Decoding", method
+// paragraph 1: the scan identifies the top-k candidates, and only "the
+// relatively small set of KV rows that ultimately wins" is fetched).
+//
+// For query head h (KV head g = h / G) and its selected keys idx_r >= 0:
+//   s_r = scale <q_h, K[g][idx_r]>,  o_h = sum_r softmax(s)_r V[g][idx_r],
+//   lse_h = log sum_r exp(s_r).
+// A decode query is one vector per head, so this is a gather of k rows of K
+// and V followed by matrix-vector work: bound by the gathered bytes, not by
+// arithmetic, and kept on the CUDA cores.
+//
+// One block of 1024 threads per query head.  Warp w takes the selected rows
+// w * U .. w * U + U - 1, then the next 32 U, ...; each lane holds d / 32
+// consecutive dimensions of q, of the running output and of every row it
+// loads.  A warp first issues the loads of its U rows (U = 8, 4 or 2 as d
+// grows) (K and V, bf16), then
+// folds them into an online softmax in base 2 (q pre-scaled by scale *
+// log2 e).  The 32 warps' partial (max, sum, output) are merged through
+// shared memory.  Indices outside [0, n) are skipped, as are -1 entries.
+#include "fathom_internal.cuh"
+
+namespace fathom {
+
+constexpr int kAttnThreads = 1024;
+constexpr int kAttnWarps = kAttnThreads / 32;
+// rows a warp has in flight: as many as its registers hold (1024 threads
+// leave 64 registers a thread)
+__host__ __device__ constexpr int attn_rows(int dpl) { return dpl <= 2 ? 8 : dpl <= 4 ? 4 : 2; }
+
+struct AttnParams {
+  const void *q;
+  int q_bf16;
+  const uint16_t *k_rows;
+  const uint16_t *v_rows;
+  const int32_t *idx;
+  int64_t n;
+  int d, G, k;
+  float qscale;  // softmax scale * log2(e)
+  float *out;
+  float *lse;
+};
+
+__device__ __forceinline__ float bf16_float(uint16_t x) {
+  return __uint_as_float((uint32_t)x << 16);
+}
+
+// DPL consecutive bf16 values starting at p (p aligned to 2 DPL bytes when
+// DPL is a power of two, else to 4 bytes when DPL is even).
+template <int DPL>
+__device__ __forceinline__ void load_row_part(const uint16_t *p, uint32_t (&w)[(DPL + 1) / 2]) {
+  if (DPL == 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if (DPL == 4) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+    w[0] = v.x; w[1] = v.y;
+  } else if (DPL % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < DPL / 2; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t *>(p) + i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < (DPL + 1) / 2; ++i) {
+      const uint32_t lo = __ldg(p + 2 * i);
+      const uint32_t hi = 2 * i + 1 < DPL ? (uint32_t)__ldg(p + 2 * i + 1) : 0u;
+      w[i] = lo | (hi << 16);
+    }
+  }
+}
+
+__device__ __forceinline__ float part_value(const uint32_t *w, int i) {
+  return bf16_float((uint16_t)(w[i >> 1] >> (16 * (i & 1))));
+}
+
+template <int DPL>
+__global__ void __launch_bounds__(kAttnThreads) attention_kernel(AttnParams a) {
+  grid_dependency_wait();
+  allow_dependent_launch();
+  constexpr int D = 32 * DPL;
+  constexpr int NW = (DPL + 1) / 2;
+  constexpr int kAttnRows = attn_rows(DPL);
+  __shared__ float s_m[kAttnWarps], s_l[kAttnWarps];
+  __shared__ float s_o[kAttnWarps][D];
+  const int h = blockIdx.x;
+  const int g = h / a.G;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c0 = lane * DPL;
+
+  float qv[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const int64_t at = (int64_t)h * D + c0 + i;
+    const float x = a.q_bf16 ? bf16_float(reinterpret_cast<const uint16_t *>(a.q)[at])
+                             : reinterpret_cast<const float *>(a.q)[at];
+    qv[i] = x * a.qscale;
+  }
+  const int32_t *ix = a.idx + (int64_t)h * a.k;
+  const uint16_t *Kg = a.k_rows + (int64_t)g * a.n * D + c0;
+  const uint16_t *Vg = a.v_rows + (int64_t)g * a.n * D + c0;
+
+  float m = -INFINITY, l = 0.0f, o[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) o[i] = 0.0f;
+
+  for (int r0 = warp * kAttnRows; r0 < a.k; r0 += kAttnWarps * kAttnRows) {
+    int row[kAttnRows];  // n < 2^31
+    uint32_t kw[kAttnRows][NW], vw[kAttnRows][NW];
+#pragma unroll
+    for (int u = 0; u < kAttnRows; ++u) {
+      const int r = r0 + u;
+      const int32_t x = r < a.k ? __ldg(ix + r) : -1;
+      row[u] = (x >= 0 && (int64_t)x < a.n) ? x : -1;
+      if (row[u] >= 0) {
+        load_row_part<DPL>(Kg + (int64_t)row[u] * D, kw[u]);
+        load_row_part<DPL>(Vg + (int64_t)row[u] * D, vw[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAttnRows; ++u) {
+      if (row[u] < 0) continue;  // the same for every lane of the warp
+      float s = 0.0f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) s = fmaf(qv[i], part_value(kw[u], i), s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      const float mn = fmaxf(m, s);
+      const float corr = exp2f(m - mn);  // 0 for the first row (m = -inf)
+      const float p = exp2f(s - mn);
+      l = fmaf(l, corr, p);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) o[i] = fmaf(o[i], corr, p * part_value(vw[u], i));
+      m = mn;
+    }
+  }
+
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_l[warp] = l;
+  }
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) s_o[warp][c0 + i] = o[i];
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w]);
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float L = 0.0f, O = 0.0f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < kAttnWarps; ++w) {
+        if (s_m[w] == -INFINITY) continue;
+        const float f = exp2f(s_m[w] - M);
+        L = fmaf(s_l[w], f, L);
+        O = fmaf(s_o[w][c], f, O);
+      }
+    }
+    a.out[(int64_t)h * D + c] = L > 0.0f ? O / L : 0.0f;
+    if (c == 0 && a.lse) a.lse[h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  }
+}
+
+cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
+                             const uint16_t *v_rows, const int32_t *idx, int64_t n, int d,
+                             int h_q, int h_kv, int k, float scale, float *out, float *lse,
+                             cudaStream_t stream) {
+  AttnParams a;
+  a.q = q;
+  a.q_bf16 = q_bf16;
+  a.k_rows = k_rows;
+  a.v_rows = v_rows;
+  a.idx = idx;
+  a.n = n;
+  a.d = d;
+  a.G = h_q / h_kv;
+  a.k = k;
+  a.qscale = scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
+  const dim3 grid(h_q), block(kAttnThreads);
+  switch (d / 32) {
+    case 1: return launch_dependent(attention_kernel<1>, grid, block, 0, stream, a);
+    case 2: return launch_dependent(attention_kernel<2>, grid, block, 0, stream, a);
+    case 3: return launch_dependent(attention_kernel<3>, grid, block, 0, stream, a);
+    case 4: return launch_dependent(attention_kernel<4>, grid, block, 0, stream, a);
+    case 5: return launch_dependent(attention_kernel<5>, grid, block, 0, stream, a);
+    case 6: return launch_dependent(attention_kernel<6>, grid, block, 0, stream, a);
+    case 7: return launch_dependent(attention_kernel<7>, grid, block, 0, stream, a);
+    case 8: return launch_dependent(attention_kernel<8>, grid, block, 0, stream, a);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fathom

@@ -39,6 +39,7 @@ EXPORTED = [
     "fathom_scan_topk",
     "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
     "fathom_scan_read_report", "fathom_profile_scan_kernel", "fathom_scan_topk_noalloc",
+    "fathom_sparse_attention",
 ]
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -58,6 +59,17 @@ class ScanArgs(ctypes.Structure):
         ("d", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("k", ctypes.c_int),
         ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
         ("debug_scores", ctypes.c_void_p), ("flags", ctypes.c_uint32),
+    ]
+
+
+class AttentionArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("q_dtype", ctypes.c_int),
+        ("k_rows", ctypes.c_void_p), ("v_rows", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+        ("n", ctypes.c_int64),
+        ("d", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("k", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
     ]
 
 
@@ -108,6 +120,8 @@ def lib() -> ctypes.CDLL:
         L.fathom_allocate.argtypes = [vp, ci, vp, ci, ci, ci, ci, vp, vp]
         L.fathom_allocate_uniform.restype = ci
         L.fathom_allocate_uniform.argtypes = [ci, ci, ci, vp, vp]
+        L.fathom_sparse_attention.restype = ci
+        L.fathom_sparse_attention.argtypes = [ctypes.POINTER(AttentionArgs), vp]
         L.fathom_scan_topk_workspace_size.restype = sz
         L.fathom_scan_topk_workspace_size.argtypes = [ctypes.POINTER(ScanArgs)]
         L.fathom_scan_topk.restype = ci
@@ -184,6 +198,36 @@ def allocate_uniform(h_q: int, d: int, budget: int, device=None, stream=None,
     _check(lib().fathom_allocate_uniform(int(h_q), int(d), int(budget), _ptr(out),
                                          _stream(stream)))
     return out
+
+
+def sparse_attention(q: torch.Tensor, k_rows: torch.Tensor, v_rows: torch.Tensor,
+                     idx: torch.Tensor, softmax_scale: Optional[float] = None, stream=None,
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """Attention of each query head over its selected keys only.
+
+    q [h_q, d] (bf16/f32); k_rows, v_rows [h_kv, n, d] bf16; idx [h_q, k] int32
+    (entries outside [0, n) are skipped).  Returns (out [h_q, d] f32,
+    lse [h_q] f32)."""
+    h_q, d = q.shape
+    h_kv, n, dk = k_rows.shape
+    if k_rows.dtype != torch.bfloat16 or v_rows.dtype != torch.bfloat16:
+        raise TypeError("k_rows and v_rows must be bfloat16")
+    if v_rows.shape != k_rows.shape or dk != d:
+        raise ValueError("k_rows/v_rows must be [h_kv, n, d] with the query's d")
+    if idx.dtype != torch.int32 or idx.dim() != 2 or idx.shape[0] != h_q:
+        raise TypeError("idx must be an int32 [h_q, k] tensor")
+    if softmax_scale is None:
+        softmax_scale = 1.0 / float(d) ** 0.5
+    if out is None:
+        out = torch.empty((h_q, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((h_q,), dtype=torch.float32, device=q.device)
+    q, k_rows, v_rows, idx = q.contiguous(), k_rows.contiguous(), v_rows.contiguous(), idx.contiguous()
+    a = AttentionArgs(q=_ptr(q), q_dtype=_dtype_code(q), k_rows=_ptr(k_rows), v_rows=_ptr(v_rows),
+                      idx=_ptr(idx), n=n, d=d, h_q=h_q, h_kv=h_kv, k=idx.shape[1],
+                      softmax_scale=float(softmax_scale), out=_ptr(out), lse=_ptr(lse))
+    _check(lib().fathom_sparse_attention(ctypes.byref(a), _stream(stream)))
+    return out, lse
 
 
 class Workspace:

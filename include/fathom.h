@@ -19,7 +19,9 @@
  *                        read that the adaptive allocation is compared with);
  *   fathom_scan_topk     scores of all n keys from the allocated prefixes and
  *                        the per-head top-k (one session);
- *   fathom_scan_topk_batched   the same for many sessions in one launch set.
+ *   fathom_scan_topk_batched   the same for many sessions in one launch set;
+ *   fathom_sparse_attention    after the scan: each query head's attention
+ *                        over only its selected keys.
  *
  * Conventions shared by every call
  *   - The caller owns every buffer.  The library never allocates or frees;
@@ -267,6 +269,39 @@ typedef struct fathom_scan_report {
 
 FATHOM_API fathom_status fathom_scan_read_report(const void *workspace, fathom_scan_report *report,
                                       void *stream);
+
+/* fathom_sparse_attention -- the step after the scan: each query head's
+ * attention over only the keys its top-k selected (method paragraph 1: the
+ * scan identifies the top-k candidates, and only "the relatively small set
+ * of KV rows that ultimately wins" is fetched).  For head h (KV head
+ * g = h / G) and its entries idx[h][r] in [0, n):
+ *   s_r = softmax_scale * <q[h], k_rows[g][idx[h][r]]>,
+ *   out[h] = sum_r softmax(s)_r v_rows[g][idx[h][r]],
+ *   lse[h] = log(sum_r exp(s_r))   (natural log).
+ * Entries outside [0, n) (the -1 padding of fathom_scan_topk) are skipped; a
+ * head with none gets out = 0 and lse = -inf.  fp32 arithmetic.
+ *   q        [h_q][d], FATHOM_BF16 or FATHOM_F32.
+ *   k_rows, v_rows   bf16 [h_kv][n][d]: the serving stack's keys and values
+ *            (16-byte aligned).
+ *   idx      int32 [h_q][k], e.g. fathom_scan_topk's out_idx.
+ *   out      float [h_q][d]; lse float [h_q] or NULL.
+ * Requires d as FATHOM_MAX_D, h_q a multiple of h_kv, k >= 0, 0 <= n < 2^31
+ * and a finite softmax_scale (1/sqrt(d) is the usual one).  No workspace.
+ */
+typedef struct fathom_attention_args {
+  const void *q;
+  fathom_dtype q_dtype;
+  const uint16_t *k_rows;
+  const uint16_t *v_rows;
+  const int32_t *idx;
+  int64_t n;
+  int d, h_q, h_kv, k;
+  float softmax_scale;
+  float *out;
+  float *lse;
+} fathom_attention_args;
+
+FATHOM_API fathom_status fathom_sparse_attention(const fathom_attention_args *args, void *stream);
 
 #ifdef __cplusplus
 }

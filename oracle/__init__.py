@@ -205,3 +205,34 @@ def scan_step(codes, qmin, qscale, q, sigma, budget: int, k: int, heads=None):
         res["score"][h] = v
         res["scores"][h] = s
     return res
+
+
+def sparse_attention(q, k_rows, v_rows, idx, scale: float):
+    """Attention of each query head over its selected keys only (the step
+    after the scan: "fetching the relatively small set of KV rows that
+    ultimately wins", method paragraph 1), by its definition in fp64:
+        s_r = scale * <q_h, K[g][idx_r]>,  w = softmax(s),  o_h = sum_r w_r V[g][idx_r],
+        lse_h = log sum_r exp(s_r),
+    over the entries idx_r >= 0 of head h's row (head h reads KV head h // G).
+    q [h_q, d]; k_rows, v_rows [h_kv, n, d]; idx [h_q, k] int.
+    Returns (o float64 [h_q, d], lse float64 [h_q]); a head with no selected
+    key gets o = 0 and lse = -inf."""
+    q = np.asarray(q, dtype=np.float64)
+    k_rows = np.asarray(k_rows, dtype=np.float64)
+    v_rows = np.asarray(v_rows, dtype=np.float64)
+    idx = np.asarray(idx)
+    h_q, d = q.shape
+    G = h_q // k_rows.shape[0]
+    out = np.zeros((h_q, d))
+    lse = np.full(h_q, -np.inf)
+    for h in range(h_q):
+        sel = idx[h][idx[h] >= 0].astype(np.int64)
+        if sel.size == 0:
+            continue
+        g = h // G
+        s = (k_rows[g][sel] @ q[h]) * float(scale)
+        m = s.max()
+        w = np.exp(s - m)
+        out[h] = (w @ v_rows[g][sel]) / w.sum()
+        lse[h] = m + np.log(w.sum())
+    return out, lse

@@ -97,6 +97,23 @@ def test_allocate_uniform_rejects_bad_arguments(L):
     assert b"alloc" in L.fathom_last_error()
 
 
+def test_sparse_attention_rejects_bad_arguments(L):
+    def args(**kw):
+        a = dict(q=None, q_dtype=F.BF16, k_rows=None, v_rows=None, idx=None, n=1000, d=128,
+                 h_q=32, h_kv=8, k=64, softmax_scale=0.088, out=None, lse=None)
+        a.update(kw)
+        return ctypes.byref(F.AttentionArgs(**a))
+    assert L.fathom_sparse_attention(None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(d=100), None) == F.ERR_UNSUPPORTED
+    assert L.fathom_sparse_attention(args(h_q=30), None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(k=-1), None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(n=-5), None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(softmax_scale=float("inf")), None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(q_dtype=9), None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(), None) == F.ERR_INVALID_ARGUMENT
+    assert b"q" in L.fathom_last_error()
+
+
 def test_scan_workspace_size_and_limits(L):
     ws = L.fathom_scan_topk_workspace_size(ctypes.byref(_args()))
     assert ws > 0 and ws % 256 == 0

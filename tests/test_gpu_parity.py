@@ -424,3 +424,81 @@ def test_ragged_32_sessions_batched(cuda_cores):
             if i in (0, 13, 31) and h in (0, 9, 18, 27):
                 ref = oracle_head(cn, h, t_h)
                 check_topk(idx[h], sc[h], ref, k, scale, "session %d head %d" % (i, h))
+
+
+# ------------------------------------------------------ sparse attention --
+
+def _bf16_rows(shape, seed, dev):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+
+def _attention_ref(q, K, V, idx, scale, h_kv):
+    """The oracle on the gathered rows only (the full K/V need not fit on the host)."""
+    q = q.float().cpu().numpy().astype(np.float64)
+    idx = idx.cpu().numpy()
+    h_q, d = q.shape
+    n = K.shape[1]
+    G = h_q // h_kv
+    out = np.zeros((h_q, d))
+    lse = np.zeros(h_q)
+    for h in range(h_q):
+        keep = (idx[h] >= 0) & (idx[h] < n)
+        rows = torch.from_numpy(idx[h][keep].astype(np.int64)).to(K.device)
+        Ks = K[h // G].index_select(0, rows).float().cpu().numpy()[None]
+        Vs = V[h // G].index_select(0, rows).float().cpu().numpy()[None]
+        sub = np.arange(len(rows), dtype=np.int32)[None]
+        o, l = oracle.sparse_attention(q[h:h + 1], Ks, Vs, sub, scale)
+        out[h], lse[h] = o[0], l[0]
+    return out, lse
+
+
+def _check_attention(out, lse, ref_o, ref_l, V, what):
+    out, lse = _np(out).astype(np.float64), _np(lse).astype(np.float64)
+    vmax = max(1.0, float(V.float().abs().max()))
+    err = np.abs(out - ref_o).max()
+    assert err <= 2e-5 * vmax, "%s: |o - oracle| = %g" % (what, err)
+    fin = np.isfinite(ref_l)
+    assert (np.isneginf(lse) == ~fin).all(), what
+    lerr = np.abs(lse[fin] - ref_l[fin]) / np.maximum(1.0, np.abs(ref_l[fin]))
+    assert lerr.size == 0 or lerr.max() <= 2e-5, "%s: lse error %g" % (what, lerr.max())
+
+
+@pytest.mark.parametrize("n,h_kv,G,d,k,qd", [(5000, 2, 4, 128, 64, "bf16"), (3000, 1, 1, 32, 300, "f32"),
+                                            (2000, 2, 2, 256, 100, "bf16"), (700, 1, 4, 96, 1000, "bf16"),
+                                            (4000, 1, 2, 160, 257, "f32")])
+def test_sparse_attention_random_rows(n, h_kv, G, d, k, qd):
+    """Random selections with -1 padding, out-of-range entries and an empty head."""
+    dev = torch.device("cuda")
+    h_q = h_kv * G
+    rng = np.random.default_rng(n + d)
+    K = _bf16_rows((h_kv, n, d), n, dev)
+    V = _bf16_rows((h_kv, n, d), n + 1, dev)
+    q = torch.from_numpy(rng.normal(size=(h_q, d)).astype(np.float32))
+    q = (q.to(torch.bfloat16) if qd == "bf16" else q).to(dev)
+    idx = rng.integers(0, n, size=(h_q, k)).astype(np.int32)
+    idx[0, k // 2:] = -1
+    if h_q > 1:
+        idx[1, 0] = n + 7
+        idx[h_q - 1, :] = -1
+    idx = torch.from_numpy(idx).to(dev)
+    scale = 1.0 / np.sqrt(d)
+    out, lse = F.sparse_attention(q, K, V, idx, scale)
+    torch.cuda.synchronize()
+    ref_o, ref_l = _attention_ref(q, K, V, idx, scale, h_kv)
+    _check_attention(out, lse, ref_o, ref_l, V, "n=%d d=%d k=%d" % (n, d, k))
+
+
+def test_sparse_attention_after_the_scan(decode_1m):
+    """The step after the 1M-token scan: attention over each head's top-2048."""
+    dev = torch.device("cuda")
+    _, _, (idx, _) = run_gpu(decode_1m, 92, 2048)
+    n, d = decode_1m.n, decode_1m.d
+    K = _bf16_rows((decode_1m.h_kv, n, d), 21, dev)
+    V = _bf16_rows((decode_1m.h_kv, n, d), 22, dev)
+    q = decode_1m.q_storage().to(dev)
+    out, lse = F.sparse_attention(q, K, V, idx)
+    torch.cuda.synchronize()
+    ref_o, ref_l = _attention_ref(q, K, V, idx, 1.0 / np.sqrt(d), decode_1m.h_kv)
+    _check_attention(out, lse, ref_o, ref_l, V, "1M top-2048")
+    del K, V

@@ -245,6 +245,70 @@ def test_uniform_allocation_is_water_filling_with_equal_importance(d):
         assert t[0].max() <= 4
 
 
+def _attention_loops(q, k_rows, v_rows, idx, scale):
+    """Tiny-case brute force with scalar loops and math.exp (no max shift)."""
+    import math
+    h_q, d = len(q), len(q[0])
+    G = h_q // len(k_rows)
+    out, lse = [], []
+    for h in range(h_q):
+        rows = [int(i) for i in idx[h] if i >= 0]
+        if not rows:
+            out.append([0.0] * d)
+            lse.append(-math.inf)
+            continue
+        e = []
+        for i in rows:
+            dot = 0.0
+            for c in range(d):
+                dot += float(q[h][c]) * float(k_rows[h // G][i][c])
+            e.append(math.exp(dot * scale))
+        z = sum(e)
+        out.append([sum(e[j] * float(v_rows[h // G][rows[j]][c]) for j in range(len(rows))) / z
+                    for c in range(d)])
+        lse.append(math.log(z))
+    return np.array(out), np.array(lse)
+
+
+def test_sparse_attention_pins():
+    """The attention over the selected rows, against scalar-loop brute force,
+    closed forms (q = 0 averages the selected values and gives log of their
+    count; one selected row returns it), permutation invariance and the
+    skipped -1 entries."""
+    rng = np.random.default_rng(5)
+    h_q, h_kv, n, d, k = 4, 2, 40, 8, 6
+    q = rng.normal(size=(h_q, d))
+    K = rng.normal(size=(h_kv, n, d))
+    V = rng.normal(size=(h_kv, n, d))
+    idx = np.stack([rng.choice(n, size=k, replace=False) for _ in range(h_q)]).astype(np.int32)
+    idx[1, 4:] = -1
+    idx[3, :] = -1
+    scale = 0.3
+    o, lse = oracle.sparse_attention(q, K, V, idx, scale)
+    bo, blse = _attention_loops(q, K, V, idx, scale)
+    np.testing.assert_allclose(o, bo, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse[:3], blse[:3], rtol=1e-12)
+    assert np.isneginf(lse[3]) and (o[3] == 0).all()
+    # q = 0: uniform weights
+    o0, l0 = oracle.sparse_attention(np.zeros_like(q), K, V, idx, scale)
+    for h in range(3):
+        sel = idx[h][idx[h] >= 0]
+        np.testing.assert_allclose(o0[h], V[h // 2][sel].mean(axis=0), rtol=1e-12, atol=1e-14)
+        assert abs(l0[h] - np.log(len(sel))) < 1e-12
+    # one selected row
+    one = np.full((h_q, k), -1, dtype=np.int32)
+    one[:, 0] = 7
+    o1, l1 = oracle.sparse_attention(q, K, V, one, scale)
+    for h in range(h_q):
+        np.testing.assert_allclose(o1[h], V[h // 2][7], rtol=1e-12)
+        assert abs(l1[h] - scale * float(q[h] @ K[h // 2][7])) < 1e-12
+    # the order of the selected rows does not matter
+    perm = idx[:, ::-1].copy()
+    op, lp = oracle.sparse_attention(q, K, V, perm, scale)
+    np.testing.assert_allclose(op, o, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lp[:3], lse[:3], rtol=1e-12)
+
+
 def test_hand_example_scores_and_topk(golden):
     ex = golden["scan"]
     codes = np.array(ex["codes_bytes"], dtype=np.uint8).reshape(ex["n"], 1)
