@@ -10,23 +10,30 @@
 // and V followed by matrix-vector work: bound by the gathered bytes, not by
 // arithmetic, and kept on the CUDA cores.
 //
-// One block of 1024 threads per query head.  Warp w takes the selected rows
-// w * U .. w * U + U - 1, then the next 32 U, ...; each lane holds d / 32
+// A cluster of 8 CTAs of 256 threads per query head, so that the gather
+// runs on 8 SMs per head.  Warp w of the head's 64 takes the selected rows
+// w * U .. w * U + U - 1, then the next 64 U, ...; each lane holds d / 32
 // consecutive dimensions of q, of the running output and of every row it
-// loads.  A warp first issues the loads of its U rows (U = 8, 4 or 2 as d
-// grows) (K and V, bf16), then
-// folds them into an online softmax in base 2 (q pre-scaled by scale *
-// log2 e).  The 32 warps' partial (max, sum, output) are merged through
-// shared memory.  Indices outside [0, n) are skipped, as are -1 entries.
+// loads.  A warp first issues the loads (K and V, bf16) of its U rows (U = 8
+// up to d = 128, else 4), then folds them into an online softmax in base 2
+// (q pre-scaled by scale * log2 e).  Each CTA merges its 8 warps' partial
+// (max, sum, output) in shared memory; CTA 0 of the cluster merges the 8 CTA
+// partials through distributed shared memory and writes the result.
+// Indices outside [0, n) are skipped, as are -1 entries.
+#include <cooperative_groups.h>
+
 #include "fathom_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace fathom {
 
-constexpr int kAttnThreads = 1024;
-constexpr int kAttnWarps = kAttnThreads / 32;
-// rows a warp has in flight: as many as its registers hold (1024 threads
-// leave 64 registers a thread)
-__host__ __device__ constexpr int attn_rows(int dpl) { return dpl <= 2 ? 8 : dpl <= 4 ? 4 : 2; }
+constexpr int kAttnSplit = 8;  // CTAs per query head: one cluster
+constexpr int kAttnThreads = 256;
+constexpr int kAttnWarps = kAttnThreads / 32;            // per CTA
+constexpr int kAttnHeadWarps = kAttnSplit * kAttnWarps;  // per head
+// rows a warp has in flight
+__host__ __device__ constexpr int attn_rows(int dpl) { return dpl <= 4 ? 8 : 4; }
 
 struct AttnParams {
   const void *q;
@@ -73,7 +80,8 @@ __device__ __forceinline__ float part_value(const uint32_t *w, int i) {
 }
 
 template <int DPL>
-__global__ void __launch_bounds__(kAttnThreads) attention_kernel(AttnParams a) {
+__global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThreads)
+    attention_kernel(AttnParams a) {
   grid_dependency_wait();
   allow_dependent_launch();
   constexpr int D = 32 * DPL;
@@ -81,7 +89,11 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(AttnParams a) {
   constexpr int kAttnRows = attn_rows(DPL);
   __shared__ float s_m[kAttnWarps], s_l[kAttnWarps];
   __shared__ float s_o[kAttnWarps][D];
-  const int h = blockIdx.x;
+  __shared__ float s_pm, s_pl;  // this CTA's partial: max, sum
+  __shared__ float s_po[D];     // and output
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int h = blockIdx.x / kAttnSplit;
   const int g = h / a.G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c0 = lane * DPL;
@@ -102,7 +114,8 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(AttnParams a) {
 #pragma unroll
   for (int i = 0; i < DPL; ++i) o[i] = 0.0f;
 
-  for (int r0 = warp * kAttnRows; r0 < a.k; r0 += kAttnWarps * kAttnRows) {
+  for (int r0 = (rank * kAttnWarps + warp) * kAttnRows; r0 < a.k;
+       r0 += kAttnHeadWarps * kAttnRows) {
     int row[kAttnRows];  // n < 2^31
     uint32_t kw[kAttnRows][NW], vw[kAttnRows][NW];
 #pragma unroll
@@ -153,9 +166,31 @@ __global__ void __launch_bounds__(kAttnThreads) attention_kernel(AttnParams a) {
         O = fmaf(s_o[w][c], f, O);
       }
     }
-    a.out[(int64_t)h * D + c] = L > 0.0f ? O / L : 0.0f;
-    if (c == 0 && a.lse) a.lse[h] = L > 0.0f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+    s_po[c] = O;
+    if (c == 0) {
+      s_pm = M;
+      s_pl = L;
+    }
   }
+  cluster.sync();  // every CTA's partial is in its shared memory
+  if (rank == 0 && threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float MM = -INFINITY;
+    for (int r = 0; r < kAttnSplit; ++r) MM = fmaxf(MM, *cluster.map_shared_rank(&s_pm, r));
+    float L = 0.0f, O = 0.0f;
+    if (MM != -INFINITY) {
+      for (int r = 0; r < kAttnSplit; ++r) {
+        const float pm = *cluster.map_shared_rank(&s_pm, r);
+        if (pm == -INFINITY) continue;
+        const float f = exp2f(pm - MM);
+        L = fmaf(*cluster.map_shared_rank(&s_pl, r), f, L);
+        O = fmaf(*cluster.map_shared_rank(&s_po[c], r), f, O);
+      }
+    }
+    a.out[(int64_t)h * D + c] = L > 0.0f ? O / L : 0.0f;
+    if (c == 0 && a.lse) a.lse[h] = L > 0.0f ? (MM + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  }
+  cluster.sync();  // CTA 0 has read the others' shared memory
 }
 
 cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
@@ -175,7 +210,7 @@ cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
   a.qscale = scale * 1.4426950408889634f;
   a.out = out;
   a.lse = lse;
-  const dim3 grid(h_q), block(kAttnThreads);
+  const dim3 grid(h_q * kAttnSplit), block(kAttnThreads);
   switch (d / 32) {
     case 1: return launch_dependent(attention_kernel<1>, grid, block, 0, stream, a);
     case 2: return launch_dependent(attention_kernel<2>, grid, block, 0, stream, a);
