@@ -9,7 +9,7 @@ library raises.
 from .fathom import (  # noqa: F401
     BF16, F32, FLAG_FORCE_FALLBACK, FLAG_NO_SAMPLING, FLAG_CUDA_CORES, PLANES_DEVICE,
     PLANES_HOST_MAPPED, BatchedScan, FathomError, Workspace, allocate, allocate_uniform, lib,
-    pack_planes,
+    append_planes, pack_planes,
     plane_words, profile_scan_kernel, read_report, scan_topk, scan_topk_batched,
     sparse_attention,
 )

@@ -15,6 +15,8 @@ cudaError_t launch_pack(const uint8_t *codes, int64_t n, int d, int h_kv, uint32
                         cudaStream_t stream);
 cudaError_t launch_allocate_uniform(int h_q, int d, int budget, uint8_t *alloc,
                                     cudaStream_t stream);
+cudaError_t launch_append(const uint8_t *codes, int64_t n, int64_t m, int d, int h_kv,
+                          const uint32_t *planes_in, uint32_t *planes_out, cudaStream_t stream);
 cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
                              const uint16_t *v_rows, const int32_t *idx, int64_t n, int d,
                              int h_q, int h_kv, int k, float scale, float *out, float *lse,
@@ -191,6 +193,31 @@ fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int d, int h_k
   REQUIRE(aligned(codes, 16) && aligned(planes, 16), "codes and planes must be 16-byte aligned");
   cudaError_t e = launch_pack(codes, n, d, h_kv, planes, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return ok();
+}
+
+fathom_status fathom_append_planes(const uint8_t *codes, int64_t n, int64_t m, int d, int h_kv,
+                                   const uint32_t *planes_in, uint32_t *planes_out, void *stream) {
+  fathom_status st = check_shape(d, h_kv, h_kv);
+  if (st != FATHOM_OK) return st;
+  REQUIRE(n >= 0 && m >= 0 && n + m < ((int64_t)1 << 31), "n=%lld m=%lld out of range",
+          (long long)n, (long long)m);
+  REQUIRE_DEV(planes_out, "planes_out");
+  if (m > 0) REQUIRE_DEV(codes, "codes");
+  const bool same = planes_in == planes_out;
+  if (!same && plane_words(n) > 0) REQUIRE_DEV(planes_in, "planes_in");
+  REQUIRE(!same || plane_words(n) == plane_words(n + m),
+          "in place needs fathom_plane_words(n + m) == fathom_plane_words(n) (%lld != %lld)",
+          (long long)plane_words(n + m), (long long)plane_words(n));
+  if (!same) {
+    const int64_t bytes_in = (int64_t)h_kv * d * 4 * plane_words(n) * 4;
+    const int64_t bytes_out = (int64_t)h_kv * d * 4 * plane_words(n + m) * 4;
+    const uintptr_t a = (uintptr_t)planes_in, b = (uintptr_t)planes_out;
+    REQUIRE(a + (uintptr_t)bytes_in <= b || b + (uintptr_t)bytes_out <= a,
+            "planes_in and planes_out overlap");
+  }
+  cudaError_t e = launch_append(codes, n, m, d, h_kv, planes_in, planes_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
   return ok();
 }
 

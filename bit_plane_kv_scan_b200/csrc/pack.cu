@@ -111,6 +111,70 @@ static cudaError_t launch_pack_d(const uint8_t *codes, int64_t n, int h_kv, uint
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------- append --
+// Decoding grows the cache one token at a time.  Appending m tokens' codes
+// to a store of n tokens changes only the plane words that hold tokens
+// n .. n + m - 1; a longer row (plane_words(n + m) > plane_words(n)) needs
+// the old words copied into the new layout first.
+
+// Out-of-place step: word w < W_in of every row comes from the old store,
+// the rest of the new row is zero (padding, or about to receive new bits).
+__global__ void append_copy_kernel(const uint32_t *__restrict__ in, int64_t W_in,
+                                   uint32_t *__restrict__ out, int64_t W_out, int64_t rows) {
+  const int64_t total = rows * W_out;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / W_out, w = i - r * W_out;
+    out[i] = w < W_in ? in[r * W_in + w] : 0u;
+  }
+}
+
+// One thread per (KV head, channel, plane, word w) with w covering tokens
+// n .. n + m - 1: OR in bit 3 - j of the new tokens' codes of channel c
+// (the old store's bits past token n - 1 are zero).
+__global__ void append_bits_kernel(const uint8_t *__restrict__ codes, int64_t n, int64_t m, int d,
+                                   int h_kv, uint32_t *__restrict__ planes, int64_t W) {
+  const int64_t w0 = n / 32, w1 = (n + m + 31) / 32;  // words [w0, w1) hold new tokens
+  const int64_t nw = w1 - w0;
+  const int64_t total = (int64_t)h_kv * d * 4 * nw;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / nw;  // (g, c, j)
+    const int64_t w = w0 + (i - row * nw);
+    const int j = (int)(row & 3);
+    const int c = (int)((row >> 2) % d);
+    const int64_t g = (row >> 2) / d;
+    uint32_t word = 0u;
+    for (int b = 0; b < 32; ++b) {
+      const int64_t tok = 32 * w + b;
+      if (tok < n || tok >= n + m) continue;
+      const uint8_t byte = codes[(g * m + (tok - n)) * (d / 2) + c / 2];
+      const uint32_t u = (c & 1) ? (uint32_t)(byte >> 4) : (uint32_t)(byte & 15u);
+      word |= ((u >> (3 - j)) & 1u) << b;
+    }
+    planes[row * W + w] |= word;
+  }
+}
+
+cudaError_t launch_append(const uint8_t *codes, int64_t n, int64_t m, int d, int h_kv,
+                          const uint32_t *planes_in, uint32_t *planes_out, cudaStream_t stream) {
+  const int64_t W_in = plane_words(n), W_out = plane_words(n + m);
+  const int64_t rows = (int64_t)h_kv * d * 4;
+  if (planes_out != planes_in && rows * W_out > 0) {
+    const int64_t total = rows * W_out;
+    const int blocks = (int)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
+    append_copy_kernel<<<blocks, 256, 0, stream>>>(planes_in, W_in, planes_out, W_out, rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (m == 0) return cudaSuccess;
+  const int64_t nw = (n + m + 31) / 32 - n / 32;
+  const int64_t total = rows * nw;
+  const int blocks = (int)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
+  append_bits_kernel<<<blocks, 256, 0, stream>>>(codes, n, m, d, h_kv, planes_out, W_out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pack(const uint8_t *codes, int64_t n, int d, int h_kv, uint32_t *planes,
                         cudaStream_t stream) {
   if (n == 0) return cudaSuccess;

@@ -35,6 +35,7 @@ FLAG_CUDA_CORES = 4
 
 EXPORTED = [
     "fathom_last_error", "fathom_plane_words", "fathom_planes_bytes", "fathom_pack_planes",
+    "fathom_append_planes",
     "fathom_allocate", "fathom_allocate_uniform", "fathom_scan_topk_workspace_size",
     "fathom_scan_topk",
     "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
@@ -118,6 +119,8 @@ def lib() -> ctypes.CDLL:
         L.fathom_pack_planes.argtypes = [vp, i64, ci, ci, vp, vp]
         L.fathom_allocate.restype = ci
         L.fathom_allocate.argtypes = [vp, ci, vp, ci, ci, ci, ci, vp, vp]
+        L.fathom_append_planes.restype = ci
+        L.fathom_append_planes.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, ci, ci, vp, vp, vp]
         L.fathom_allocate_uniform.restype = ci
         L.fathom_allocate_uniform.argtypes = [ci, ci, ci, vp, vp]
         L.fathom_sparse_attention.restype = ci
@@ -176,6 +179,27 @@ def pack_planes(codes: torch.Tensor, stream=None) -> torch.Tensor:
     planes = torch.empty((h_kv, d, 4, plane_words(n)), dtype=torch.int32, device=codes.device)
     _check(lib().fathom_pack_planes(_ptr(codes), n, d, h_kv, _ptr(planes), _stream(stream)))
     return planes
+
+
+def append_planes(planes: torch.Tensor, n: int, codes_new: torch.Tensor, stream=None) -> torch.Tensor:
+    """Add m tokens' codes [h_kv, m, d/2] (uint8, CUDA) to a store of n tokens.
+
+    Returns the store of n + m tokens: `planes` itself, updated in place, when
+    the row length does not change, else a new tensor."""
+    if codes_new.dtype != torch.uint8 or codes_new.dim() != 3 or not codes_new.is_contiguous():
+        raise TypeError("codes_new must be a contiguous uint8 [h_kv, m, d/2] tensor")
+    h_kv, m, half = codes_new.shape
+    d = 2 * half
+    if tuple(planes.shape) != (h_kv, d, 4, plane_words(n)):
+        raise ValueError("planes must be [h_kv, d, 4, plane_words(n)]")
+    if plane_words(n + m) == plane_words(n):
+        out = planes
+    else:
+        out = torch.empty((h_kv, d, 4, plane_words(n + m)), dtype=torch.int32, device=planes.device)
+    _check(lib().fathom_append_planes(_ptr(codes_new) if m else None, int(n), int(m), d, h_kv,
+                                      _ptr(planes) if planes.numel() else None, _ptr(out),
+                                      _stream(stream)))
+    return out
 
 
 def allocate(q: torch.Tensor, sigma: torch.Tensor, budget: int, stream=None,

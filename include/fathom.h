@@ -12,7 +12,8 @@
  *
  * Four steps, three calls on the hot path:
  *   fathom_pack_planes   4-bit codes -> bit planes (once per cache, off the
- *                        per-step path);
+ *                        per-step path); fathom_append_planes adds decoded
+ *                        tokens to a packed store;
  *   fathom_allocate      per query head, bits per channel (the allocation);
  *   fathom_allocate_uniform   the same B bits per key for every query head,
  *                        spread evenly over the channels (the fixed-depth
@@ -115,6 +116,28 @@ FATHOM_API size_t fathom_planes_bytes(int64_t n, int d, int h_kv);
  */
 FATHOM_API fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int d, int h_kv,
                                  uint32_t *planes, void *stream);
+
+/* fathom_append_planes -- add m decoded tokens to a store of n tokens
+ * (decoding grows the cache a token at a time).
+ *   codes       [h_kv][m][d/2] uint8: the new tokens' 4-bit codes, laid out as
+ *               for fathom_pack_planes.  The codes come from the caller's
+ *               quantiser with the store's existing per-channel m_c, s_c,
+ *               clamped to 0..15: the scan's dequantisation stays that of
+ *               the store.  Requantising for a new min/max means packing
+ *               anew.
+ *   planes_in   [h_kv][d][4][fathom_plane_words(n)], the store of tokens
+ *               0 .. n - 1 (padding bits zero, as fathom_pack_planes leaves
+ *               them).
+ *   planes_out  [h_kv][d][4][fathom_plane_words(n + m)].  It may be planes_in
+ *               itself when the row length does not change
+ *               (fathom_plane_words(n + m) == fathom_plane_words(n)); then only
+ *               the words holding the new tokens are touched.  Otherwise it
+ *               must not overlap planes_in, which is copied into it first.
+ * The result equals fathom_pack_planes of all n + m tokens' codes.
+ */
+FATHOM_API fathom_status fathom_append_planes(const uint8_t *codes, int64_t n, int64_t m, int d,
+                                   int h_kv, const uint32_t *planes_in, uint32_t *planes_out,
+                                   void *stream);
 
 /* fathom_allocate -- per-query bit allocation by reverse water-filling
  * (method paragraph 3: "a reverse water-filling rule to assign more bits to

@@ -88,6 +88,14 @@ def _args(**kw):
     return F.ScanArgs(**a)
 
 
+def test_append_rejects_bad_arguments(L):
+    assert L.fathom_append_planes(None, 100, 1, 33, 1, None, None, None) == F.ERR_UNSUPPORTED
+    assert L.fathom_append_planes(None, -1, 1, 128, 1, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_append_planes(None, 100, -1, 128, 1, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_append_planes(None, 100, 1, 128, 1, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert b"planes_out" in L.fathom_last_error()
+
+
 def test_allocate_uniform_rejects_bad_arguments(L):
     assert L.fathom_allocate_uniform(32, 100, 92, None, None) == F.ERR_UNSUPPORTED
     assert L.fathom_allocate_uniform(0, 128, 92, None, None) == F.ERR_INVALID_ARGUMENT

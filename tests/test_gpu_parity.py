@@ -502,3 +502,37 @@ def test_sparse_attention_after_the_scan(decode_1m):
     ref_o, ref_l = _attention_ref(q, K, V, idx, 1.0 / np.sqrt(d), decode_1m.h_kv)
     _check_attention(out, lse, ref_o, ref_l, V, "1M top-2048")
     del K, V
+
+
+# ----------------------------------------------------------------- append --
+
+@pytest.mark.parametrize("n,m,d,h_kv", [(0, 1, 128, 1), (1, 1, 128, 2), (31, 1, 64, 1), (32, 1, 128, 1),
+                                        (127, 1, 128, 2), (128, 1, 128, 1), (1000, 37, 256, 1),
+                                        (4096, 200, 32, 3), (5000, 1, 96, 2), (777, 0, 128, 1)])
+def test_append_equals_packing_everything(n, m, d, h_kv):
+    """Appending m decoded tokens to a packed store of n gives the store of
+    all n + m tokens, bit for bit (in place while the row length holds)."""
+    rng = np.random.default_rng(n * 7 + m + d)
+    codes = rng.integers(0, 256, size=(h_kv, n + m, d // 2), dtype=np.uint8)
+    dev = torch.device("cuda")
+    old = torch.from_numpy(np.ascontiguousarray(codes[:, :n])).to(dev)
+    new = torch.from_numpy(np.ascontiguousarray(codes[:, n:])).to(dev)
+    planes = F.pack_planes(old) if n > 0 else torch.empty((h_kv, d, 4, 0), dtype=torch.int32,
+                                                           device=dev)
+    got = F.append_planes(planes, n, new)
+    torch.cuda.synchronize()
+    if F.plane_words(n + m) == F.plane_words(n) and n > 0:
+        assert got.data_ptr() == planes.data_ptr()
+    np.testing.assert_array_equal(_planes_np(got), oracle.pack_planes(codes))
+
+
+def test_append_token_by_token():
+    """A store grown one token at a time equals one packed at once."""
+    case = synthkv.make_case(seed=31, n=300, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+    dev = torch.device("cuda")
+    codes = case.codes.to(dev)
+    planes = F.pack_planes(codes[:, :250].contiguous())
+    for i in range(250, 300):
+        planes = F.append_planes(planes, i, codes[:, i:i + 1].contiguous())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(_planes_np(planes), oracle.pack_planes(_np(case.codes)))
