@@ -202,6 +202,7 @@ fathom_status fathom_append_planes(const uint8_t *codes, int64_t n, int64_t m, i
   if (st != FATHOM_OK) return st;
   REQUIRE(n >= 0 && m >= 0 && n + m < ((int64_t)1 << 31), "n=%lld m=%lld out of range",
           (long long)n, (long long)m);
+  if (n + m == 0) return ok();  // nothing stored, nothing to add
   REQUIRE_DEV(planes_out, "planes_out");
   if (m > 0) REQUIRE_DEV(codes, "codes");
   const bool same = planes_in == planes_out;

@@ -99,13 +99,10 @@ static cudaError_t launch_pack_d(const uint8_t *codes, int64_t n, int h_kv, uint
                                  cudaStream_t stream) {
   const int64_t W = plane_words(n);
   const int smem = D * 4 * 32 * 4;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(pack_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // per launch: the opt-in belongs to the current device
+  cudaError_t e = cudaFuncSetAttribute(pack_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem);
+  if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((W + 31) / 32), (unsigned)h_kv);
   pack_kernel<D><<<grid, D * 4, smem, stream>>>(codes, n, planes, W);
   return cudaGetLastError();

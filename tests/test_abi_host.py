@@ -94,6 +94,7 @@ def test_append_rejects_bad_arguments(L):
     assert L.fathom_append_planes(None, 100, -1, 128, 1, None, None, None) == F.ERR_INVALID_ARGUMENT
     assert L.fathom_append_planes(None, 100, 1, 128, 1, None, None, None) == F.ERR_INVALID_ARGUMENT
     assert b"planes_out" in L.fathom_last_error()
+    assert L.fathom_append_planes(None, 0, 0, 128, 1, None, None, None) == F.OK
 
 
 def test_allocate_uniform_rejects_bad_arguments(L):
