@@ -112,3 +112,23 @@ def test_reference_arm_line():
     assert out["e2e"] == {"value": out["value"], "unit": out["unit"], "h2d_bytes_per_step": 0,
                           "d2h_bytes_per_step": 0}
     assert out["config"]["workload"].startswith("tiny_4k")
+
+
+def test_reference_arm_uniform_allocation():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--config", "tiny_4k", "--uniform",
+                        "--budget", "136"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    out = json.loads([ln for ln in r.stdout.splitlines() if ln.strip()][-1])
+    assert "uniform allocation" in out["config"]["workload"]
+    assert out["config"]["budget_bits"] == 136
+
+
+def test_profile_traffic_needs_matching_workload():
+    src = "bit_plane_kv_scan_b200/csrc/scan_tc.cu"
+    assert bench.profiled_traffic("decode_1m_uniform", src) is None
+    assert bench.profiled_traffic("no_such_workload", src) is None
+    t = bench.profiled_traffic("decode_1m", src)
+    assert t is None or t > 155_000_000  # at least the algorithmic union bytes when current
