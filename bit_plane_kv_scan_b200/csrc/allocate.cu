@@ -1,8 +1,8 @@
 // Per-query bit allocation by reverse water-filling (method paragraph 3 of
 // "Fathom Makes KV-Cache Scans Query-Adaptive...": more bits go to the
-// channels that matter more for the current query, in closed form; abstract
-// of arXiv 2609.17652: "over the variance-weighted importance of its
-// channels").
+// channels that weigh most for the query at hand, in closed form; abstract
+// of arXiv 2609.17652: the weights are the channels' variance-weighted
+// importance).
 //
 // Closed form: b_c = clip(log2(w_c / theta) / 2, 0, 4), sum_c b_c = B, with
 // w_c = q_c^2 sigma_c^2.  Its exact integer form: each channel offers four

@@ -1,7 +1,7 @@
 // Sparse attention over the selected keys: the step after the scan ("Fathom
 // Makes KV-Cache Scans Query-Adaptive for Long-Context Decoding", method
-// paragraph 1: the scan identifies the top-k candidates, and only "the
-// relatively small set of KV rows that ultimately wins" is fetched).
+// paragraph 1: the scan finds the top-k candidates, and only the few KV rows
+// that win are then fetched).
 //
 // For query head h (KV head g = h / G) and its selected keys idx_r >= 0:
 //   s_r = scale <q_h, K[g][idx_r]>,  o_h = sum_r softmax(s)_r V[g][idx_r],

@@ -1,7 +1,7 @@
 // Bit-plane packer: 4-bit K codes (token-major nibbles) -> channel-major bit
 // planes ("Fathom Makes KV-Cache Scans Query-Adaptive...", method paragraph
-// 2: the 4-bit K cache "is stored in channel-major bit planes"; abstract:
-// "a prefix of t planes is exactly the channel's t-bit quantizer").
+// 2: the 4-bit K cache is kept as channel-major bit planes; abstract: a
+// channel's leading t planes are precisely its t-bit quantiser).
 //
 // One block turns 1024 tokens (32 plane words) of one KV head into every
 // plane row of those words.  Thread (token group tg, code word cw) loads the

@@ -5,7 +5,7 @@
  * KV Caches", arXiv 2609.17652; summarised in "Fathom Makes KV-Cache Scans
  * Query-Adaptive for Long-Context Decoding", cctest.ai) ranks all n cached
  * keys for each decode step's top-k.  Its 4-bit K cache is stored as
- * channel-major bit planes, so the first t planes of a channel are that
+ * channel-major bit planes, so a channel's first t planes are that
  * channel's t-bit quantiser; each query spends a budget of B bits per key
  * over its channels by reverse water-filling, and only the allocated plane
  * prefixes are read.
@@ -93,9 +93,9 @@ typedef enum fathom_planes_location {
 FATHOM_API const char *fathom_last_error(void);
 
 /* ---------------------------------------------------------------------------
- * Bit-plane store layout (method paragraph 2, "stored in channel-major bit
- * planes"; abstract, "a prefix of t planes is exactly the channel's t-bit
- * quantizer"):
+ * Bit-plane store layout (method paragraph 2: the K cache is kept as
+ * channel-major bit planes; abstract: a channel's first t planes are
+ * precisely its t-bit quantiser):
  *   planes[g][c][j][w], uint32, w < W = fathom_plane_words(n);
  *   bit b of word w of plane j holds bit (3 - j) of the code of token
  *   32 w + b; rows are padded to a multiple of 128 tokens (16 bytes) and
@@ -108,8 +108,8 @@ FATHOM_API size_t fathom_planes_bytes(int64_t n, int d, int h_kv);
 /* fathom_pack_planes -- build the bit-plane store from a 4-bit K cache.
  *   codes   [h_kv][n][d/2] uint8, token-major, two channels per byte, low
  *           nibble = even channel: the per-channel asymmetric 4-bit codes a
- *           quantised serving stack holds (abstract: "the store is the 4-bit
- *           K copy a quantized serving stack already holds").  Read only.
+ *           quantised serving stack holds (abstract: the store is the
+ *           4-bit copy of K that such a stack keeps anyway).  Read only.
  *   planes  [h_kv][d][4][fathom_plane_words(n)] uint32, written in full
  *           (padding zeroed).  16-byte aligned.
  * n >= 0 (n = 0 writes nothing), d as FATHOM_MAX_D, h_kv >= 1.
@@ -140,10 +140,9 @@ FATHOM_API fathom_status fathom_append_planes(const uint8_t *codes, int64_t n, i
                                    void *stream);
 
 /* fathom_allocate -- per-query bit allocation by reverse water-filling
- * (method paragraph 3: "a reverse water-filling rule to assign more bits to
- * channels that matter more for the current query... a closed-form
- * solution"; abstract: "over the variance-weighted importance of its
- * channels").
+ * (method paragraph 3: reverse water-filling gives more bits to the
+ * channels that weigh most for the query at hand, in closed form;
+ * abstract: the weights are the channels' variance-weighted importance).
  *   q       [h_q][d], FATHOM_BF16 or FATHOM_F32.
  *   sigma   [h_kv][d] float, the channel statistics sigma_c (head h uses row
  *           h / G).  Importance w_c = q_c^2 sigma_c^2 (fp64).
@@ -161,8 +160,8 @@ FATHOM_API fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, co
 
 /* fathom_allocate_uniform -- a query-independent allocation of the same
  * budget: the fixed-depth read that the pages' measurements set the
- * adaptive read against (findings: "1.67x faster GPU time than 136-bit
- * scans"; abstract: "at equal bytes").
+ * adaptive read against (findings: GPU time against scans that read 136
+ * bits per key; abstract: comparisons at the same number of bytes read).
  *   alloc   [h_q][d] uint8 out: t_c = budget_bits / d for every channel,
  *           plus one for channels c < budget_bits % d; the same row for
  *           every head, so sum_c t_c = budget_bits.
@@ -177,8 +176,8 @@ FATHOM_API fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits
 
 /* fathom_scan_topk -- score all n keys of one session from the allocated
  * plane prefixes and return each query head's top-k (method paragraph 1:
- * "scan a large number of keys to identify the top-k candidates"; abstract:
- * "the scan that ranks all n keys for a top-k step").
+ * sparse decoding finds its top-k candidates by scanning many keys;
+ * abstract: the scan ranks every one of the n keys for each top-k step).
  *
  * Score of key i for query head h (KV head g = h / G):
  *   s_h(i) = sum_c q_c * deq_{t_c}(v_{t_c}(i, c)),
@@ -216,7 +215,7 @@ FATHOM_API size_t fathom_scan_topk_workspace_size(const fathom_scan_args *args);
 FATHOM_API fathom_status fathom_scan_topk(const fathom_scan_args *args, void *workspace,
                                size_t workspace_bytes, void *stream);
 
-/* Batched ragged sessions ("many sessions resident at once", abstract): one
+/* Batched ragged sessions (abstract: many sessions are resident together): one
  * set of launches scores every session; sessions share d, h_q, h_kv, k and
  * the dtype and differ in n and buffers.  `sessions` is a DEVICE array of S
  * descriptors (pointers in it are not checked on the host). */
@@ -295,8 +294,8 @@ FATHOM_API fathom_status fathom_scan_read_report(const void *workspace, fathom_s
 
 /* fathom_sparse_attention -- the step after the scan: each query head's
  * attention over only the keys its top-k selected (method paragraph 1: the
- * scan identifies the top-k candidates, and only "the relatively small set
- * of KV rows that ultimately wins" is fetched).  For head h (KV head
+ * scan finds the top-k candidates, and only the few KV rows that win are
+ * then fetched).  For head h (KV head
  * g = h / G) and its entries idx[h][r] in [0, n):
  *   s_r = softmax_scale * <q[h], k_rows[g][idx[h][r]]>,
  *   out[h] = sum_r softmax(s)_r v_rows[g][idx[h][r]],

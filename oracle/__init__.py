@@ -209,8 +209,8 @@ def scan_step(codes, qmin, qscale, q, sigma, budget: int, k: int, heads=None):
 
 def sparse_attention(q, k_rows, v_rows, idx, scale: float):
     """Attention of each query head over its selected keys only (the step
-    after the scan: "fetching the relatively small set of KV rows that
-    ultimately wins", method paragraph 1), by its definition in fp64:
+    after the scan: only the few KV rows that win are fetched, method
+    paragraph 1), by its definition in fp64:
         s_r = scale * <q_h, K[g][idx_r]>,  w = softmax(s),  o_h = sum_r w_r V[g][idx_r],
         lse_h = log sum_r exp(s_r),
     over the entries idx_r >= 0 of head h's row (head h reads KV head h // G).

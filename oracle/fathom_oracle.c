@@ -25,7 +25,7 @@
  *     slots of channel c.  This is the exact integer optimum of
  *     sum_c w_c 4^-t_c subject to sum_c t_c = B, 0 <= t_c <= 4, whose
  *     continuous relaxation is the closed form b_c = clip(log2(w_c/theta)/2,
- *     0, 4) ("reverse water-filling", abstract);
+ *     0, 4) (the abstract's reverse water-filling);
  *   - scores are the raw dot product (no 1/sqrt(d)); top-k is ordered by
  *     score descending, then index ascending; k > n pads with index -1.
  *
@@ -45,8 +45,8 @@ static unsigned code_at(const uint8_t *codes_g, int d, int64_t i, int c) {
   return (c & 1) ? (unsigned)(byte >> 4) : (unsigned)(byte & 15u);
 }
 
-/* Channel-major bit planes (method paragraph 2: "The underlying 4-bit K cache
- * is stored in channel-major bit planes").  codes: [h_kv][n][d/2] nibbles,
+/* Channel-major bit planes (method paragraph 2: the 4-bit K cache is kept as
+ * bit planes, channel by channel).  codes: [h_kv][n][d/2] nibbles,
  * planes: [h_kv][d][4][W]. */
 void oracle_pack_planes(const uint8_t *codes, int64_t n, int d, int h_kv, uint32_t *planes) {
   int64_t W = oracle_plane_words(n);
@@ -99,8 +99,8 @@ static int slot_order(const void *pa, const void *pb) {
   return 0;
 }
 
-/* Importance w_c = q_c^2 * sigma_c^2 ("variance-weighted importance of its
- * channels", abstract), one rounding after two exact squares. */
+/* Importance w_c = q_c^2 * sigma_c^2 (abstract: the channels' importance
+ * weighted by their variance), one rounding after two exact squares. */
 double oracle_importance(double q, double sigma) { return (q * q) * (sigma * sigma); }
 
 /* One query head: t[c] in 0..4 with sum t = budget (0 <= budget <= 4d). */
@@ -123,8 +123,8 @@ void oracle_allocate(const double *q, const double *sigma, int d, int budget, ui
 /* ---- scores -------------------------------------------------------------- */
 
 /* Cell-centre reconstruction of a t-bit prefix value v of a channel with
- * offset m and step s (method paragraph 2: "Reading the first t planes of a
- * channel is equivalent to using that channel's t-bit quantized value"). */
+ * offset m and step s (method paragraph 2: a channel's first t planes
+ * give that channel's t-bit quantised value). */
 double oracle_dequant_prefix(double m, double s, int t, unsigned v) {
   double cell = ldexp(1.0, 4 - t); /* 2^(4-t) */
   return m + s * (cell * (double)v + (cell - 1.0) / 2.0);
@@ -199,7 +199,7 @@ static int scored_order(const void *pa, const void *pb) {
 }
 
 /* Brute force: sort all n by (score desc, index asc), keep the first k
- * ("the scan that ranks all n keys for a top-k step", abstract). */
+ * (abstract: the scan ranks every one of the n keys for the top-k step). */
 void oracle_topk(const double *scores, int64_t n, int k, int32_t *idx, double *val) {
   scored_t *all = (scored_t *)malloc(sizeof(scored_t) * (size_t)(n > 0 ? n : 1));
   for (int64_t i = 0; i < n; ++i) {
