@@ -10,17 +10,18 @@
  * over its channels by reverse water-filling, and only the allocated plane
  * prefixes are read.
  *
- * Four steps, three calls on the hot path:
+ * The hot path is four steps in three calls:
  *   fathom_pack_planes   4-bit codes -> bit planes (once per cache, off the
- *                        per-step path); fathom_append_planes adds decoded
- *                        tokens to a packed store;
+ *                        per-step path);
  *   fathom_allocate      per query head, bits per channel (the allocation);
- *   fathom_allocate_uniform   the same B bits per key for every query head,
- *                        spread evenly over the channels (the fixed-depth
- *                        read that the adaptive allocation is compared with);
  *   fathom_scan_topk     scores of all n keys from the allocated prefixes and
  *                        the per-head top-k (one session);
- *   fathom_scan_topk_batched   the same for many sessions in one launch set;
+ *   fathom_scan_topk_batched   the same for many sessions in one launch set.
+ * Around it:
+ *   fathom_append_planes       adds decoded tokens to a packed store;
+ *   fathom_allocate_uniform    the same B bits per key for every query head,
+ *                        spread evenly over the channels (the fixed-depth
+ *                        read that the adaptive allocation is compared with);
  *   fathom_sparse_attention    after the scan: each query head's attention
  *                        over only its selected keys.
  *
