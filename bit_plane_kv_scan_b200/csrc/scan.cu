@@ -35,6 +35,8 @@
 //    streaming single-block scan.
 #include <float.h>
 
+#include <atomic>
+
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -1192,17 +1194,27 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
 
 // ------------------------------------------------------------- launchers --
 
-static int g_num_sms = 0;
+// SM count of the current device, cached per device (a process may drive
+// several).  Concurrent first calls may both query it and store the same
+// value.
+static std::atomic<int> g_num_sms[64];
 
 static cudaError_t num_sms(int *out) {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) {
+    const int cached = g_num_sms[dev].load(std::memory_order_relaxed);
+    if (cached > 0) {
+      *out = cached;
+      return cudaSuccess;
+    }
   }
-  *out = g_num_sms;
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) g_num_sms[dev].store(sms, std::memory_order_relaxed);
+  *out = sms;
   return cudaSuccess;
 }
 
