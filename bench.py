@@ -552,35 +552,62 @@ def run_native(args):
     attention = None
     if args.attention and not ragged:
         # the step after the scan, timed on its own: each head's attention over
-        # the top-k rows this step selected (random bf16 keys and values)
+        # the top-k rows this step selected, with random bf16 values and keys
+        # either as bf16 rows or as 4-bit codes (dequantised in the gather),
+        # in device memory or in pinned host memory (only the selected rows
+        # cross the host link)
         gen = torch.Generator(device=device).manual_seed(1234 + rank)
         n1 = cases[0].n
-        k_rows = torch.randn((h_kv, n1, d), generator=gen, device=device).to(torch.bfloat16)
         v_rows = torch.randn((h_kv, n1, d), generator=gen, device=device).to(torch.bfloat16)
+        k_rows = torch.randn((h_kv, n1, d), generator=gen, device=device).to(torch.bfloat16)
+        k_codes = torch.randint(0, 256, (h_kv, n1, d // 2), generator=gen, device=device,
+                                dtype=torch.uint8)
         idx = outs[0][0]
         a_out = torch.empty((h_q, d), dtype=torch.float32, device=device)
         a_lse = torch.empty((h_q,), dtype=torch.float32, device=device)
-        for _ in range(3):
-            F.sparse_attention(q_all, k_rows, v_rows, idx, out=a_out, lse=a_lse)
-        ab = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        ae = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        for i in range(K):
-            flush.zero_()
-            ab[i].record(stream)
-            F.sparse_attention(q_all, k_rows, v_rows, idx, out=a_out, lse=a_lse)
-            ae[i].record(stream)
-        torch.cuda.synchronize()
-        a_ms = float(np.mean([x.elapsed_time(y) for x, y in zip(ab, ae)]))
         rows = int(((idx >= 0) & (idx < n1)).sum().item())
-        a_bytes = rows * d * 2 * 2 + idx.numel() * 4 + q_all.numel() * q_all.element_size() + \
-            a_out.numel() * 4 + a_lse.numel() * 4
-        a_peak, a_kind = load_peaks()
-        a_gbs = a_bytes / (a_ms * 1e-3) / 1e9
-        attention = {"kernel": "attention_kernel", "ms": a_ms, "rows": rows,
-                     "algorithmic_bytes": a_bytes, "achieved": a_gbs, "peak": a_peak,
-                     "unit": "GB/s", "frac": a_gbs / a_peak, "peak_kind": a_kind,
-                     "l2": "flushed before each launch"}
-        del k_rows, v_rows
+        small = idx.numel() * 4 + q_all.numel() * q_all.element_size() + a_out.numel() * 4 + \
+            a_lse.numel() * 4
+        hbm_peak, hbm_kind = load_peaks()
+
+        def time_attn(call):
+            for _ in range(3):
+                call()
+            ab = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+            ae = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+            for i in range(K):
+                flush.zero_()
+                ab[i].record(stream)
+                call()
+                ae[i].record(stream)
+            torch.cuda.synchronize()
+            return float(np.mean([x.elapsed_time(y) for x, y in zip(ab, ae)]))
+
+        def entry(name, ms, row_bytes, peak, kind, link):
+            b = rows * row_bytes + small
+            gbs = b / (ms * 1e-3) / 1e9
+            return {"variant": name, "ms": ms, "rows": rows, "algorithmic_bytes": b,
+                    "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                    "peak_kind": kind, "bound": link}
+
+        qs = dict(k_qmin=cases[0].qmin, k_qscale=cases[0].qscale)
+        ents = []
+        ms = time_attn(lambda: F.sparse_attention(q_all, k_rows, v_rows, idx, out=a_out, lse=a_lse))
+        ents.append(entry("bf16 K, bf16 V, device", ms, 4 * d, hbm_peak, hbm_kind, "hbm"))
+        ms = time_attn(lambda: F.sparse_attention(q_all, None, v_rows, idx, out=a_out, lse=a_lse,
+                                                  k_codes=k_codes, **qs))
+        ents.append(entry("4-bit K, bf16 V, device", ms, 2 * d + d // 2, hbm_peak, hbm_kind, "hbm"))
+        del k_rows
+        hv = v_rows.cpu().pin_memory()
+        hc = k_codes.cpu().pin_memory()
+        link = measure_h2d_gbs(device)
+        ms = time_attn(lambda: F.sparse_attention(q_all, None, hv, idx, out=a_out, lse=a_lse,
+                                                  k_codes=hc, host_mapped=True, **qs))
+        ents.append(entry("4-bit K, bf16 V, pinned host memory", ms, 2 * d + d // 2, link,
+                          "measured pinned host->device copy", "host-link"))
+        attention = {"kernel": "attention_kernel", "k": k, "l2": "flushed before each launch",
+                     "variants": ents}
+        del v_rows, k_codes, hv, hc
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not ragged:

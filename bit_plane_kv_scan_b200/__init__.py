@@ -7,9 +7,10 @@ library raises.
 """
 
 from .fathom import (  # noqa: F401
-    BF16, F32, FLAG_FORCE_FALLBACK, FLAG_NO_SAMPLING, FLAG_CUDA_CORES, PLANES_DEVICE,
-    PLANES_HOST_MAPPED, BatchedScan, FathomError, Workspace, allocate, allocate_uniform, lib,
-    append_planes, pack_planes,
-    plane_words, profile_scan_kernel, read_report, scan_topk, scan_topk_batched,
-    sparse_attention,
+    BF16, ERR_CUDA, ERR_DEVICE_CHECK, ERR_INVALID_ARGUMENT, ERR_UNSUPPORTED,
+    ERR_WORKSPACE_TOO_SMALL, F32, FLAG_CUDA_CORES, FLAG_FORCE_FALLBACK, FLAG_NO_SAMPLING,
+    MAX_MERGE_PARTS, OK, PLANES_DEVICE, PLANES_HOST_MAPPED, BatchedScan, FathomError, ScanReport,
+    Workspace, allocate, allocate_uniform, append_planes, gather_parts, lib, merge_topk,
+    pack_planes, plane_words, profile_scan_kernel, read_report, scan_topk, scan_topk_batched,
+    sharded_scan_topk, sparse_attention,
 )

@@ -18,12 +18,16 @@ cudaError_t launch_allocate_uniform(int h_q, int d, int budget, uint8_t *alloc,
 cudaError_t launch_append(const uint8_t *codes, int64_t n, int64_t m, int d, int h_kv,
                           const uint32_t *planes_in, uint32_t *planes_out, cudaStream_t stream);
 cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
+                             const uint8_t *k_codes, const float *k_qmin, const float *k_qscale,
                              const uint16_t *v_rows, const int32_t *idx, int64_t n, int d,
                              int h_q, int h_kv, int k, float scale, float *out, float *lse,
                              cudaStream_t stream);
 cudaError_t launch_allocate(const void *q, int q_bf16, const float *sigma, int h_q, int h_kv, int d,
                             int budget, uint8_t *alloc, cudaStream_t stream);
 cudaError_t launch_scan_pipeline(const ScanParams &p, bool any_sampling, cudaStream_t stream);
+cudaError_t launch_merge_parts(const int32_t *in_idx, const float *in_score, int parts,
+                               const int64_t *offsets, int h_q, int k_in, int k, int32_t *out_idx,
+                               float *out_score, cudaStream_t stream);
 int tc_plan_bytes(int d);
 }  // namespace fathom
 
@@ -261,18 +265,39 @@ fathom_status fathom_sparse_attention(const fathom_attention_args *a, void *stre
           (long long)a->n);
   REQUIRE(a->k >= 0, "k=%d is negative", a->k);
   REQUIRE(std::isfinite(a->softmax_scale), "softmax_scale is not finite");
+  REQUIRE(a->kv_location == FATHOM_PLANES_DEVICE || a->kv_location == FATHOM_PLANES_HOST_MAPPED,
+          "kv_location=%d unknown", a->kv_location);
   REQUIRE_DEV(a->q, "q");
   if (a->k > 0) REQUIRE_DEV(a->idx, "idx");
   REQUIRE_DEV(a->out, "out");
   if (a->lse) REQUIRE_DEV(a->lse, "lse");
   if (a->n > 0 && a->k > 0) {
-    REQUIRE_DEV(a->k_rows, "k_rows");
-    REQUIRE_DEV(a->v_rows, "v_rows");
-    REQUIRE(aligned(a->k_rows, 16) && aligned(a->v_rows, 16), "k_rows/v_rows not 16-byte aligned");
+    const PtrKind want = a->kv_location == FATHOM_PLANES_DEVICE ? kPtrDevice : kPtrHostMapped;
+    const char *where = a->kv_location == FATHOM_PLANES_DEVICE
+                            ? "not a device pointer (kv_location=DEVICE)"
+                            : "not pinned, mapped host memory (kv_location=HOST_MAPPED)";
+    auto check_kv = [&](const void *ptr, const char *name) -> fathom_status {
+      if (ptr == nullptr) return fail(FATHOM_ERR_INVALID_ARGUMENT, "%s is NULL", name);
+      if (ptr_kind(ptr) != want) return fail(FATHOM_ERR_INVALID_ARGUMENT, "%s is %s", name, where);
+      return FATHOM_OK;
+    };
+    fathom_status st2 = a->k_codes ? check_kv(a->k_codes, "k_codes") : check_kv(a->k_rows, "k_rows");
+    if (st2 != FATHOM_OK) return st2;
+    st2 = check_kv(a->v_rows, "v_rows");
+    if (st2 != FATHOM_OK) return st2;
+    if (a->k_codes) {
+      REQUIRE_DEV(a->k_qmin, "k_qmin");
+      REQUIRE_DEV(a->k_qscale, "k_qscale");
+      REQUIRE(aligned(a->k_codes, 16), "k_codes not 16-byte aligned");
+    } else {
+      REQUIRE(aligned(a->k_rows, 16), "k_rows not 16-byte aligned");
+    }
+    REQUIRE(aligned(a->v_rows, 16), "v_rows not 16-byte aligned");
   }
-  cudaError_t e = launch_attention(a->q, a->q_dtype == FATHOM_BF16, a->k_rows, a->v_rows, a->idx,
-                                   a->n, a->d, a->h_q, a->h_kv, a->k, a->softmax_scale, a->out,
-                                   a->lse, (cudaStream_t)stream);
+  cudaError_t e = launch_attention(a->q, a->q_dtype == FATHOM_BF16, a->k_rows, a->k_codes,
+                                   a->k_qmin, a->k_qscale, a->v_rows, a->idx, a->n, a->d, a->h_q,
+                                   a->h_kv, a->k, a->softmax_scale, a->out, a->lse,
+                                   (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();
 }
@@ -327,6 +352,7 @@ fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_by
   p.one.q = a->q;
   p.one.alloc = a->alloc;
   p.one.n = a->n;
+  p.n_max = a->n;
   p.one.out_idx = a->out_idx;
   p.one.out_score = a->out_score;
   p.batched = 0;
@@ -382,6 +408,7 @@ fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, s
   ScanParams p;
   memset(&p, 0, sizeof(p));
   p.sessions = a->sessions;
+  p.n_max = a->n_max;
   p.batched = 1;
   p.S = a->num_sessions;
   p.d = a->d;
@@ -399,6 +426,28 @@ fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, s
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = launch_scan_pipeline(p, L.m_max > 0, s);
   if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+  return ok();
+}
+
+fathom_status fathom_merge_topk(const int32_t *in_idx, const float *in_score, int parts,
+                                const int64_t *offsets, int h_q, int k_in, int k, int32_t *out_idx,
+                                float *out_score, void *stream) {
+  REQUIRE(parts >= 1 && parts <= FATHOM_MAX_MERGE_PARTS, "parts=%d out of range [1, %d]", parts,
+          FATHOM_MAX_MERGE_PARTS);
+  REQUIRE(h_q >= 1, "h_q=%d: need >= 1", h_q);
+  REQUIRE(k_in >= 1 && k_in <= FATHOM_MAX_K, "k_in=%d out of range [1, %d]", k_in, FATHOM_MAX_K);
+  REQUIRE(k >= 1 && k <= FATHOM_MAX_K, "k=%d out of range [1, %d]", k, FATHOM_MAX_K);
+  REQUIRE(offsets != nullptr, "offsets is NULL");
+  for (int b = 0; b < parts; ++b)
+    REQUIRE(offsets[b] >= 0 && offsets[b] < ((int64_t)1 << 31), "offsets[%d]=%lld out of range",
+            b, (long long)offsets[b]);
+  REQUIRE_DEV(in_idx, "in_idx");
+  REQUIRE_DEV(in_score, "in_score");
+  REQUIRE_DEV(out_idx, "out_idx");
+  REQUIRE_DEV(out_score, "out_score");
+  cudaError_t e = launch_merge_parts(in_idx, in_score, parts, offsets, h_q, k_in, k, out_idx,
+                                     out_score, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
 }
 

@@ -20,6 +20,13 @@
 // (max, sum, output) in shared memory; CTA 0 of the cluster merges the 8 CTA
 // partials through distributed shared memory and writes the result.
 // Indices outside [0, n) are skipped, as are -1 entries.
+//
+// Keys come either as bf16 rows or as the 4-bit codes the scan's store is
+// packed from (k = m_c + s_c u, dequantised in the gather: a quarter of the
+// bytes of a bf16 row).  Keys and values may live in device memory or in
+// pinned host memory mapped into the device (the pages' offloaded cache,
+// "Fathom: Per-Query Read Depth for Sparse Decoding over Offloaded KV
+// Caches", abstract): then only the selected rows cross the host link.
 #include <cooperative_groups.h>
 
 #include "fathom_internal.cuh"
@@ -39,6 +46,9 @@ struct AttnParams {
   const void *q;
   int q_bf16;
   const uint16_t *k_rows;
+  const uint8_t *k_codes;  // when set: 4-bit keys [h_kv][n][d/2], k = m + s u
+  const float *k_qmin;
+  const float *k_qscale;
   const uint16_t *v_rows;
   const int32_t *idx;
   int64_t n;
@@ -79,7 +89,23 @@ __device__ __forceinline__ float part_value(const uint32_t *w, int i) {
   return bf16_float((uint16_t)(w[i >> 1] >> (16 * (i & 1))));
 }
 
+// The DPL 4-bit codes of dimensions c0 .. c0 + DPL - 1 of a code row (two
+// channels per byte, low nibble = even channel), packed in order from bit 0.
 template <int DPL>
+__device__ __forceinline__ uint32_t load_codes_part(const uint8_t *row, int c0) {
+  if (DPL == 8) return __ldg(reinterpret_cast<const uint32_t *>(row + c0 / 2));
+  if (DPL == 4) return __ldg(reinterpret_cast<const uint16_t *>(row + c0 / 2));
+  if (DPL == 2) return __ldg(row + c0 / 2);
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const int c = c0 + i;
+    w |= (uint32_t)((__ldg(row + c / 2) >> (4 * (c & 1))) & 15u) << (4 * i);
+  }
+  return w;
+}
+
+template <int DPL, bool CODES>
 __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThreads)
     attention_kernel(AttnParams a) {
   grid_dependency_wait();
@@ -107,8 +133,15 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThread
     qv[i] = x * a.qscale;
   }
   const int32_t *ix = a.idx + (int64_t)h * a.k;
-  const uint16_t *Kg = a.k_rows + (int64_t)g * a.n * D + c0;
+  const uint16_t *Kg = CODES ? nullptr : a.k_rows + (int64_t)g * a.n * D + c0;
+  const uint8_t *Cg = CODES ? a.k_codes + (int64_t)g * a.n * (D / 2) : nullptr;
   const uint16_t *Vg = a.v_rows + (int64_t)g * a.n * D + c0;
+  float km[DPL], ks[DPL];  // dequantisation of this lane's dimensions (4-bit keys)
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    km[i] = CODES ? a.k_qmin[(int64_t)g * D + c0 + i] : 0.0f;
+    ks[i] = CODES ? a.k_qscale[(int64_t)g * D + c0 + i] : 0.0f;
+  }
 
   float m = -INFINITY, l = 0.0f, o[DPL];
 #pragma unroll
@@ -117,14 +150,17 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThread
   for (int r0 = (rank * kAttnWarps + warp) * kAttnRows; r0 < a.k;
        r0 += kAttnHeadWarps * kAttnRows) {
     int row[kAttnRows];  // n < 2^31
-    uint32_t kw[kAttnRows][NW], vw[kAttnRows][NW];
+    uint32_t kw[kAttnRows][CODES ? 1 : NW], vw[kAttnRows][NW];
 #pragma unroll
     for (int u = 0; u < kAttnRows; ++u) {
       const int r = r0 + u;
       const int32_t x = r < a.k ? __ldg(ix + r) : -1;
       row[u] = (x >= 0 && (int64_t)x < a.n) ? x : -1;
       if (row[u] >= 0) {
-        load_row_part<DPL>(Kg + (int64_t)row[u] * D, kw[u]);
+        if constexpr (CODES)
+          kw[u][0] = load_codes_part<DPL>(Cg + (int64_t)row[u] * (D / 2), c0);
+        else
+          load_row_part<DPL>(Kg + (int64_t)row[u] * D, kw[u]);
         load_row_part<DPL>(Vg + (int64_t)row[u] * D, vw[u]);
       }
     }
@@ -133,7 +169,14 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThread
       if (row[u] < 0) continue;  // the same for every lane of the warp
       float s = 0.0f;
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) s = fmaf(qv[i], part_value(kw[u], i), s);
+      for (int i = 0; i < DPL; ++i) {
+        float kv;
+        if constexpr (CODES)
+          kv = fmaf(ks[i], (float)((kw[u][0] >> (4 * i)) & 15u), km[i]);
+        else
+          kv = part_value(kw[u], i);
+        s = fmaf(qv[i], kv, s);
+      }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
       const float mn = fmaxf(m, s);
@@ -193,7 +236,24 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThread
   cluster.sync();  // CTA 0 has read the others' shared memory
 }
 
+template <bool CODES>
+static cudaError_t launch_attention_d(const AttnParams &a, int d, dim3 grid, dim3 block,
+                                     cudaStream_t stream) {
+  switch (d / 32) {
+    case 1: return launch_dependent(attention_kernel<1, CODES>, grid, block, 0, stream, a);
+    case 2: return launch_dependent(attention_kernel<2, CODES>, grid, block, 0, stream, a);
+    case 3: return launch_dependent(attention_kernel<3, CODES>, grid, block, 0, stream, a);
+    case 4: return launch_dependent(attention_kernel<4, CODES>, grid, block, 0, stream, a);
+    case 5: return launch_dependent(attention_kernel<5, CODES>, grid, block, 0, stream, a);
+    case 6: return launch_dependent(attention_kernel<6, CODES>, grid, block, 0, stream, a);
+    case 7: return launch_dependent(attention_kernel<7, CODES>, grid, block, 0, stream, a);
+    case 8: return launch_dependent(attention_kernel<8, CODES>, grid, block, 0, stream, a);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
+                             const uint8_t *k_codes, const float *k_qmin, const float *k_qscale,
                              const uint16_t *v_rows, const int32_t *idx, int64_t n, int d,
                              int h_q, int h_kv, int k, float scale, float *out, float *lse,
                              cudaStream_t stream) {
@@ -201,6 +261,9 @@ cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
   a.q = q;
   a.q_bf16 = q_bf16;
   a.k_rows = k_rows;
+  a.k_codes = k_codes;
+  a.k_qmin = k_qmin;
+  a.k_qscale = k_qscale;
   a.v_rows = v_rows;
   a.idx = idx;
   a.n = n;
@@ -211,17 +274,8 @@ cudaError_t launch_attention(const void *q, int q_bf16, const uint16_t *k_rows,
   a.out = out;
   a.lse = lse;
   const dim3 grid(h_q * kAttnSplit), block(kAttnThreads);
-  switch (d / 32) {
-    case 1: return launch_dependent(attention_kernel<1>, grid, block, 0, stream, a);
-    case 2: return launch_dependent(attention_kernel<2>, grid, block, 0, stream, a);
-    case 3: return launch_dependent(attention_kernel<3>, grid, block, 0, stream, a);
-    case 4: return launch_dependent(attention_kernel<4>, grid, block, 0, stream, a);
-    case 5: return launch_dependent(attention_kernel<5>, grid, block, 0, stream, a);
-    case 6: return launch_dependent(attention_kernel<6>, grid, block, 0, stream, a);
-    case 7: return launch_dependent(attention_kernel<7>, grid, block, 0, stream, a);
-    case 8: return launch_dependent(attention_kernel<8>, grid, block, 0, stream, a);
-    default: return cudaErrorInvalidValue;
-  }
+  return k_codes ? launch_attention_d<true>(a, d, grid, block, stream)
+                 : launch_attention_d<false>(a, d, grid, block, stream);
 }
 
 }  // namespace fathom

@@ -112,6 +112,7 @@ struct ScanParams {
   int sample_rank;  // r: threshold = r-th largest sampled score
   int64_t cap;      // candidate capacity per query head
   int64_t m_max;    // sample slots per query head
+  int64_t n_max;    // the workspace's bound on every session's n
   // workspace
   uint32_t *zero;    // prefix of the workspace the plan kernel clears (status, counts, tau)
   int zero_words;
@@ -129,6 +130,19 @@ struct ScanParams {
 
 __device__ __forceinline__ const fathom_session &session_of(const ScanParams &p, int s) {
   return p.batched ? p.sessions[s] : p.one;
+}
+
+// Keys of session s as the kernels use them.  A batched descriptor is read
+// from device memory that the host never checked: an n outside [0, n_max]
+// (the bound the workspace was sized for) makes the session empty, so that no
+// kernel reads or writes past its buffers; the plan kernel records it as a
+// device fault.
+__device__ __forceinline__ bool session_n_valid(const ScanParams &p, int64_t n) {
+  return n >= 0 && n <= p.n_max;
+}
+__device__ __forceinline__ int64_t session_n(const ScanParams &p, int s) {
+  const int64_t n = session_of(p, s).n;
+  return session_n_valid(p, n) ? n : 0;
 }
 
 __host__ __device__ inline int64_t plane_words(int64_t n) { return ((n + 127) / 128) * 4; }

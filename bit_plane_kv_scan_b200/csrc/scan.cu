@@ -249,7 +249,7 @@ __device__ __forceinline__ TileLoc locate(const ScanParams &p, const int *s_tpre
   TileLoc L;
   L.s = lo;
   const fathom_session &se = session_of(p, lo);
-  L.n = se.n;
+  L.n = session_n(p, lo);
   L.W = plane_words(L.n);
   L.planes = se.planes;
   const int per = (int)tiles_per_group<MODE>(L.n, p);
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
   for (int base = 0; base < p.S; base += kScanThreads) {
     const int s = base + tid;
     int v = 0;
-    if (s < p.S) v = (int)(tiles_per_group<MODE>(session_of(p, s).n, p) * p.h_kv);
+    if (s < p.S) v = (int)(tiles_per_group<MODE>(session_n(p, s), p) * p.h_kv);
     const int carry = base > 0 ? s_tprefix[base] : 0;
     __syncthreads();
     const int incl = block_inclusive_scan(v, s_tmp);
@@ -811,7 +811,7 @@ __global__ void __launch_bounds__(1024) threshold_kernel(ScanParams p) {
   allow_dependent_launch();
   const int64_t h = blockIdx.x;
   const int s = (int)(h / p.h_q);
-  const int64_t n = session_of(p, s).n;
+  const int64_t n = session_n(p, s);
   __shared__ unsigned hist[kSelBins];
   __shared__ unsigned s_wsum[32];
   __shared__ float s_mm[2][32];
@@ -929,7 +929,7 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   const fathom_session &se = session_of(p, s);
   const int d = p.d;
   const int g = hl / p.G;
-  const int64_t n = se.n;
+  const int64_t n = session_n(p, s);
   const int64_t W = plane_words(n);
   __shared__ float s_qs[FATHOM_MAX_D];
   __shared__ uint8_t s_t[FATHOM_MAX_D];
@@ -1046,7 +1046,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
   const int s = (int)(h / p.h_q);
   const int hl = (int)(h - (int64_t)s * p.h_q);
   const fathom_session &se = session_of(p, s);
-  const int64_t n = se.n;
+  const int64_t n = session_n(p, s);
+  // a descriptor whose n lies outside [0, n_max] was scanned as empty
+  if (hl == 0 && threadIdx.x == 0 && !session_n_valid(p, se.n))
+    atomicAdd(&p.status->device_faults, 1u);
   const int k = p.k;
   unsigned long long *buf = p.cand + h * p.cap;
   int64_t cnt = p.counts[h];

@@ -40,9 +40,11 @@ EXPORTED = [
     "fathom_scan_topk",
     "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
     "fathom_scan_read_report", "fathom_profile_scan_kernel", "fathom_scan_topk_noalloc",
+    "fathom_scan_read_report_noalloc", "fathom_merge_topk",
     "fathom_sparse_attention",
 ]
 NOALLOC_SCRATCH_BYTES = 16 << 20
+MAX_MERGE_PARTS = 64
 
 
 class FathomError(RuntimeError):
@@ -71,6 +73,8 @@ class AttentionArgs(ctypes.Structure):
         ("d", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("k", ctypes.c_int),
         ("softmax_scale", ctypes.c_float),
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("kv_location", ctypes.c_int), ("k_codes", ctypes.c_void_p),
+        ("k_qmin", ctypes.c_void_p), ("k_qscale", ctypes.c_void_p),
     ]
 
 
@@ -139,6 +143,11 @@ def lib() -> ctypes.CDLL:
         L.fathom_profile_scan_kernel.argtypes = [vp, vp]
         L.fathom_scan_topk_noalloc.restype = ci
         L.fathom_scan_topk_noalloc.argtypes = [ctypes.POINTER(ScanArgs), vp]
+        L.fathom_merge_topk.restype = ci
+        L.fathom_merge_topk.argtypes = [vp, vp, ci, ctypes.POINTER(ctypes.c_int64), ci, ci, ci, vp,
+                                        vp, vp]
+        L.fathom_scan_read_report_noalloc.restype = ci
+        L.fathom_scan_read_report_noalloc.argtypes = [ctypes.POINTER(ScanReport), vp]
         _lib = L
         return L
 
@@ -224,20 +233,33 @@ def allocate_uniform(h_q: int, d: int, budget: int, device=None, stream=None,
     return out
 
 
-def sparse_attention(q: torch.Tensor, k_rows: torch.Tensor, v_rows: torch.Tensor,
+def sparse_attention(q: torch.Tensor, k_rows: Optional[torch.Tensor], v_rows: torch.Tensor,
                      idx: torch.Tensor, softmax_scale: Optional[float] = None, stream=None,
-                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, *,
+                     k_codes: Optional[torch.Tensor] = None, k_qmin: Optional[torch.Tensor] = None,
+                     k_qscale: Optional[torch.Tensor] = None, host_mapped: bool = False):
     """Attention of each query head over its selected keys only.
 
-    q [h_q, d] (bf16/f32); k_rows, v_rows [h_kv, n, d] bf16; idx [h_q, k] int32
-    (entries outside [0, n) are skipped).  Returns (out [h_q, d] f32,
-    lse [h_q] f32)."""
+    q [h_q, d] (bf16/f32); v_rows [h_kv, n, d] bf16; keys either k_rows
+    [h_kv, n, d] bf16 or 4-bit k_codes [h_kv, n, d/2] uint8 with k_qmin,
+    k_qscale [h_kv, d] f32 (k = qmin + qscale * code); idx [h_q, k] int32
+    (entries outside [0, n) are skipped).  host_mapped: the K and V tensors
+    are pinned host memory read across the host link.  Returns (out [h_q, d]
+    f32, lse [h_q] f32)."""
     h_q, d = q.shape
-    h_kv, n, dk = k_rows.shape
-    if k_rows.dtype != torch.bfloat16 or v_rows.dtype != torch.bfloat16:
-        raise TypeError("k_rows and v_rows must be bfloat16")
-    if v_rows.shape != k_rows.shape or dk != d:
-        raise ValueError("k_rows/v_rows must be [h_kv, n, d] with the query's d")
+    h_kv, n, dv = v_rows.shape
+    if v_rows.dtype != torch.bfloat16:
+        raise TypeError("v_rows must be bfloat16")
+    if k_codes is None:
+        if k_rows is None or k_rows.dtype != torch.bfloat16 or k_rows.shape != v_rows.shape:
+            raise TypeError("k_rows must be bfloat16 [h_kv, n, d] like v_rows")
+    else:
+        if k_codes.dtype != torch.uint8 or tuple(k_codes.shape) != (h_kv, n, d // 2):
+            raise TypeError("k_codes must be uint8 [h_kv, n, d/2]")
+        if k_qmin is None or k_qscale is None:
+            raise TypeError("k_codes needs k_qmin and k_qscale")
+    if dv != d:
+        raise ValueError("v_rows must be [h_kv, n, d] with the query's d")
     if idx.dtype != torch.int32 or idx.dim() != 2 or idx.shape[0] != h_q:
         raise TypeError("idx must be an int32 [h_q, k] tensor")
     if softmax_scale is None:
@@ -246,10 +268,13 @@ def sparse_attention(q: torch.Tensor, k_rows: torch.Tensor, v_rows: torch.Tensor
         out = torch.empty((h_q, d), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((h_q,), dtype=torch.float32, device=q.device)
-    q, k_rows, v_rows, idx = q.contiguous(), k_rows.contiguous(), v_rows.contiguous(), idx.contiguous()
-    a = AttentionArgs(q=_ptr(q), q_dtype=_dtype_code(q), k_rows=_ptr(k_rows), v_rows=_ptr(v_rows),
+    q, idx = q.contiguous(), idx.contiguous()
+    a = AttentionArgs(q=_ptr(q), q_dtype=_dtype_code(q),
+                      k_rows=None if k_codes is not None else _ptr(k_rows), v_rows=_ptr(v_rows),
                       idx=_ptr(idx), n=n, d=d, h_q=h_q, h_kv=h_kv, k=idx.shape[1],
-                      softmax_scale=float(softmax_scale), out=_ptr(out), lse=_ptr(lse))
+                      softmax_scale=float(softmax_scale), out=_ptr(out), lse=_ptr(lse),
+                      kv_location=PLANES_HOST_MAPPED if host_mapped else PLANES_DEVICE,
+                      k_codes=_ptr(k_codes), k_qmin=_ptr(k_qmin), k_qscale=_ptr(k_qscale))
     _check(lib().fathom_sparse_attention(ctypes.byref(a), _stream(stream)))
     return out, lse
 
@@ -380,6 +405,69 @@ def scan_topk_batched(sessions: Sequence[dict], k: int, d: int, h_q: int, h_kv: 
     alloc, n (and optionally out_idx/out_score).  Returns a list of (idx, score)."""
     return BatchedScan(sessions, k, d, h_q, h_kv, q_dtype, host_mapped=host_mapped, flags=flags,
                        device=device)(workspace, stream)
+
+
+def merge_topk(idx_parts: torch.Tensor, score_parts: torch.Tensor, offsets: Sequence[int], k: int,
+               stream=None, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+    """The top-k of token-range shards' top-k lists.
+
+    idx_parts int32 [parts, h_q, k_in] (local indices, -1 padding) and
+    score_parts f32 [parts, h_q, k_in], each part sorted as fathom_scan_topk
+    returns it; offsets[p] is the first token of part p's range.  Returns
+    (idx int32 [h_q, k], score f32 [h_q, k]) with global indices."""
+    if idx_parts.dtype != torch.int32 or score_parts.dtype != torch.float32:
+        raise TypeError("idx_parts must be int32 and score_parts float32")
+    if idx_parts.dim() != 3 or idx_parts.shape != score_parts.shape:
+        raise ValueError("idx_parts and score_parts must both be [parts, h_q, k_in]")
+    parts, h_q, k_in = idx_parts.shape
+    if len(offsets) != parts:
+        raise ValueError("one offset per part")
+    if out is None:
+        out = (torch.empty((h_q, k), dtype=torch.int32, device=idx_parts.device),
+               torch.empty((h_q, k), dtype=torch.float32, device=idx_parts.device))
+    offs = (ctypes.c_int64 * parts)(*[int(o) for o in offsets])
+    ip, sp = idx_parts.contiguous(), score_parts.contiguous()
+    _check(lib().fathom_merge_topk(_ptr(ip), _ptr(sp), parts, offs, h_q, k_in, int(k),
+                                   _ptr(out[0]), _ptr(out[1]), _stream(stream)))
+    return out
+
+
+def gather_parts(idx: torch.Tensor, score: torch.Tensor, n_local: int, group=None):
+    """The collective step of token-range sharding: every rank's top-k lists
+    (idx int32 [h_q, k] local indices, score f32 [h_q, k]) and key count go to
+    every rank.  Returns (idx_parts [world, h_q, k], score_parts
+    [world, h_q, k], offsets) in rank order, offsets[r] being the first token
+    of rank r's range (ranks hold consecutive ranges in rank order)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    n_t = torch.tensor([int(n_local)], dtype=torch.int64, device=idx.device)
+    ns = [torch.empty_like(n_t) for _ in range(world)]
+    dist.all_gather(ns, n_t, group=group)
+    counts = [int(x.item()) for x in ns]
+    offsets = [sum(counts[:r]) for r in range(world)]
+    idx_l = [torch.empty_like(idx) for _ in range(world)]
+    sc_l = [torch.empty_like(score) for _ in range(world)]
+    dist.all_gather(idx_l, idx.contiguous(), group=group)
+    dist.all_gather(sc_l, score.contiguous(), group=group)
+    return torch.stack(idx_l), torch.stack(sc_l), offsets
+
+
+def sharded_scan_topk(planes: torch.Tensor, qmin: torch.Tensor, qscale: torch.Tensor,
+                      q: torch.Tensor, alloc: torch.Tensor, k: int, n_local: int, *,
+                      group=None, workspace: Optional[Workspace] = None, stream=None):
+    """Token-range sharding over the ranks of a torch.distributed group.
+
+    Every rank holds the planes of its own contiguous range of the context
+    (rank order = token order; n_local keys here) and the same q and alloc.
+    Each rank scans its range (fathom_scan_topk), one all-gather brings every
+    rank's k (index, score) pairs per head to every rank (gather_parts), and
+    fathom_merge_topk returns the context's top-k with global indices
+    (identical on every rank).  The quantiser statistics (qmin, qscale) are
+    the context's, shared by every range."""
+    idx, sc = scan_topk(planes, qmin, qscale, q, alloc, k, n_local, workspace=workspace,
+                        stream=stream)
+    idx_all, sc_all, offsets = gather_parts(idx, sc, n_local, group=group)
+    return merge_topk(idx_all, sc_all, offsets, k, stream=stream)
 
 
 def profile_scan_kernel(begin: Optional[torch.cuda.Event], end: Optional[torch.cuda.Event]):

@@ -81,6 +81,7 @@ typedef enum fathom_planes_location {
 #define FATHOM_MAX_D 256    /* d is a multiple of 32, 32 <= d <= 256 */
 #define FATHOM_MAX_GROUP 4  /* G = h_q / h_kv is 1, 2 or 4 */
 #define FATHOM_MAX_K 8192   /* 1 <= k <= 8192 */
+#define FATHOM_MAX_MERGE_PARTS 64  /* partial lists one fathom_merge_topk call merges */
 
 /* Test knobs for fathom_scan_args.flags (0 in normal use). */
 #define FATHOM_FLAG_NO_SAMPLING 1u     /* skip the threshold sample: every key is a candidate */
@@ -219,7 +220,11 @@ FATHOM_API fathom_status fathom_scan_topk(const fathom_scan_args *args, void *wo
 /* Batched ragged sessions (abstract: many sessions are resident together): one
  * set of launches scores every session; sessions share d, h_q, h_kv, k and
  * the dtype and differ in n and buffers.  `sessions` is a DEVICE array of S
- * descriptors (pointers in it are not checked on the host). */
+ * descriptors, which the host never reads: its pointers are not checked.
+ * The kernels check each descriptor's n against n_max (the bound the
+ * workspace was sized for): a session with n < 0 or n > n_max is scanned as
+ * empty (its heads get index -1, score -inf) and counted in the report's
+ * device_faults, so fathom_scan_read_report returns FATHOM_ERR_DEVICE_CHECK. */
 typedef struct fathom_session {
   const uint32_t *planes;  /* [h_kv][d][4][fathom_plane_words(n)] */
   const float *qmin;       /* [h_kv][d] */
@@ -263,7 +268,10 @@ FATHOM_API fathom_status fathom_scan_topk_batched(const fathom_batched_args *arg
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.  The
  *     first call on each device looks up the scratch array's device address
  *     (cudaGetSymbolAddress, which may load the library's kernels onto that
- *     device); make that first call before any stream capture.
+ *     device); make that first call before any stream capture.  The address
+ *     is kept per device together with the id of the CUDA context it belongs
+ *     to: after a device reset (cudaDeviceReset) the next call runs that
+ *     set-up again, so it too should come before any capture.
  *   - All calls share the one array, which keeps the previous call's data;
  *     each call clears the counters that must start at zero.  Calls whose
  *     work overlaps on the GPU (different streams, or different host threads
@@ -293,6 +301,40 @@ typedef struct fathom_scan_report {
 FATHOM_API fathom_status fathom_scan_read_report(const void *workspace, fathom_scan_report *report,
                                       void *stream);
 
+/* fathom_scan_read_report_noalloc -- the report of the last
+ * fathom_scan_topk_noalloc on the current device (its status block lives in
+ * the built-in scratch, whose address the caller never sees).  Same fields
+ * and status as fathom_scan_read_report; synchronises `stream`.  Like the
+ * scan itself it allocates nothing; no counterpart in the paper. */
+FATHOM_API fathom_status fathom_scan_read_report_noalloc(fathom_scan_report *report, void *stream);
+
+/* fathom_merge_topk -- the top-k of a scan whose keys were split into token
+ * ranges: the last step of token-range sharding, where each GPU scans the
+ * planes of its own range of the context (fathom_scan_topk, local indices)
+ * and the per-range lists are gathered (one all-gather of parts x k
+ * (index, score) pairs per head over NVLink).  The pages rank every key of
+ * the context for each top-k step (abstract); the k best of the context are
+ * the k best of the union of every range's k best, so the merged answer is
+ * the unsplit scan's.
+ *   in_idx     int32 [parts][h_q][k_in], in_score float [parts][h_q][k_in]:
+ *              each part's fathom_scan_topk output for its range -- sorted by
+ *              score descending then index ascending, -1 padding at the tail;
+ *              indices local to the range.
+ *   offsets    HOST array int64 [parts]: first token of each range, so that
+ *              a part's global index is offsets[p] + local index.  Ranges
+ *              must not overlap; global indices must stay below 2^31 - 1
+ *              (larger ones are dropped).
+ *   out_idx    int32 [h_q][k], out_score float [h_q][k]: the k best by score
+ *              descending then global index ascending; -1 / -inf past the
+ *              number of entries.
+ * Requires 1 <= parts <= FATHOM_MAX_MERGE_PARTS, 1 <= k_in, k <= FATHOM_MAX_K,
+ * h_q >= 1.  Device pointers; no workspace.  An input list that is not
+ * sorted gives an unspecified (but in-bounds) result.
+ */
+FATHOM_API fathom_status fathom_merge_topk(const int32_t *in_idx, const float *in_score, int parts,
+                                           const int64_t *offsets, int h_q, int k_in, int k,
+                                           int32_t *out_idx, float *out_score, void *stream);
+
 /* fathom_sparse_attention -- the step after the scan: each query head's
  * attention over only the keys its top-k selected (method paragraph 1: the
  * scan finds the top-k candidates, and only the few KV rows that win are
@@ -306,6 +348,15 @@ FATHOM_API fathom_status fathom_scan_read_report(const void *workspace, fathom_s
  *   q        [h_q][d], FATHOM_BF16 or FATHOM_F32.
  *   k_rows, v_rows   bf16 [h_kv][n][d]: the serving stack's keys and values
  *            (16-byte aligned).
+ *   k_codes  optional uint8 [h_kv][n][d/2]: the 4-bit key codes (the layout
+ *            fathom_pack_planes reads) with k_qmin, k_qscale float [h_kv][d];
+ *            when set, key row i is k_qmin + k_qscale * code (the 4-bit
+ *            dequantisation, a quarter of a bf16 row's bytes per gathered
+ *            key) and k_rows is not read (it may be NULL).
+ *   kv_location  FATHOM_PLANES_DEVICE, or FATHOM_PLANES_HOST_MAPPED when
+ *            k_rows / k_codes and v_rows are pinned host memory mapped into
+ *            the device (the pages' offloaded KV cache, whose title names it):
+ *            only the selected rows cross the host link.
  *   idx      int32 [h_q][k], e.g. fathom_scan_topk's out_idx.
  *   out      float [h_q][d]; lse float [h_q] or NULL.
  * Requires d as FATHOM_MAX_D, h_q a multiple of h_kv, k >= 0, 0 <= n < 2^31
@@ -322,6 +373,10 @@ typedef struct fathom_attention_args {
   float softmax_scale;
   float *out;
   float *lse;
+  int kv_location;          /* fathom_planes_location of the K and V rows */
+  const uint8_t *k_codes;   /* optional 4-bit keys (then k_rows is unused) */
+  const float *k_qmin;      /* [h_kv][d], with k_codes */
+  const float *k_qscale;    /* [h_kv][d], with k_codes */
 } fathom_attention_args;
 
 FATHOM_API fathom_status fathom_sparse_attention(const fathom_attention_args *args, void *stream);

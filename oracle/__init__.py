@@ -213,7 +213,9 @@ def sparse_attention(q, k_rows, v_rows, idx, scale: float):
     paragraph 1), by its definition in fp64:
         s_r = scale * <q_h, K[g][idx_r]>,  w = softmax(s),  o_h = sum_r w_r V[g][idx_r],
         lse_h = log sum_r exp(s_r),
-    over the entries idx_r >= 0 of head h's row (head h reads KV head h // G).
+    over the entries of head h's row that name a key, 0 <= idx_r < n (head h
+    reads KV head h // G); other entries (the scan's -1 padding, anything at
+    or past n) select nothing.
     q [h_q, d]; k_rows, v_rows [h_kv, n, d]; idx [h_q, k] int.
     Returns (o float64 [h_q, d], lse float64 [h_q]); a head with no selected
     key gets o = 0 and lse = -inf."""
@@ -223,10 +225,11 @@ def sparse_attention(q, k_rows, v_rows, idx, scale: float):
     idx = np.asarray(idx)
     h_q, d = q.shape
     G = h_q // k_rows.shape[0]
+    n = k_rows.shape[1]
     out = np.zeros((h_q, d))
     lse = np.full(h_q, -np.inf)
     for h in range(h_q):
-        sel = idx[h][idx[h] >= 0].astype(np.int64)
+        sel = idx[h][(idx[h] >= 0) & (idx[h] < n)].astype(np.int64)
         if sel.size == 0:
             continue
         g = h // G

@@ -119,6 +119,8 @@ def test_sparse_attention_rejects_bad_arguments(L):
     assert L.fathom_sparse_attention(args(n=-5), None) == F.ERR_INVALID_ARGUMENT
     assert L.fathom_sparse_attention(args(softmax_scale=float("inf")), None) == F.ERR_INVALID_ARGUMENT
     assert L.fathom_sparse_attention(args(q_dtype=9), None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_sparse_attention(args(kv_location=5), None) == F.ERR_INVALID_ARGUMENT
+    assert b"kv_location" in L.fathom_last_error()
     assert L.fathom_sparse_attention(args(), None) == F.ERR_INVALID_ARGUMENT
     assert b"q" in L.fathom_last_error()
 
@@ -159,3 +161,25 @@ def test_batched_rejects_bad_arguments(L):
 
 def test_report_rejects_null(L):
     assert L.fathom_scan_read_report(None, None, None) == F.ERR_INVALID_ARGUMENT
+
+
+def test_merge_rejects_bad_arguments(L):
+    offs = (ctypes.c_int64 * 2)(0, 100)
+    m = L.fathom_merge_topk
+    assert m(None, None, 0, offs, 8, 64, 64, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert m(None, None, F.MAX_MERGE_PARTS + 1, offs, 8, 64, 64, None, None, None) == \
+        F.ERR_INVALID_ARGUMENT
+    assert m(None, None, 2, offs, 0, 64, 64, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert m(None, None, 2, offs, 8, 0, 64, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert m(None, None, 2, offs, 8, 64, 8193, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert m(None, None, 2, None, 8, 64, 64, None, None, None) == F.ERR_INVALID_ARGUMENT
+    bad = (ctypes.c_int64 * 2)(0, 1 << 31)
+    assert m(None, None, 2, bad, 8, 64, 64, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert b"offsets" in L.fathom_last_error()
+    assert m(None, None, 2, offs, 8, 64, 64, None, None, None) == F.ERR_INVALID_ARGUMENT
+    assert b"in_idx" in L.fathom_last_error()
+
+
+def test_noalloc_report_rejects_null(L):
+    assert L.fathom_scan_read_report_noalloc(None, None) == F.ERR_INVALID_ARGUMENT
+    assert b"report" in L.fathom_last_error()

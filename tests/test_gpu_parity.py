@@ -14,7 +14,8 @@ import torch
 
 import oracle
 import synthkv
-from parity import check_dense, check_scores_at, check_topk, check_topk_sampled, score_scale
+from parity import (check_dense, check_scores_at, check_topk, check_topk_sampled,
+                    fixed_point_bound, score_scale)
 
 pytestmark = pytest.mark.gpu
 
@@ -145,6 +146,17 @@ def _want_alloc(case, cn, budget, uniform):
     return oracle.allocate_heads(cn[3], _np(case.sigma), budget)
 
 
+def _tol(flags, q_h, qmin_g, qscale_g, t_h):
+    """Score tolerance of one head (tests/parity.py): the paths that
+    accumulate fp32 products (the CUDA-core scan and the exact single-block
+    fallback) take the S_h / 8 floor; the tensor-core path takes the bare
+    1e-5 and, for a score so close to 0 that 1e-5 of it is below the
+    fixed-point resolution, its exact fixed-point bound B Delta_h / 2."""
+    if flags & (F.FLAG_CUDA_CORES | F.FLAG_FORCE_FALLBACK):
+        return dict(floor=score_scale(q_h, qmin_g, qscale_g) / 8.0)
+    return dict(abs_tol=fixed_point_bound(q_h, qscale_g, t_h))
+
+
 def _full_check(case, budget, k, flags=0, what="", uniform=False):
     planes, alloc, (idx, sc, dbg) = run_gpu(case, budget, k, flags=flags, debug=True,
                                             uniform=uniform)
@@ -159,7 +171,8 @@ def _full_check(case, budget, k, flags=0, what="", uniform=False):
         ref = oracle_head(cn, h, want_alloc[h])
         scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
         check_dense(dbg[h], ref, scale, "%s head %d" % (what, h))
-        check_topk(idx[h], sc[h], ref, k, scale, "%s head %d" % (what, h))
+        check_topk(idx[h], sc[h], ref, k, what="%s head %d" % (what, h),
+                   **_tol(flags, cn[3][h], cn[1][g], cn[2][g], want_alloc[h]))
 
 
 @pytest.mark.parametrize("h_q,d,B", [(1, 32, 0), (4, 64, 100), (32, 128, 92), (32, 128, 136),
@@ -210,6 +223,82 @@ def test_degenerate_budgets(B):
     if B == 0:
         _, _, (idx, sc) = run_gpu(case, 0, 50)
         assert (_np(idx) == np.arange(50)[None, :]).all()
+
+
+@pytest.mark.parametrize("cuda_cores", [False, True])
+def test_empty_union_on_a_stale_workspace(cuda_cores):
+    """B = 0 (every union prefix empty) on a workspace that holds no plan of
+    this call: first a scan at another d fills it, then a fresh workspace is
+    filled with 0xFF bytes.  Both must give the oracle's answer (the scan may
+    read nothing outside the planes of this call)."""
+    flags = F.FLAG_CUDA_CORES if cuda_cores else 0
+    dev = torch.device("cuda")
+    other = synthkv.make_case(seed=41, n=9000, h_kv=2, h_q=8, d=256, q_dtype="bf16")
+    run_gpu(other, 700, 40, flags=flags)
+    case = synthkv.make_case(seed=42, n=7000, h_kv=2, h_q=8, d=128, q_dtype="bf16")
+    for fill in (None, 0xFF):
+        ws = None
+        if fill is not None:
+            ws = F.Workspace(dev)
+            ws.buf = torch.full((64 << 20,), fill, dtype=torch.uint8, device=dev)
+        q = case.q_storage().to(dev)
+        alloc = F.allocate(q, case.sigma.to(dev), 0)
+        planes = F.pack_planes(case.codes.to(dev))
+        idx, sc, dbg = F.scan_topk(planes, case.qmin.to(dev), case.qscale.to(dev), q, alloc, 50,
+                                   case.n, debug_scores=True, flags=flags, workspace=ws)
+        torch.cuda.synchronize()
+        rep = F.read_report(ws)
+        assert rep.device_faults == 0 and rep.union_planes == 0
+        cn = case_np(case)
+        for h in range(case.h_q):
+            g = h // case.group
+            ref = oracle_head(cn, h, np.zeros(case.d, dtype=np.uint8))
+            scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
+            check_dense(_np(dbg)[h], ref, scale, "B=0 fill=%s head %d" % (fill, h))
+            check_topk(_np(idx)[h], _np(sc)[h], ref, 50, what="B=0 fill=%s head %d" % (fill, h),
+                       **_tol(flags, cn[3][h], cn[1][g], cn[2][g], np.zeros(case.d, np.uint8)))
+            assert (_np(idx)[h] == np.arange(50)).all()
+
+
+@pytest.mark.parametrize("cuda_cores", [False, True])
+def test_batched_descriptor_beyond_n_max(cuda_cores):
+    """A session descriptor whose n exceeds the n_max the workspace was sized
+    for is scanned as empty and reported as a device fault; the other
+    sessions are unaffected."""
+    import ctypes
+    flags = F.FLAG_CUDA_CORES if cuda_cores else 0
+    dev = torch.device("cuda")
+    cases = [synthkv.make_case(seed=50 + i, n=n, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+             for i, n in enumerate((6000, 3000))]
+    descs = []
+    for c in cases:
+        q = c.q_storage().to(dev)
+        descs.append(dict(planes=F.pack_planes(c.codes.to(dev)), qmin=c.qmin.to(dev),
+                          qscale=c.qscale.to(dev), q=q, alloc=F.allocate(q, c.sigma.to(dev), 92),
+                          n=c.n))
+    scan = F.BatchedScan(descs, 64, 128, 4, 1, torch.bfloat16, flags=flags, device=dev)
+    scan.args.n_max = 4000  # session 0 (n = 6000) is beyond the bound
+    L = F.lib()
+    need = L.fathom_scan_topk_batched_workspace_size(ctypes.byref(scan.args))
+    ws = F.Workspace(dev)
+    buf = ws.get(need)
+    st = L.fathom_scan_topk_batched(ctypes.byref(scan.args), ctypes.c_void_p(buf.data_ptr()), need,
+                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == F.OK, L.fathom_last_error()
+    torch.cuda.synchronize()
+    rep = F.ScanReport()
+    st = L.fathom_scan_read_report(ctypes.c_void_p(buf.data_ptr()), ctypes.byref(rep), None)
+    assert st == F.ERR_DEVICE_CHECK and rep.device_faults == 1
+    i0, s0 = scan.outs[0]
+    assert (_np(i0) == -1).all() and np.isneginf(_np(s0)).all()
+    c = cases[1]
+    cn = case_np(c)
+    want = oracle.allocate_heads(cn[3], _np(c.sigma), 92)
+    i1, s1 = _np(scan.outs[1][0]), _np(scan.outs[1][1])
+    for h in range(4):
+        ref = oracle_head(cn, h, want[h])
+        check_topk(i1[h], s1[h], ref, 64, what="session 1 head %d" % h,
+                   **_tol(flags, cn[3][h], cn[1][0], cn[2][0], want[h]))
 
 
 def test_k_larger_than_n_and_empty():
@@ -272,8 +361,8 @@ def test_fallback_with_compaction():
     cn = case_np(case)
     for h in range(4):
         ref = oracle_head(cn, h, _np(alloc)[h])
-        check_topk(_np(idx)[h], _np(sc)[h], ref, 1000, score_scale(cn[3][h], cn[1][0], cn[2][0]),
-                   "fallback head %d" % h)
+        check_topk(_np(idx)[h], _np(sc)[h], ref, 1000, what="fallback head %d" % h,
+                   **_tol(F.FLAG_FORCE_FALLBACK, cn[3][h], cn[1][0], cn[2][0], _np(alloc)[h]))
 
 
 # --------------------------------------------------- CUDA-core scan kernel --
@@ -312,14 +401,14 @@ def _check_config(case, budget, k, heads_full, what, host_mapped=False, flags=0,
     G = case.group
     for h in range(case.h_q):
         g = h // G
-        scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
         kk = min(k, case.n)
         ref_at = oracle.scores_at(cn[0][g], cn[1][g], cn[2][g], cn[3][h], want_alloc[h],
                                   idx[h, :kk].astype(np.int64))
-        check_topk_sampled(idx[h], sc[h], ref_at, k, case.n, scale, "%s head %d" % (what, h))
+        tol = _tol(flags, cn[3][h], cn[1][g], cn[2][g], want_alloc[h])
+        check_topk_sampled(idx[h], sc[h], ref_at, k, case.n, what="%s head %d" % (what, h), **tol)
         if h in heads_full:
             ref = oracle_head(cn, h, want_alloc[h])
-            check_topk(idx[h], sc[h], ref, k, scale, "%s head %d" % (what, h))
+            check_topk(idx[h], sc[h], ref, k, what="%s head %d" % (what, h), **tol)
     return idx, sc
 
 
@@ -344,9 +433,10 @@ def decode_1m():
 
 @pytest.mark.parametrize("B", [92, 136])
 def test_decode_1m(decode_1m, B):
-    # full brute force on one query head of every KV head; sampled checks on all
-    _check_config(decode_1m, B, 2048, heads_full={0, 5, 10, 15, 16, 21, 26, 31},
-                  what="1M B=%d" % B)
+    # B = 92 (the benchmarked step): full brute force on every query head;
+    # B = 136: on one query head of every KV head; sampled checks on all
+    heads = set(range(32)) if B == 92 else {0, 5, 10, 15, 16, 21, 26, 31}
+    _check_config(decode_1m, B, 2048, heads_full=heads, what="1M B=%d" % B)
     rep = F.read_report()
     assert rep.fallback_heads == 0
 
@@ -376,13 +466,14 @@ def test_host_resident_1m_budget_sweep():
     case = synthkv.make_case(c["seed"], c["n"], c["h_kv"], c["h_q"], c["d"], c["q_dtype"],
                              device="cuda", keep_keys=False)
     for B in c["budgets"]:
-        idx_h, sc_h = _check_config(case, B, 2048, heads_full={3} if B in (92, 512) else set(),
+        # full brute force on one query head of every KV head, for every budget
+        idx_h, sc_h = _check_config(case, B, 2048, heads_full={3, 4, 9, 14, 19, 20, 25, 30},
                                     what="host B=%d" % B, host_mapped=True)
         _, _, (idx_d, sc_d) = run_gpu(case, B, 2048)
         np.testing.assert_array_equal(idx_h, _np(idx_d))
         np.testing.assert_array_equal(sc_h, _np(sc_d))
     # the CUDA-core scan reads host-resident planes too
-    idx_h, sc_h = _check_config(case, 92, 2048, heads_full={3}, what="cc host B=92",
+    idx_h, sc_h = _check_config(case, 92, 2048, heads_full={3, 30}, what="cc host B=92",
                                 host_mapped=True, flags=F.FLAG_CUDA_CORES)
     _, _, (idx_d, sc_d) = run_gpu(case, 92, 2048, flags=F.FLAG_CUDA_CORES)
     np.testing.assert_array_equal(idx_h, _np(idx_d))
@@ -417,13 +508,14 @@ def test_ragged_32_sessions_batched(cuda_cores):
         for h in range(32):
             g = h // 4
             t_h = want_alloc[i * 32 + h]
-            scale = score_scale(cn[3][h], cn[1][g], cn[2][g])
             ref_at = oracle.scores_at(cn[0][g], cn[1][g], cn[2][g], cn[3][h], t_h,
                                       idx[h, :min(k, s.n)].astype(np.int64))
-            check_topk_sampled(idx[h], sc[h], ref_at, k, s.n, scale, "session %d head %d" % (i, h))
+            tol = _tol(flags, cn[3][h], cn[1][g], cn[2][g], t_h)
+            check_topk_sampled(idx[h], sc[h], ref_at, k, s.n, what="session %d head %d" % (i, h),
+                               **tol)
             if i in (0, 13, 31) and h in (0, 9, 18, 27):
                 ref = oracle_head(cn, h, t_h)
-                check_topk(idx[h], sc[h], ref, k, scale, "session %d head %d" % (i, h))
+                check_topk(idx[h], sc[h], ref, k, what="session %d head %d" % (i, h), **tol)
 
 
 # ------------------------------------------------------ sparse attention --
@@ -485,8 +577,70 @@ def test_sparse_attention_random_rows(n, h_kv, G, d, k, qd):
     scale = 1.0 / np.sqrt(d)
     out, lse = F.sparse_attention(q, K, V, idx, scale)
     torch.cuda.synchronize()
-    ref_o, ref_l = _attention_ref(q, K, V, idx, scale, h_kv)
+    # the oracle on the whole K/V and the raw entries (it skips those outside [0, n))
+    ref_o, ref_l = oracle.sparse_attention(_np(q.float()).astype(np.float64),
+                                           _np(K.float()), _np(V.float()), _np(idx), scale)
     _check_attention(out, lse, ref_o, ref_l, V, "n=%d d=%d k=%d" % (n, d, k))
+
+
+def _dequant_rows(codes, qmin, qscale):
+    """Key rows m_c + s_c u from 4-bit codes [h_kv, n, d/2] (low nibble =
+    even channel), in fp64 from the fp32 statistics."""
+    c = np.asarray(codes)
+    u = np.empty(c.shape[:-1] + (2 * c.shape[-1],), dtype=np.float64)
+    u[..., 0::2] = c & 15
+    u[..., 1::2] = c >> 4
+    m = np.asarray(qmin, dtype=np.float64)[:, None, :]
+    s = np.asarray(qscale, dtype=np.float64)[:, None, :]
+    return m + s * u
+
+
+@pytest.mark.parametrize("host_mapped", [False, True])
+@pytest.mark.parametrize("n,h_kv,G,d,k,qd", [(5000, 2, 4, 128, 64, "bf16"), (3000, 1, 1, 32, 300, "f32"),
+                                            (2000, 2, 2, 256, 100, "bf16"), (700, 1, 4, 96, 1000, "bf16"),
+                                            (4000, 1, 2, 160, 257, "f32")])
+def test_sparse_attention_4bit_keys_and_host_rows(n, h_kv, G, d, k, qd, host_mapped):
+    """Keys gathered as 4-bit codes and dequantised in the gather, bf16
+    values; with host_mapped the codes and values sit in pinned host memory
+    and only the selected rows cross the host link.  Also bf16 key rows from
+    host memory."""
+    dev = torch.device("cuda")
+    h_q = h_kv * G
+    rng = np.random.default_rng(3 * n + d)
+    codes = torch.from_numpy(rng.integers(0, 256, size=(h_kv, n, d // 2), dtype=np.uint8))
+    qmin = torch.from_numpy(rng.normal(size=(h_kv, d)).astype(np.float32))
+    qscale = torch.from_numpy(np.exp(rng.uniform(-3, 0, size=(h_kv, d))).astype(np.float32))
+    Kb = _bf16_rows((h_kv, n, d), n + 5, dev)
+    V = _bf16_rows((h_kv, n, d), n + 6, dev)
+    q = torch.from_numpy(rng.normal(size=(h_q, d)).astype(np.float32))
+    q = (q.to(torch.bfloat16) if qd == "bf16" else q).to(dev)
+    idx = rng.integers(0, n, size=(h_q, k)).astype(np.int32)
+    idx[0, k // 3:] = -1
+    if h_q > 1:
+        idx[1, 0] = n
+        idx[h_q - 1, :] = -1
+    idx_t = torch.from_numpy(idx).to(dev)
+    scale = 1.0 / np.sqrt(d)
+    if host_mapped:
+        codes_u = codes.pin_memory()
+        V_u = V.cpu().pin_memory()
+        Kb_u = Kb.cpu().pin_memory()
+    else:
+        codes_u, V_u, Kb_u = codes.to(dev), V, Kb
+    out, lse = F.sparse_attention(q, None, V_u, idx_t, scale, k_codes=codes_u,
+                                  k_qmin=qmin.to(dev), k_qscale=qscale.to(dev),
+                                  host_mapped=host_mapped)
+    torch.cuda.synchronize()
+    Kd = _dequant_rows(codes.numpy(), qmin.numpy(), qscale.numpy())
+    ref_o, ref_l = oracle.sparse_attention(_np(q.float()).astype(np.float64), Kd,
+                                           _np(V.float()), idx, scale)
+    _check_attention(out, lse, ref_o, ref_l, V, "4-bit keys n=%d d=%d host=%d" % (n, d, host_mapped))
+    if host_mapped:
+        out2, lse2 = F.sparse_attention(q, Kb_u, V_u, idx_t, scale, host_mapped=True)
+        torch.cuda.synchronize()
+        ref_o2, ref_l2 = oracle.sparse_attention(_np(q.float()).astype(np.float64),
+                                                 _np(Kb.float()), _np(V.float()), idx, scale)
+        _check_attention(out2, lse2, ref_o2, ref_l2, V, "host bf16 keys n=%d d=%d" % (n, d))
 
 
 def test_sparse_attention_after_the_scan(decode_1m):
@@ -536,3 +690,47 @@ def test_append_token_by_token():
         planes = F.append_planes(planes, i, codes[:, i:i + 1].contiguous())
     torch.cuda.synchronize()
     np.testing.assert_array_equal(_planes_np(planes), oracle.pack_planes(_np(case.codes)))
+
+
+# ---------------------------------------------------- token-range sharding --
+
+@pytest.mark.parametrize("cuts,k", [((0, 3000, 9000), 50), ((0, 1, 4096, 4097, 20000), 300),
+                                    ((0, 20000), 64), ((0, 6000, 12000, 18000, 20000), 2000)])
+def test_token_range_shards_merge_to_the_unsplit_topk(cuts, k):
+    """The scan split into token ranges (as sharded_scan_topk splits it over
+    GPUs, here all on one device): each range packed and scanned on its own,
+    the lists merged by fathom_merge_topk, equals the oracle's top-k of the
+    whole context."""
+    dev = torch.device("cuda")
+    n = cuts[-1]
+    case = synthkv.make_case(seed=70 + len(cuts), n=n, h_kv=2, h_q=8, d=128, q_dtype="bf16")
+    q = case.q_storage().to(dev)
+    alloc = F.allocate(q, case.sigma.to(dev), 92)
+    codes = case.codes.to(dev)
+    idx_parts, sc_parts = [], []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        planes = F.pack_planes(codes[:, lo:hi].contiguous())
+        i, s = F.scan_topk(planes, case.qmin.to(dev), case.qscale.to(dev), q, alloc, k, hi - lo)
+        idx_parts.append(i)
+        sc_parts.append(s)
+    mi, ms = F.merge_topk(torch.stack(idx_parts), torch.stack(sc_parts), list(cuts[:-1]), k)
+    torch.cuda.synchronize()
+    cn = case_np(case)
+    want = oracle.allocate_heads(cn[3], _np(case.sigma), 92)
+    for h in range(case.h_q):
+        ref = oracle_head(cn, h, want[h])
+        check_topk(_np(mi)[h], _np(ms)[h], ref, k, what="shards %s head %d" % (cuts, h),
+                   **_tol(0, cn[3][h], cn[1][h // 4], cn[2][h // 4], want[h]))
+
+
+def test_merge_topk_hand_lists():
+    """Hand-made partial lists: equal scores go to the lower global index,
+    padding is skipped, and fewer entries than k leave -1 / -inf."""
+    dev = torch.device("cuda")
+    idx = torch.tensor([[[2, 0, -1]], [[1, 0, -1]]], dtype=torch.int32, device=dev)
+    sc = torch.tensor([[[5.0, 3.0, -np.inf]], [[5.0, 4.0, -np.inf]]], dtype=torch.float32,
+                      device=dev)
+    mi, ms = F.merge_topk(idx, sc, [0, 10], 5)
+    torch.cuda.synchronize()
+    assert _np(mi)[0].tolist() == [2, 11, 10, 0, -1]
+    assert _np(ms)[0][:4].tolist() == [5.0, 5.0, 4.0, 3.0] and np.isneginf(_np(ms)[0][4])

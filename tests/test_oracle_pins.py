@@ -252,7 +252,7 @@ def _attention_loops(q, k_rows, v_rows, idx, scale):
     G = h_q // len(k_rows)
     out, lse = [], []
     for h in range(h_q):
-        rows = [int(i) for i in idx[h] if i >= 0]
+        rows = [int(i) for i in idx[h] if 0 <= i < len(k_rows[0])]
         if not rows:
             out.append([0.0] * d)
             lse.append(-math.inf)
@@ -307,6 +307,16 @@ def test_sparse_attention_pins():
     op, lp = oracle.sparse_attention(q, K, V, perm, scale)
     np.testing.assert_allclose(op, o, rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(lp[:3], lse[:3], rtol=1e-12)
+    # entries at or past n select nothing, like the -1 padding
+    far = idx.copy()
+    far[1, 4] = n
+    far[1, 5] = n + 7
+    far[3, :2] = [2 * n, n]
+    of, lf = oracle.sparse_attention(q, K, V, far, scale)
+    bf, blf = _attention_loops(q, K, V, far, scale)
+    np.testing.assert_allclose(of, o, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(of, bf, rtol=1e-12, atol=1e-12)
+    assert np.isneginf(lf[3]) and np.isneginf(blf[3])
 
 
 def test_hand_example_scores_and_topk(golden):

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import synthkv
-from parity import check_scores_at, score_scale
+from parity import check_scores_at
 
 pytestmark = pytest.mark.gpu
 
@@ -45,6 +45,7 @@ def test_noalloc_matches_workspace_entry_point(F):
     planes, qmin, qscale, q, alloc = _inputs(F, case, 92)
     ref_idx, ref_sc = F.scan_topk(planes, qmin, qscale, q, alloc, k, case.n)
     torch.cuda.synchronize()
+    ref_rep = F.read_report()
     ref_idx, ref_sc = ref_idx.cpu().numpy(), ref_sc.cpu().numpy()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     for call in range(2):
@@ -56,10 +57,14 @@ def test_noalloc_matches_workspace_entry_point(F):
         torch.cuda.synchronize()
         got_i, got_s = idx.cpu().numpy(), sc.cpu().numpy()
         np.testing.assert_array_equal(got_i, ref_idx, err_msg="call %d" % call)
+        # the status block in the scratch: the same report as the workspace's
+        rep = F.ScanReport()
+        st = L.fathom_scan_read_report_noalloc(ctypes.byref(rep), stream)
+        assert st == F.OK, L.fathom_last_error()
+        assert rep.union_planes == ref_rep.union_planes, "call %d" % call
+        assert rep.device_faults == 0 and rep.fallback_heads == ref_rep.fallback_heads
         for h in range(8):
-            g = h // 4
-            scale = score_scale(case.q.numpy()[h], case.qmin.numpy()[g], case.qscale.numpy()[g])
-            check_scores_at(got_s[h], ref_sc[h], scale, "call %d head %d" % (call, h))
+            check_scores_at(got_s[h], ref_sc[h], 0.0, "call %d head %d" % (call, h))
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(F):
