@@ -128,6 +128,21 @@ struct ScanParams {
   cudaEvent_t prof_end;
 };
 
+// Device bounds checks of the checked build (compiled with
+// -DFATHOM_DEVICE_CHECKS into libfathom_checked.so).  In_bounds(ok, st) is
+// true in the normal build, where the index arithmetic is trusted; in the
+// checked build an index that fails its bound is counted in the workspace
+// status (device_faults, read by fathom_scan_read_report) and the caller
+// skips the access.
+#ifdef FATHOM_DEVICE_CHECKS
+__device__ __forceinline__ bool in_bounds(bool ok, WsStatus *st) {
+  if (!ok) atomicAdd(&st->device_faults, 1u);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, WsStatus *) { return true; }
+#endif
+
 __device__ __forceinline__ const fathom_session &session_of(const ScanParams &p, int s) {
   return p.batched ? p.sessions[s] : p.one;
 }

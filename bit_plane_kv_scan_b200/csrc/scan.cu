@@ -441,8 +441,9 @@ __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
         gw = (int64_t)L.ti * kTileWords + q * 4;
         ok = gw < L.W;
       }
+      ok = ok && in_bounds(rows[slot] < 4 * p.d && gw >= 0 && gw + 4 <= L.W, p.status);
       cp_async16(dst_base + slot * kTileWords + q * 4,
-                 ok ? (const void *)(row + gw) : (const void *)row, ok ? 16u : 0u);
+                 ok ? (const void *)(row + gw) : (const void *)gbase, ok ? 16u : 0u);
     }
   };
 
@@ -499,6 +500,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) scan_kernel(ScanParams p) {
       if (sj >= sampled_sectors(L.n)) return;
       const int64_t tok0 = (sj * kSampleStride * kSectorWords + (word & 7)) * 32;
       const int64_t slot0 = sj * 256 + (word & 7) * 32;
+      if (!in_bounds(slot0 + 32 <= p.m_max && head0 + G <= (int64_t)p.S * p.h_q, p.status)) return;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         uint32_t *dst = p.sample + (head0 + h) * p.m_max + slot0;
@@ -823,7 +825,8 @@ __global__ void __launch_bounds__(1024) threshold_kernel(ScanParams p) {
     if (threadIdx.x == 0) p.tau[h] = 0u;
     return;
   }
-  const int m = (int)(sampled_sectors(n) * 256);
+  int m = (int)(sampled_sectors(n) * 256);
+  if (!in_bounds(m <= p.m_max, p.status)) m = (int)p.m_max;
   const uint32_t *keys = p.sample + h * p.m_max;
   const bool inreg = m <= kThrKeys * (int)blockDim.x;
   // element (j, e) of a thread: key 4 (j blockDim + tid) + e
@@ -970,7 +973,10 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
         sc = fmaf(s_qs[c], (float)y, sc);
       }
       const unsigned long long v = composite(sc, (uint32_t)i);
-      if (v > theta) buf[atomicAdd(&s_nbuf, 1ull)] = v;
+      if (v > theta) {
+        const unsigned long long at = atomicAdd(&s_nbuf, 1ull);
+        if (in_bounds((int64_t)at < p.cap, p.status)) buf[at] = v;
+      }
     }
     __syncthreads();
     const int64_t nb = (int64_t)s_nbuf;

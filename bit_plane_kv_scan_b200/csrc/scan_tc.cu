@@ -34,33 +34,37 @@
 // (8 M-blocks x N = 16 columns) and four A slots of one K-step each (8
 // M-blocks x 8 columns: 32 planes of u8).
 //
-// Warp roles (one 544-thread CTA per SM, persistent over a contiguous run of
+// Warp roles (one 672-thread CTA per SM, persistent over a contiguous run of
 // tiles).  Each hand-over moves one K-step (4 KB of plane words, 1024 keys x
 // 32 planes): the per-hand-over work of every role (waits, barrier and
 // address arithmetic) is paid once per 4 KB.
-//  * load warps 0-3: warps 2w and 2w + 1 load the K-steps u = w (mod 2).
-//    Thread (plane quad i, word quad m) fetches words 4m..4m+3 of four plane
-//    rows with 16-byte loads (a row's 128 bytes come from 8 threads), three
-//    K-steps ahead in registers, transposes the bytes into T and stores them
-//    in an eight-stage shared-memory ring, where a build warp reads its T
-//    values without bank conflicts;
-//  * build warps 4-11: warp (quarter q, parity) turns the T values of the
+//  * epilogue warps 0-7: warp (quarter q, half hh) reads M-blocks 4hh..4hh+3
+//    of the lanes of quarter q of a finished tile (tcgen05.ld) and tests,
+//    writes or samples those keys.  A key that may clear a head's threshold
+//    is staged in shared memory as its exact integer parts (U, L, index); at
+//    the end of a run the staged keys are scored in fp64, tested exactly and
+//    written to the workspace with one global atomic per warp and head;
+//  * build warps 8-15: warp (quarter q, parity) turns the T values of the
 //    K-steps of its parity into cells and stores them in the K-step's A slot
 //    with tcgen05.st;
-//  * epilogue warps 12-15: warp q reads the lanes of quarter q of a finished
-//    tile (tcgen05.ld) and tests, writes or samples its keys.  A key that may
-//    clear a head's threshold is staged in shared memory as its exact
-//    integer parts (U, L, index); at the end of a run the staged keys are
-//    scored in fp64, tested exactly and written to the workspace with one
-//    global atomic per warp and head;
-//  * MMA warp 16: one elected thread issues the eight MMAs (M-blocks) of every
-//    K-step and one commit (measured on B200: a thread issues an N = 16 MMA
+//  * load warps 16-19: warps 16 + 2w and 17 + 2w load the K-steps u = w
+//    (mod 2).  Thread (plane quad i, word quad m) copies words 4m..4m+3 of
+//    four plane rows with 16-byte cp.async copies (a row's 128 bytes come
+//    from 8 threads) into its own slots of a raw ring in shared memory, seven
+//    of its K-steps ahead, transposes the bytes into T and stores them in an
+//    eight-stage ring, where a build warp reads its T values without bank
+//    conflicts.  Four load warps keep about 56 KB of copies in flight per SM
+//    while holding no plane words in registers;
+//  * MMA warp 20: one elected thread issues the eight MMAs (M-blocks) and one
+//    commit of every K-step (measured on B200: a thread issues an N = 16 MMA
 //    about every 11 cycles, near the tensor pipe's rate for this shape), so
 //    every accumulator is fed in order by that thread.
 // Stages, A slots and accumulator buffers are handed over with mbarriers.
 // Every wait is bounded in time; a timeout records a device fault in the
 // workspace status, every role stops, and no further MMA is issued.
 #include <limits.h>
+
+#include <type_traits>
 
 #include "fathom_internal.cuh"
 
@@ -79,15 +83,18 @@ constexpr int kTcAColBase = kTcAccBufs * kTcAccCols;    // 256
 constexpr int kTcTmemCols = 512;
 static_assert(kTcAColBase + kTcASlots * kTcASlotCols <= kTcTmemCols, "tensor memory budget");
 
-constexpr int kTcLoadWarps = 4;                          // warps 0-3
-constexpr int kTcBuildWarp0 = kTcLoadWarps;              // warps 4-11
+constexpr int kTcEpiWarp0 = 0;                           // warps 0-7
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcBuildWarp0 = kTcEpiWarp0 + kTcEpiWarps;  // warps 8-15
 constexpr int kTcBuildPerQuarter = 2;
 constexpr int kTcBuildWarps = 4 * kTcBuildPerQuarter;
-constexpr int kTcEpiWarp0 = kTcBuildWarp0 + kTcBuildWarps;  // warps 12-15
-constexpr int kTcEpiWarps = 4;
-constexpr int kTcMmaWarp = kTcEpiWarp0 + kTcEpiWarps;    // warp 16
-constexpr int kTcWarps = kTcMmaWarp + 1;
-constexpr int kTcThreads = 32 * kTcWarps;                // 544
+constexpr int kTcLoadWarp0 = kTcBuildWarp0 + kTcBuildWarps;  // warps 16-19
+constexpr int kTcLoadWarps = 4;
+constexpr int kTcLoadPairs = kTcLoadWarps / 2;  // pair w loads the K-steps u = w (mod 2)
+constexpr int kTcMmaWarp0 = kTcLoadWarp0 + kTcLoadWarps;  // warp 20
+constexpr int kTcMmaWarps = 1;
+constexpr int kTcWarps = kTcMmaWarp0 + kTcMmaWarps;
+constexpr int kTcThreads = 32 * kTcWarps;                // 672
 static_assert(kTcBuildWarp0 % 4 == 0 && kTcEpiWarp0 % 4 == 0,
               "a warp reaches the tensor-memory lanes of quarter warp % 4");
 
@@ -96,7 +103,11 @@ constexpr int kTcStages = 8;       // shared-memory ring of K-steps
 // of a load warp's quarter warp (one plane quad, eight word quads) and the
 // word loads of a build warp both cover 32 consecutive words.
 constexpr int kTcStageWords = 8 * 4 * kTcTileWords;
-constexpr int kTcRing = 3;         // K-steps a load thread holds in registers
+// K-steps each load thread keeps in flight: 16-byte cp.async copies into a
+// ring of raw plane words in shared memory (its own four rows of each
+// K-step, so the ring needs no barrier); the registers hold none of it.
+constexpr int kTcRawDepth = 8;
+constexpr int kTcRawWords = kTcKStep * kTcTileWords;  // one K-step: 32 rows x 32 words
 constexpr int kTcCandCap = 1024;   // candidates per head staged in shared memory
 constexpr int kTcSampleSectorsPerTile = kTcTileWords / kSectorWords;  // 4
 
@@ -150,13 +161,15 @@ int tc_plan_bytes(int d) { return tc_plan_layout(d).bytes; }
 
 // Shared memory of the scan kernel, in bytes from the (128-byte aligned) base.
 struct TcSmem {
-  int stage, plan, rows, cand, tprefix, bytes;
+  int stage, raw, plan, rows, cand, tprefix, bytes;
 };
 __host__ __device__ inline TcSmem tc_smem_layout(int d, int S) {
   TcSmem m;
   int o = 0;
   m.stage = o;
   o += kTcStages * kTcStageWords * 4;
+  m.raw = o;
+  o += kTcLoadPairs * kTcRawDepth * kTcRawWords * 4;
   m.plan = o;  // 128-byte aligned (B blocks are read by the MMAs)
   o += (tc_plan_layout(d).bytes + 127) & ~127;
   m.rows = o;  // uint32 row index of every union-plane slot
@@ -238,6 +251,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_try(bar, parity)) return true;
     if (clock64() - t0 > (1ll << 31)) return false;
   }
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void tc_cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tc_cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+// Waits until at most N of this thread's committed copy groups are pending.
+template <int N>
+__device__ __forceinline__ void tc_cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void named_sync(int id, int count) {
@@ -579,7 +607,9 @@ __device__ __forceinline__ float tc_record_score(const TcPlanHeader *hdr, int h,
   return tc_score(U, L, hdr->D[h] * tc_pow2_neg(e), hdr->K[h]);
 }
 
-template <int G, int MODE>
+// DEBUG (filtering pass only): also write every score to p.debug_scores; a
+// separate instance, so that the scan's hot loop carries none of it.
+template <int G, int MODE, bool DEBUG>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   // the prologue below (tile space, tensor memory, barriers) reads only the
   // call's inputs, so it overlaps the previous kernel; the plans, thresholds
@@ -595,6 +625,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   const TcPlanLayout PL = tc_plan_layout(d);
   const TcSmem SM = tc_smem_layout(d, p.S);
   uint32_t *sStage = reinterpret_cast<uint32_t *>(smem + SM.stage);
+  uint32_t *sRaw = reinterpret_cast<uint32_t *>(smem + SM.raw);
   unsigned char *sPlan = smem + SM.plan;
   uint32_t *sRow = reinterpret_cast<uint32_t *>(smem + SM.rows);
   int4 *sRec = reinterpret_cast<int4 *>(smem + SM.cand);
@@ -676,18 +707,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   }
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(stage_full(s), 2);   // the two load warps of the K-step
+      mbar_init(stage_full(s), 2);   // the pair of load warps of the K-step
       mbar_init(stage_empty(s), 4);  // the four quarter build warps
     }
     for (int s = 0; s < kTcASlots; ++s) {
       mbar_init(a_full(s), 4);   // the four quarter build warps
-      mbar_init(a_empty(s), 1);  // the MMA warp's commit
+      mbar_init(a_empty(s), 1);  // the MMA thread's commit
     }
     for (int b = 0; b < kTcAccBufs; ++b) {
-      mbar_init(acc_full(b), 1);  // the MMA warp's commit at a tile's end
-      mbar_init(acc_empty(b), kTcEpiWarps);
+      mbar_init(acc_full(b), 1);  // the MMA thread's commit at a tile's end
+      mbar_init(acc_empty(b), kTcEpiWarps);  // every epilogue warp
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(drain_bar, kTcMmaWarps);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     s_fault = 0;
   }
@@ -763,14 +794,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     const int64_t head0 = (int64_t)L0.s * p.h_q + L0.g * G;
     const int nkst = ntiles * nks;  // K-steps of the run, tile by tile
 
-    if (warp < kTcLoadWarps) {
+    if (warp >= kTcLoadWarp0 && warp < kTcMmaWarp0) {
       // --------------------------------------------------------------- load --
-      // Warps 2w and 2w + 1 load the K-steps u = w (mod 2); thread (plane quad
-      // qi, word quad m) loads words 4m..4m+3 of rows 4qi..4qi+3.
-      const int t64 = ((warp & 1) << 5) | lane;
+      // Each pair of load warps loads every other K-step; thread (plane quad
+      // qi, word quad m) copies words 4m..4m+3 of rows 4qi..4qi+3 into its
+      // slots of the pair's raw ring, kTcRawDepth - 1 of its K-steps ahead,
+      // then transposes them.
+      const int t64 = (((warp - kTcLoadWarp0) & 1) << 5) | lane;
       const int qi = t64 >> 3;
       const int m = t64 & 7;
-      const int wpar = warp >> 1;
+      const int wpar = (warp - kTcLoadWarp0) >> 1;  // this pair loads the K-steps u = wpar (mod 2)
+      const int vfirst = (int)((uint32_t)(wpar + 2 - (int)(u0 & 1u)) & 1u);
       const uint32_t *gbase = L0.planes + (int64_t)L0.g * d * 4 * L0.W;
       const int64_t nsamp = MODE == kModeSample ? sampled_sectors(L0.n) : 0;
       const int64_t wlast = L0.W - 4;  // words past the data hold keys the epilogue drops
@@ -785,106 +819,117 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
         }
         return gw < wlast ? gw : wlast;
       };
-      const int v0 = (int)((uint32_t)(wpar + 2 - (int)(u0 & 1u)) & 1u);
-      int lv = v0, ltl = v0 / nks, lk = v0 - (v0 / nks) * nks;  // cursor of the next load
-      auto load_next = [&](uint4 (&r)[4]) {
-        if (lv < nkst && kTcKStep * lk + 4 * qi < P) {
+      // raw ring slot of this thread's row j for K-step v
+      auto raw_at = [&](int v, int j) -> uint32_t * {
+        return sRaw + ((v >> 1) % kTcRawDepth) * kTcRawWords + (4 * qi + j) * kTcTileWords + 4 * m +
+               wpar * (kTcRawDepth * kTcRawWords);
+      };
+      int ltl = vfirst / nks, lk = vfirst - (vfirst / nks) * nks;  // cursor of the next K-step to copy
+      auto copy_next = [&](int lv) {
+        if (lv < nkst) {
           const int64_t gw = quad_word(ti0 + ltl);
           const uint4 o = *reinterpret_cast<const uint4 *>(sRow + lk * kTcKStep + 4 * qi);
-          r[0] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.x * L0.W + gw));
-          r[1] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.y * L0.W + gw));
-          r[2] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.z * L0.W + gw));
-          r[3] = __ldcg(reinterpret_cast<const uint4 *>(gbase + (int64_t)o.w * L0.W + gw));
-        } else {
+          const bool real = kTcKStep * lk + 4 * qi < P &&
+                            in_bounds(max(max(o.x, o.y), max(o.z, o.w)) < (uint32_t)(4 * d) &&
+                                          gw >= 0 && gw + 4 <= L0.W,
+                                      p.status);
+          const uint32_t rows[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) r[k] = make_uint4(0u, 0u, 0u, 0u);
+          for (int j = 0; j < 4; ++j)
+            tc_cp_async16(tc_smem_u32(raw_at(lv, j)),
+                          real ? (const void *)(gbase + (int64_t)rows[j] * L0.W + gw)
+                               : (const void *)gbase,
+                          real ? 16u : 0u);
+          lk += 2;
+          while (lk >= nks) { lk -= nks; ++ltl; }
         }
-        lv += 2;
-        lk += 2;
-        while (lk >= nks) { lk -= nks; ++ltl; }
+        tc_cp_async_commit();  // one group per K-step (empty past the end)
       };
-      uint4 ring[kTcRing][4];
+#pragma unroll 1
+      for (int j = 0; j < kTcRawDepth - 1; ++j) copy_next(vfirst + 2 * j);
+      for (int v = vfirst; v < nkst; v += 2) {
+        copy_next(v + 2 * (kTcRawDepth - 1));
+        tc_cp_async_wait<kTcRawDepth - 1>();  // K-step v's copies have landed
+        uint4 x[4];
 #pragma unroll
-      for (int j = 0; j < kTcRing; ++j) load_next(ring[j]);
-      bool alive = true;
-      for (int vb = v0; vb < nkst && alive; vb += 2 * kTcRing) {
+        for (int j = 0; j < 4; ++j) x[j] = *reinterpret_cast<const uint4 *>(raw_at(v, j));
+        const uint32_t u = u0 + (uint32_t)v;
+        const int s = (int)(u % kTcStages);
+        if (u >= (uint32_t)kTcStages && !warp_wait(stage_empty(s), ((u / kTcStages) - 1) & 1))
+          break;
+        uint32_t *dst = sStage + s * kTcStageWords + qi * (4 * kTcTileWords) + 4 * m;
+        uint32_t Tq[4][4];  // [quarter][word]
 #pragma unroll
-        for (int jj = 0; jj < kTcRing; ++jj) {
-          const int vv = vb + 2 * jj;
-          if (vv >= nkst) break;
-          const uint32_t u = u0 + (uint32_t)vv;
-          const int s = (int)(u % kTcStages);
-          if (u >= (uint32_t)kTcStages && !warp_wait(stage_empty(s), ((u / kTcStages) - 1) & 1)) {
-            alive = false;
-            break;
-          }
-          uint32_t *dst = sStage + s * kTcStageWords + qi * (4 * kTcTileWords) + 4 * m;
-          uint32_t Tq[4][4];  // [quarter][word]
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t x0 = (&ring[jj][0].x)[w], x1 = (&ring[jj][1].x)[w];
-            const uint32_t x2 = (&ring[jj][2].x)[w], x3 = (&ring[jj][3].x)[w];
-            const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
-            const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
-            Tq[0][w] = __byte_perm(a_lo, b_lo, 0x5410);
-            Tq[1][w] = __byte_perm(a_lo, b_lo, 0x7632);
-            Tq[2][w] = __byte_perm(a_hi, b_hi, 0x5410);
-            Tq[3][w] = __byte_perm(a_hi, b_hi, 0x7632);
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4 *>(dst + q * kTcTileWords) =
-                make_uint4(Tq[q][0], Tq[q][1], Tq[q][2], Tq[q][3]);
-          warp_arrive(stage_full(s));
-          load_next(ring[jj]);
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t x0 = (&x[0].x)[w], x1 = (&x[1].x)[w];
+          const uint32_t x2 = (&x[2].x)[w], x3 = (&x[3].x)[w];
+          const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
+          const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
+          Tq[0][w] = __byte_perm(a_lo, b_lo, 0x5410);
+          Tq[1][w] = __byte_perm(a_lo, b_lo, 0x7632);
+          Tq[2][w] = __byte_perm(a_hi, b_hi, 0x5410);
+          Tq[3][w] = __byte_perm(a_hi, b_hi, 0x7632);
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4 *>(dst + q * kTcTileWords) =
+              make_uint4(Tq[q][0], Tq[q][1], Tq[q][2], Tq[q][3]);
+        warp_arrive(stage_full(s));
       }
-    } else if (warp < kTcEpiWarp0) {
+      tc_cp_async_wait<0>();  // no copy into the ring outlives the run
+    } else if (warp >= kTcBuildWarp0 && warp < kTcLoadWarp0) {
       // ------------------------------------------------------------ build --
       // Warp (quarter q, parity) builds the K-steps u = parity (mod 2): the
       // cells of M-blocks 0-7 for its lanes, the 64 columns of the K-step's
       // slot, stored 32 columns (four M-blocks) at a time.
       const int par = (warp - kTcBuildWarp0) >> 2;
-      for (int v = (int)((uint32_t)(par + 2 - (int)(u0 & 1u)) & 1u); v < nkst; v += 2) {
-        const uint32_t u = u0 + (uint32_t)v;
-        const int s = (int)(u % kTcStages);
-        if (!warp_wait(stage_full(s), (u / kTcStages) & 1)) break;
-        const uint32_t *src = sStage + s * kTcStageWords + quarter * kTcTileWords + lane;
-        uint32_t T[8];
+      // the cell form (0/2^r or 0/1) is fixed for the run: one loop each
+      auto build_run = [&](auto big_c) {
+        constexpr bool kBig = decltype(big_c)::value;
+        for (int v = (int)((uint32_t)(par + kTcBuildPerQuarter - (int)(u0 % kTcBuildPerQuarter)) %
+                           kTcBuildPerQuarter);
+             v < nkst; v += kTcBuildPerQuarter) {
+          const uint32_t u = u0 + (uint32_t)v;
+          const int s = (int)(u % kTcStages);
+          if (!warp_wait(stage_full(s), (u / kTcStages) & 1)) break;
+          const uint32_t *src = sStage + s * kTcStageWords + quarter * kTcTileWords + lane;
+          uint32_t T[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) T[i] = src[i * 4 * kTcTileWords];
-        warp_arrive(stage_empty(s));
-        const int slot = (int)(u % kTcASlots);
-        // the slot was last read by the MMAs of K-step u - kTcASlots
-        if (u >= (uint32_t)kTcASlots && !warp_wait(a_empty(slot), ((u / kTcASlots) - 1) & 1))
-          break;
-        const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + slot * kTcASlotCols);
+          for (int i = 0; i < 8; ++i) T[i] = src[i * 4 * kTcTileWords];
+          warp_arrive(stage_empty(s));
+          const int slot = (int)(u % kTcASlots);
+          // the slot was last read by the MMAs of K-step u - kTcASlots
+          if (u >= (uint32_t)kTcASlots && !warp_wait(a_empty(slot), ((u / kTcASlots) - 1) & 1))
+            break;
+          const uint32_t acol = tmem + lane_base + (uint32_t)(kTcAColBase + slot * kTcASlotCols);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t cell[32];
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t cell[32];
 #pragma unroll
-          for (int rr = 0; rr < 4; ++rr) {
-            const int r = 4 * hf + rr;
-            if (!big) {
-              const uint32_t msk = 0x01010101u << r;
+            for (int rr = 0; rr < 4; ++rr) {
+              const int r = 4 * hf + rr;
 #pragma unroll
-              for (int i = 0; i < 8; ++i) cell[8 * rr + i] = T[i] & msk;
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) cell[8 * rr + i] = (T[i] >> r) & 0x01010101u;
+              for (int i = 0; i < 8; ++i)
+                cell[8 * rr + i] = kBig ? (T[i] >> r) & 0x01010101u : T[i] & (0x01010101u << r);
             }
+            tc_st32(acol + (uint32_t)(32 * hf), cell);
           }
-          tc_st32(acol + (uint32_t)(32 * hf), cell);
+          tc_wait_st();
+          tc_fence_before();
+          warp_arrive(a_full(slot));
         }
-        tc_wait_st();
-        tc_fence_before();
-        warp_arrive(a_full(slot));
-      }
-    } else if (warp < kTcMmaWarp) {
+      };
+      if (big)
+        build_run(std::true_type());
+      else
+        build_run(std::false_type());
+    } else if (warp < kTcEpiWarp0 + kTcEpiWarps) {
       // ---------------------------------------------------------- epilogue --
-      // Lane (q, l) holds keys 32 l + 8 q + r of each tile (M-block r);
-      // accumulator columns 16 r + 4 h + m.  Read 32 columns (two M-blocks)
-      // at a time.
+      // Warp (quarter q, half hh) holds, in lane l, keys 32 l + 8 q + r of
+      // each tile for M-blocks r = 4 hh .. 4 hh + 3: accumulator columns
+      // 16 r + 4 h + m, 64 columns read with two loads and one wait.
+      const int hh = (warp - kTcEpiWarp0) >> 2;
+      const int r0 = 4 * hh;
       const int nkeys = (int)L0.n;
       const int nsamp = MODE == kModeSample ? (int)sampled_sectors(L0.n) : 0;
       for (int tl = 0; tl < ntiles; ++tl) {
@@ -892,87 +937,91 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
         const int ab = (int)(tt % kTcAccBufs);
         if (!warp_wait(acc_full(ab), (tt / kTcAccBufs) & 1)) break;
         tc_fence_after();
-        const uint32_t abase = tmem + lane_base + (uint32_t)(ab * kTcAccCols);
+        const uint32_t abase = tmem + lane_base + (uint32_t)(ab * kTcAccCols + 16 * r0);
+        uint32_t a0[32], a1[32];
+        tc_ld32(abase, a0);
+        tc_ld32(abase + 32u, a1);
+        tc_wait_ld();
+        // column i of the warp's 64 (indexes are compile-time after unrolling)
+        auto A = [&](int i) -> uint32_t { return i < 32 ? a0[i] : a1[i - 32]; };
+        // every column this warp needs is in registers: the MMAs may refill it
+        tc_fence_before();
+        warp_arrive(acc_empty(ab));
         const int ti = ti0 + tl;
-#pragma unroll 1
-        for (int c = 0; c < kTcMBlocks / 2; ++c) {
-          uint32_t a[32];
-          tc_ld32(abase + (uint32_t)(32 * c), a);
-          tc_wait_ld();
-          if (c == kTcMBlocks / 2 - 1) {
-            // every column of the buffer is in registers: the MMAs may refill it
-            tc_fence_before();
-            warp_arrive(acc_empty(ab));
-          }
-          if (MODE == kModeSample) {
-            const int sj = ti * kTcSampleSectorsPerTile + (lane >> 3);
-            const int wis = lane & 7;
-            const int tok0 = (sj * kSampleStride * kSectorWords + wis) * 32 + 8 * quarter + 2 * c;
-            const int slot0 = sj * 256 + wis * 32 + 8 * quarter + 2 * c;
-            if (sj < nsamp) {
-#pragma unroll
-              for (int h = 0; h < G; ++h) {
-                uint32_t kv[2];
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                  const uint32_t *x = a + 16 * rr + 4 * h;
-                  const int U = (int)(x[3] << 8) + (int)x[2];
-                  const int L = (int)(x[1] << 8) + (int)x[0];
-                  const float De = sHdr->D[h] * tc_pow2_neg(big ? 0 : 2 * c + rr);
-                  kv[rr] = tok0 + rr < nkeys ? float_key(tc_score(U, L, De, sHdr->K[h])) : 0u;
-                }
-                *reinterpret_cast<uint2 *>(p.sample + (head0 + h) * p.m_max + slot0) =
-                    make_uint2(kv[0], kv[1]);
-              }
-            }
-          } else {
-            const int tok0 = (ti * kTcTileWords + lane) * 32 + 8 * quarter + 2 * c;
-            if (p.debug_scores) {
-#pragma unroll
-              for (int h = 0; h < G; ++h)
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                  const uint32_t *x = a + 16 * rr + 4 * h;
-                  const int U = (int)(x[3] << 8) + (int)x[2];
-                  const int L = (int)(x[1] << 8) + (int)x[0];
-                  const float De = sHdr->D[h] * tc_pow2_neg(big ? 0 : 2 * c + rr);
-                  if (tok0 + rr < nkeys)
-                    p.debug_scores[(head0 + h) * (int64_t)nkeys + tok0 + rr] =
-                        tc_score(U, L, De, sHdr->K[h]);
-                }
-            }
-            // bit 2 h + rr: key tok0 + rr may clear head h's threshold
-            uint32_t cm = 0u;
+        if (MODE == kModeSample) {
+          const int sj = ti * kTcSampleSectorsPerTile + (lane >> 3);
+          const int wis = lane & 7;
+          const int tok0 = (sj * kSampleStride * kSectorWords + wis) * 32 + 8 * quarter + r0;
+          const int slot0 = sj * 256 + wis * 32 + 8 * quarter + r0;
+          if (sj < nsamp &&
+              in_bounds(slot0 + 4 <= p.m_max && head0 + G <= (int64_t)p.S * p.h_q, p.status)) {
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-              const int2 tu = *reinterpret_cast<const int2 *>(&s_TU[h][2 * c]);
-              cm |= ((int)(a[4 * h + 3] << 8) + (int)a[4 * h + 2] >= tu.x ? 1u : 0u) << (2 * h);
-              cm |= ((int)(a[16 + 4 * h + 3] << 8) + (int)a[16 + 4 * h + 2] >= tu.y ? 1u : 0u)
-                    << (2 * h + 1);
+              uint32_t kv[4];
+#pragma unroll
+              for (int rr = 0; rr < 4; ++rr) {
+                const int c = 16 * rr + 4 * h;
+                const int U = (int)(A(c + 3) << 8) + (int)A(c + 2);
+                const int L = (int)(A(c + 1) << 8) + (int)A(c);
+                const float De = sHdr->D[h] * tc_pow2_neg(big ? 0 : r0 + rr);
+                kv[rr] = tok0 + rr < nkeys ? float_key(tc_score(U, L, De, sHdr->K[h])) : 0u;
+              }
+              *reinterpret_cast<uint4 *>(p.sample + (head0 + h) * p.m_max + slot0) =
+                  make_uint4(kv[0], kv[1], kv[2], kv[3]);
             }
-            if (tok0 + 1 >= nkeys) cm &= tok0 < nkeys ? 0x55555555u : 0u;  // keys past n
-            if (__any_sync(0xffffffffu, cm != 0u)) {
+          }
+        } else {
+          const int tok0 = (ti * kTcTileWords + lane) * 32 + 8 * quarter + r0;
+          if (DEBUG) {
 #pragma unroll
-              for (int h = 0; h < G; ++h) {
+            for (int h = 0; h < G; ++h)
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                  if ((cm >> (2 * h + rr)) & 1u) {
-                    const uint32_t *x = a + 16 * rr + 4 * h;
-                    const int U = (int)(x[3] << 8) + (int)x[2];
-                    const int L = (int)(x[1] << 8) + (int)x[0];
-                    const uint32_t tok = (uint32_t)(tok0 + rr);
-                    const unsigned pos = atomicAdd(&s_ccount[h], 1u);
-                    if (pos < (unsigned)kTcCandCap) {
-                      sRec[h * kTcCandCap + pos] = make_int4(U, L, (int)tok, 0);
-                    } else {
-                      // shared staging full: score now, straight to the workspace
-                      const float sc = tc_record_score(sHdr, h, U, L, tok);
-                      if (sc >= s_tau[h]) {
-                        const unsigned gp = atomicAdd(&p.counts[head0 + h], 1u);
-                        if ((int64_t)gp < p.cap) p.cand[(head0 + h) * p.cap + gp] = composite(sc, tok);
-                      }
-                    }
-                  }
+              for (int rr = 0; rr < 4; ++rr) {
+                const int c = 16 * rr + 4 * h;
+                const int U = (int)(A(c + 3) << 8) + (int)A(c + 2);
+                const int L = (int)(A(c + 1) << 8) + (int)A(c);
+                const float De = sHdr->D[h] * tc_pow2_neg(big ? 0 : r0 + rr);
+                if (tok0 + rr < nkeys)
+                  p.debug_scores[(head0 + h) * (int64_t)nkeys + tok0 + rr] =
+                      tc_score(U, L, De, sHdr->K[h]);
+              }
+          }
+          // bit 4 h + rr: key tok0 + rr may clear head h's threshold
+          uint32_t cm = 0u;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const int4 tu = *reinterpret_cast<const int4 *>(&s_TU[h][r0]);
+            cm |= ((int)(a0[4 * h + 3] << 8) + (int)a0[4 * h + 2] >= tu.x ? 1u : 0u) << (4 * h);
+            cm |= ((int)(a0[16 + 4 * h + 3] << 8) + (int)a0[16 + 4 * h + 2] >= tu.y ? 1u : 0u)
+                  << (4 * h + 1);
+            cm |= ((int)(a1[4 * h + 3] << 8) + (int)a1[4 * h + 2] >= tu.z ? 1u : 0u)
+                  << (4 * h + 2);
+            cm |= ((int)(a1[16 + 4 * h + 3] << 8) + (int)a1[16 + 4 * h + 2] >= tu.w ? 1u : 0u)
+                  << (4 * h + 3);
+          }
+          // keys past n (only in a segment's last tile)
+          if (tok0 + 3 >= nkeys) {
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr)
+              if (tok0 + rr >= nkeys) cm &= ~(0x1111u << rr);
+          }
+          // stage each key that passed (rare: one in a few hundred) as its exact
+          // parts; a head whose staging is full is answered by the exact
+          // fallback instead
+          if (__any_sync(0xffffffffu, cm != 0u)) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+#pragma unroll
+              for (int rr = 0; rr < 4; ++rr) {
+                if ((cm >> (4 * h + rr)) & 1u) {
+                  const int c = 16 * rr + 4 * h;
+                  const unsigned pos = atomicAdd(&s_ccount[h], 1u);
+                  if (pos < (unsigned)kTcCandCap &&
+                      in_bounds(tok0 + rr < nkeys && h * kTcCandCap + (int)pos < 4 * kTcCandCap,
+                                p.status))
+                    sRec[h * kTcCandCap + pos] =
+                        make_int4((int)(A(c + 3) << 8) + (int)A(c + 2),
+                                  (int)(A(c + 1) << 8) + (int)A(c), tok0 + rr, 0);
                 }
               }
             }
@@ -985,7 +1034,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
         // Epilogue warp h takes head h.
         named_sync(1, 32 * kTcEpiWarps);
         const int h = warp - kTcEpiWarp0;
-        if (h < G) {
+        if (h < G && s_ccount[h] > (unsigned)kTcCandCap) {
+          // more keys passed than the staging holds: the merge answers this
+          // head exactly (a count above the buffer's capacity sends it to the
+          // fallback)
+          if (lane == 0) {
+            atomicMax(&p.counts[head0 + h], 0x7fffffffu);
+            s_ccount[h] = 0u;
+          }
+        } else if (h < G) {
           const unsigned nc = min(s_ccount[h], (unsigned)kTcCandCap);
           unsigned long long *dst = p.cand + (head0 + h) * p.cap;
           const float tau = s_tau[h];
@@ -1005,18 +1062,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
             base = __shfl_sync(0xffffffffu, base, 0);
             if (keep) {
               const int64_t pos = (int64_t)base + __popc(bal & ((1u << lane) - 1u));
-              if (pos < p.cap) dst[pos] = cv;
+              if (pos < p.cap && in_bounds(head0 + h < (int64_t)p.S * p.h_q, p.status)) dst[pos] = cv;
             }
           }
           __syncwarp();
           if (lane == 0) s_ccount[h] = 0u;
         }
       }
-    } else {
+    } else if (warp == kTcMmaWarp0) {
       // -------------------------------------------------------------- MMA --
-      // One elected thread feeds every accumulator: M-block r of a K-step
-      // reads A columns 8 r of the K-step's slot into columns 16 r of the
-      // tile's buffer; one commit per K-step frees the slot.
+      // One elected thread issues every MMA, in K-step order, so each
+      // accumulator is fed in order.  M-block r of a K-step reads A columns
+      // 8 r of the K-step's slot into columns 16 r of the tile's buffer; one
+      // commit per K-step frees the slot.  (The whole warp runs the loop and
+      // waits: measured faster on B200 than a loop in lane 0 alone.)
       const uint64_t b_desc0 = tc_smem_desc(tc_smem_u32(sPlan + PL.off_b), kTcLBO, kTcSBO);
       int tl = 0, kx = 0;
       for (int v = 0; v < nkst; ++v) {
@@ -1054,11 +1113,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   }
 
   // ---- teardown ------------------------------------------------------------
-  // The MMA warp commits once more after its last MMA; when that commit has
-  // arrived every MMA is complete.  Then the slots' last commits are waited
-  // for, so that no arrival is pending when the barriers go away.
+  // Each MMA warp commits once more after its last MMA; when those commits
+  // have arrived every MMA is complete.  Then the slots' last commits are
+  // waited for, so that no arrival is pending when the barriers go away.
   __syncthreads();
-  if (warp == kTcMmaWarp) {
+  if (warp == kTcMmaWarp0) {
     if (tc_elect_one()) tc_commit(drain_bar);
     __syncwarp();
   }
@@ -1089,13 +1148,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
 
 // ------------------------------------------------------------- launchers --
 
-template <int G, int MODE>
+template <int G, int MODE, bool DEBUG>
 static cudaError_t launch_tc_gm(const ScanParams &p, int sms, cudaStream_t stream) {
   const int smem = tc_smem_bytes(p.d, p.S);
-  cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<G, MODE>,
+  cudaError_t e = cudaFuncSetAttribute(tc_scan_kernel<G, MODE, DEBUG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return launch_dependent(tc_scan_kernel<G, MODE>, dim3(sms), dim3(kTcThreads), (size_t)smem, stream, p);
+  return launch_dependent(tc_scan_kernel<G, MODE, DEBUG>, dim3(sms), dim3(kTcThreads), (size_t)smem,
+                          stream, p);
 }
 
 cudaError_t launch_tc_plan(const ScanParams &p, cudaStream_t stream) {
@@ -1105,15 +1165,21 @@ cudaError_t launch_tc_plan(const ScanParams &p, cudaStream_t stream) {
 cudaError_t launch_tc_scan(const ScanParams &p, int mode, int sms, cudaStream_t stream) {
   if (mode == kModeSample) {
     switch (p.G) {
-      case 1: return launch_tc_gm<1, kModeSample>(p, sms, stream);
-      case 2: return launch_tc_gm<2, kModeSample>(p, sms, stream);
-      case 4: return launch_tc_gm<4, kModeSample>(p, sms, stream);
+      case 1: return launch_tc_gm<1, kModeSample, false>(p, sms, stream);
+      case 2: return launch_tc_gm<2, kModeSample, false>(p, sms, stream);
+      case 4: return launch_tc_gm<4, kModeSample, false>(p, sms, stream);
+    }
+  } else if (p.debug_scores) {
+    switch (p.G) {
+      case 1: return launch_tc_gm<1, kModeFilter, true>(p, sms, stream);
+      case 2: return launch_tc_gm<2, kModeFilter, true>(p, sms, stream);
+      case 4: return launch_tc_gm<4, kModeFilter, true>(p, sms, stream);
     }
   } else {
     switch (p.G) {
-      case 1: return launch_tc_gm<1, kModeFilter>(p, sms, stream);
-      case 2: return launch_tc_gm<2, kModeFilter>(p, sms, stream);
-      case 4: return launch_tc_gm<4, kModeFilter>(p, sms, stream);
+      case 1: return launch_tc_gm<1, kModeFilter, false>(p, sms, stream);
+      case 2: return launch_tc_gm<2, kModeFilter, false>(p, sms, stream);
+      case 4: return launch_tc_gm<4, kModeFilter, false>(p, sms, stream);
     }
   }
   return cudaErrorInvalidValue;

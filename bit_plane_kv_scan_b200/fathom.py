@@ -16,7 +16,11 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfathom.so")
+# FATHOM_LIB=checked loads the checked build (device bounds checks on every
+# plane-row, sample and candidate index; a failed check is a device fault in
+# the scan report)
+LIB_PATH = os.path.join(_HERE, "libfathom_checked.so" if os.environ.get("FATHOM_LIB") == "checked"
+                        else "libfathom.so")
 
 OK = 0
 ERR_INVALID_ARGUMENT = 1
