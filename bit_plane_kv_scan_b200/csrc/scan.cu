@@ -923,7 +923,8 @@ __device__ unsigned long long block_kth(const unsigned long long *a, int64_t cnt
 }
 
 // Exact single-block answer for one head: stream all n keys, score each from
-// its allocated prefixes (fp32), keep a candidate buffer above a running
+// its allocated prefixes (accumulated in fp64 from the exact products
+// q_c s_c, rounded once to fp32), keep a candidate buffer above a running
 // k-th best, compact it when it fills.  Used when the sampled threshold
 // fails.  Returns the number of buffered candidates (= min(k, n)).
 __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned long long *buf,
@@ -934,7 +935,7 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   const int g = hl / p.G;
   const int64_t n = session_n(p, s);
   const int64_t W = plane_words(n);
-  __shared__ float s_qs[FATHOM_MAX_D];
+  __shared__ double s_qs[FATHOM_MAX_D];
   __shared__ uint8_t s_t[FATHOM_MAX_D];
   __shared__ double s_kc[32];
   __shared__ unsigned long long s_nbuf;
@@ -945,7 +946,7 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
     const float qv = load_q(se.q, p.q_bf16, (int64_t)hl * d + c);
     const float m = se.qmin[(int64_t)g * d + c], sc = se.qscale[(int64_t)g * d + c];
     s_t[c] = (uint8_t)t;
-    s_qs[c] = qv * sc;
+    s_qs[c] = (double)qv * (double)sc;  // exact
     const double cell = (double)(1 << (4 - t));
     kc += (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5));
   }
@@ -956,23 +957,23 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   __syncthreads();
   double ksum = 0.0;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) ksum += s_kc[w];
-  const float K = (float)ksum;
+  const double K = ksum;
   const uint32_t *gp = se.planes + (int64_t)g * d * 4 * W;
   unsigned long long theta = 0ull;
   const unsigned k = (unsigned)p.k;
   for (int64_t base = 0; base < n; base += blockDim.x) {
     const int64_t i = base + threadIdx.x;
     if (i < n) {
-      float sc = K;
+      double acc = K;
       for (int c = 0; c < d; ++c) {
         const int t = s_t[c];
         if (t == 0) continue;
         uint32_t y = 0;
         for (int j = 0; j < t; ++j)
           y |= ((gp[((int64_t)c * 4 + j) * W + (i >> 5)] >> (i & 31)) & 1u) << (3 - j);
-        sc = fmaf(s_qs[c], (float)y, sc);
+        acc = fma(s_qs[c], (double)y, acc);
       }
-      const unsigned long long v = composite(sc, (uint32_t)i);
+      const unsigned long long v = composite((float)acc, (uint32_t)i);
       if (v > theta) {
         const unsigned long long at = atomicAdd(&s_nbuf, 1ull);
         if (in_bounds((int64_t)at < p.cap, p.status)) buf[at] = v;

@@ -41,9 +41,11 @@
 //  * epilogue warps 0-7: warp (quarter q, half hh) reads M-blocks 4hh..4hh+3
 //    of the lanes of quarter q of a finished tile (tcgen05.ld) and tests,
 //    writes or samples those keys.  A key that may clear a head's threshold
-//    is staged in shared memory as its exact integer parts (U, L, index); at
-//    the end of a run the staged keys are scored in fp64, tested exactly and
-//    written to the workspace with one global atomic per warp and head;
+//    is staged in the warp's own shared-memory region as its exact integer
+//    parts (U, L, index); when a region might not hold another tile's keys,
+//    and at the end of a run, the warp scores its staged keys in fp64, tests
+//    them exactly and writes them to the workspace with one global atomic per
+//    32 keys (no barrier between epilogue warps);
 //  * build warps 8-15: warp (quarter q, parity) turns the T values of the
 //    K-steps of its parity into cells and stores them in the K-step's A slot
 //    with tcgen05.st;
@@ -108,7 +110,10 @@ constexpr int kTcStageWords = 8 * 4 * kTcTileWords;
 // K-step, so the ring needs no barrier); the registers hold none of it.
 constexpr int kTcRawDepth = 8;
 constexpr int kTcRawWords = kTcKStep * kTcTileWords;  // one K-step: 32 rows x 32 words
-constexpr int kTcCandCap = 1024;   // candidates per head staged in shared memory
+// Candidates staged in shared memory per epilogue warp and head.  A warp
+// adds at most 128 per head and tile (its 32 lanes x 4 M-blocks), so a region
+// holding more than kTcWarpCap - 128 is flushed before the next tile.
+constexpr int kTcWarpCap = 192;
 constexpr int kTcSampleSectorsPerTile = kTcTileWords / kSectorWords;  // 4
 
 // B for one K-step: 16 rows (head, digit) x 32 int8 K elements (planes),
@@ -174,8 +179,8 @@ __host__ __device__ inline TcSmem tc_smem_layout(int d, int S) {
   o += (tc_plan_layout(d).bytes + 127) & ~127;
   m.rows = o;  // uint32 row index of every union-plane slot
   o += 4 * 4 * d;
-  m.cand = o;  // int4 {U, L, index, 0} per staged candidate, [head][kTcCandCap]
-  o += 4 * kTcCandCap * 16;
+  m.cand = o;  // int4 {U, L, index, 0} per staged candidate, [warp][head][kTcWarpCap]
+  o += kTcEpiWarps * 4 * kTcWarpCap * 16;
   m.tprefix = o;
   o += 4 * (S + 1);
   m.bytes = o;
@@ -266,10 +271,6 @@ __device__ __forceinline__ void tc_cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void tc_cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
 }
 
 // D[tmem_d] (+)= A[tmem_a] x B[bdesc]; accumulate = 0 overwrites D.
@@ -638,7 +639,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   __shared__ uint32_t s_tmem;
   __shared__ int s_tmp[32];
   __shared__ volatile int s_fault;
-  __shared__ unsigned s_ccount[4];  // candidates staged per head in this run
+  __shared__ unsigned s_wcount[kTcEpiWarps][4];  // candidates staged per epilogue warp and head
   __shared__ float s_tau[4];
   // Integer thresholds of the run, [head][M-block]: a key whose fp32 score
   // reaches tau_h has U >= s_TU (the bound on |L| and on the score's rounding
@@ -658,19 +659,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   };
   const uint32_t drain_bar = bar0 + 8u * (uint32_t)(kBars - 1);
   // A wait that gives up records a fault; every role then leaves its loops.
-  // Every lane probes (one shared-memory word, so all see the same phase);
-  // only a phase still open sends lane 0 into the bounded wait.
+  // Every lane waits on the barrier itself (measured faster on B200 than one
+  // lane waiting and broadcasting the outcome); the warp goes on only when
+  // all of its lanes saw the phase complete.
   auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
-    if (!__all_sync(0xffffffffu, mbar_test(bar, parity))) {
-      int ok = 1;
-      if (lane == 0) {
-        if (s_fault || !mbar_wait(bar, parity)) {
-          s_fault = 1;
-          ok = 0;
-        }
+    bool ok = mbar_try(bar, parity);
+    if (!ok) {
+      const long long t0 = clock64();
+      while (!(ok = mbar_try(bar, parity))) {
+        if (s_fault || clock64() - t0 > (1ll << 31)) break;
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) return false;
+    }
+    if (!__all_sync(0xffffffffu, ok)) {
+      s_fault = 1;
+      return false;
     }
     return true;
   };
@@ -722,7 +724,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     s_fault = 0;
   }
-  if (tid < 4) s_ccount[tid] = 0u;
+  if (tid < 4 * kTcEpiWarps) (&s_wcount[0][0])[tid] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -932,6 +934,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
       const int r0 = 4 * hh;
       const int nkeys = (int)L0.n;
       const int nsamp = MODE == kModeSample ? (int)sampled_sectors(L0.n) : 0;
+      // this warp's staging: wRec[h][kTcWarpCap] records, wCnt[h] of them in use
+      int4 *wRec = sRec + (warp - kTcEpiWarp0) * (4 * kTcWarpCap);
+      unsigned *wCnt = s_wcount[warp - kTcEpiWarp0];
+      // Flush of the staged keys of every head whose region holds more than
+      // `above` of them: each is scored in fp64 and tested against tau_h
+      // exactly (its composite, or 0, written back in place), then one global
+      // atomic per head reserves the room of all its passing keys (the heads'
+      // atomics in flight together), and the composites are written there.
+      auto flush = [&](unsigned above) {
+        const unsigned lt = (1u << lane) - 1u;
+        unsigned kept = 0u;  // lane h: passing keys of head h
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+          const unsigned nc = wCnt[h];
+          if (nc <= above) continue;
+          const float tau = s_tau[h];
+          unsigned kh = 0u;
+          for (unsigned i0 = 0; i0 < nc; i0 += 32) {
+            const unsigned i = i0 + lane;
+            bool keep = false;
+            if (i < nc && in_bounds(i < (unsigned)kTcWarpCap, p.status)) {
+              int4 *slot = &wRec[h * kTcWarpCap + i];
+              const int4 rec = *slot;
+              const float sc = tc_record_score(sHdr, h, rec.x, rec.y, (uint32_t)rec.z);
+              keep = sc >= tau;
+              *reinterpret_cast<unsigned long long *>(slot) =
+                  keep ? composite(sc, (uint32_t)rec.z) : 0ull;
+            }
+            kh += (unsigned)__popc(__ballot_sync(0xffffffffu, keep));
+          }
+          if (lane == h) kept = kh;
+        }
+        unsigned base = 0u;
+        if (lane < G && kept > 0u) base = atomicAdd(&p.counts[head0 + lane], kept);
+        __syncwarp();
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+          const unsigned nc = wCnt[h];
+          if (nc <= above) continue;
+          unsigned long long *dst = p.cand + (head0 + h) * p.cap;
+          unsigned pos0 = __shfl_sync(0xffffffffu, base, h);
+          for (unsigned i0 = 0; i0 < nc; i0 += 32) {
+            const unsigned i = i0 + lane;
+            unsigned long long cv = 0ull;
+            if (i < nc && i < (unsigned)kTcWarpCap)
+              cv = *reinterpret_cast<const unsigned long long *>(&wRec[h * kTcWarpCap + i]);
+            const unsigned bal = __ballot_sync(0xffffffffu, cv != 0ull);
+            if (cv != 0ull) {
+              const int64_t pos = (int64_t)pos0 + __popc(bal & lt);
+              if (pos < p.cap && in_bounds(head0 + h < (int64_t)p.S * p.h_q, p.status)) dst[pos] = cv;
+            }
+            pos0 += (unsigned)__popc(bal);
+          }
+        }
+        __syncwarp();
+        if (lane < G && wCnt[lane] > above) wCnt[lane] = 0u;
+        __syncwarp();
+      };
       for (int tl = 0; tl < ntiles; ++tl) {
         const uint32_t tt = tt0 + (uint32_t)tl;
         const int ab = (int)(tt % kTcAccBufs);
@@ -1006,8 +1066,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
               if (tok0 + rr >= nkeys) cm &= ~(0x1111u << rr);
           }
           // stage each key that passed (rare: one in a few hundred) as its exact
-          // parts; a head whose staging is full is answered by the exact
-          // fallback instead
+          // parts in this warp's region (positions from ballots: no atomics)
           if (__any_sync(0xffffffffu, cm != 0u)) {
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -1015,59 +1074,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
               for (int rr = 0; rr < 4; ++rr) {
                 if ((cm >> (4 * h + rr)) & 1u) {
                   const int c = 16 * rr + 4 * h;
-                  const unsigned pos = atomicAdd(&s_ccount[h], 1u);
-                  if (pos < (unsigned)kTcCandCap &&
-                      in_bounds(tok0 + rr < nkeys && h * kTcCandCap + (int)pos < 4 * kTcCandCap,
-                                p.status))
-                    sRec[h * kTcCandCap + pos] =
+                  const unsigned pos = atomicAdd(&wCnt[h], 1u);
+                  if (in_bounds(pos < (unsigned)kTcWarpCap && tok0 + rr < nkeys, p.status))
+                    wRec[h * kTcWarpCap + pos] =
                         make_int4((int)(A(c + 3) << 8) + (int)A(c + 2),
                                   (int)(A(c + 1) << 8) + (int)A(c), tok0 + rr, 0);
                 }
               }
             }
+            __syncwarp();
+            // a region that might not hold another tile's keys is flushed now
+            bool near_full = false;
+#pragma unroll
+            for (int h = 0; h < G; ++h) near_full |= wCnt[h] > (unsigned)(kTcWarpCap - 128);
+            if (near_full) flush((unsigned)(kTcWarpCap - 128));
           }
         }
       }
       if (MODE == kModeFilter) {
-        // The run's staged candidates: scored in fp64, tested against tau_h
-        // exactly, and written with one global atomic per warp and head.
-        // Epilogue warp h takes head h.
-        named_sync(1, 32 * kTcEpiWarps);
-        const int h = warp - kTcEpiWarp0;
-        if (h < G && s_ccount[h] > (unsigned)kTcCandCap) {
-          // more keys passed than the staging holds: the merge answers this
-          // head exactly (a count above the buffer's capacity sends it to the
-          // fallback)
-          if (lane == 0) {
-            atomicMax(&p.counts[head0 + h], 0x7fffffffu);
-            s_ccount[h] = 0u;
-          }
-        } else if (h < G) {
-          const unsigned nc = min(s_ccount[h], (unsigned)kTcCandCap);
-          unsigned long long *dst = p.cand + (head0 + h) * p.cap;
-          const float tau = s_tau[h];
-          for (unsigned i0 = 0; i0 < nc; i0 += 32) {
-            const unsigned i = i0 + lane;
-            bool keep = false;
-            unsigned long long cv = 0ull;
-            if (i < nc) {
-              const int4 rec = sRec[h * kTcCandCap + i];
-              const float sc = tc_record_score(sHdr, h, rec.x, rec.y, (uint32_t)rec.z);
-              keep = sc >= tau;
-              cv = composite(sc, (uint32_t)rec.z);
-            }
-            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-            unsigned base = 0;
-            if (lane == 0 && bal) base = atomicAdd(&p.counts[head0 + h], (unsigned)__popc(bal));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (keep) {
-              const int64_t pos = (int64_t)base + __popc(bal & ((1u << lane) - 1u));
-              if (pos < p.cap && in_bounds(head0 + h < (int64_t)p.S * p.h_q, p.status)) dst[pos] = cv;
-            }
-          }
-          __syncwarp();
-          if (lane == 0) s_ccount[h] = 0u;
-        }
+        flush(0u);  // the run's remaining staged candidates
       }
     } else if (warp == kTcMmaWarp0) {
       // -------------------------------------------------------------- MMA --
