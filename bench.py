@@ -617,16 +617,17 @@ def run_native(args):
         c.codes = synthkv.make_case(cfg["seed"], cfg["n"], h_kv, h_q, d, cfg["q_dtype"],
                                     device=device, keep_keys=False).codes
         cn = case_numpy(c)
-        heads = list(range(8))
+        heads = list(range(min(8, h_q)))
         secs = oracle_sample(cn, B, k, heads, args.uniform)
         cpu = {"value": len(heads) * c.n / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "query heads 0-7 (KV heads 0-1) of this step: allocation, fp64 scores "
-                         "of all %d keys, brute-force top-%d; single thread, %.1f s" % (c.n, k, secs)}
+               "sample": "query heads 0-%d of this step: allocation, fp64 scores of all %d "
+                         "keys, brute-force top-%d; single thread, %.1f s"
+                         % (len(heads) - 1, c.n, k, secs)}
 
     if rank == 0:
         traffic = None
         if not ragged and not host:
-            traffic = profiled_traffic(cfg["name"] + ("_uniform" if args.uniform else ""),
+            traffic = profiled_traffic("%s_b%d%s" % (cfg["name"], B, "_uniform" if args.uniform else ""),
                                        "bit_plane_kv_scan_b200/csrc/scan.cu"
                                        if flags else "bit_plane_kv_scan_b200/csrc/scan_tc.cu")
         res = {

@@ -1018,25 +1018,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
                                                               int sort_cap) {
   grid_dependency_wait();
   allow_dependent_launch();
-  if (blockIdx.x == 0) {
-    // union planes of every (session, KV head), from the plan headers
-    __shared__ unsigned s_up[32];
-    unsigned v = 0;
-    for (int gid = threadIdx.x; gid < p.S * p.h_kv; gid += blockDim.x) {
-      const unsigned char *plan = p.plans + (size_t)gid * p.plan_stride;
-      v += (p.flags & FATHOM_FLAG_CUDA_CORES)
-               ? (unsigned)reinterpret_cast<const PlanHeader *>(plan)->union_planes
-               : (unsigned)*reinterpret_cast<const int *>(plan);  // the tc plan's P
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    if ((threadIdx.x & 31) == 0) s_up[threadIdx.x >> 5] = v;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      unsigned t = 0;
-      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += s_up[w];
-      p.status->union_planes = t;
-    }
+  // union planes of every (session, KV head), from the plan headers: the
+  // block of each KV head's first query head adds its group's
+  if (threadIdx.x == 0 && blockIdx.x % p.G == 0) {
+    const unsigned char *plan = p.plans + (size_t)(blockIdx.x / p.G) * p.plan_stride;
+    atomicAdd(&p.status->union_planes,
+              (p.flags & FATHOM_FLAG_CUDA_CORES)
+                  ? (unsigned)reinterpret_cast<const PlanHeader *>(plan)->union_planes
+                  : (unsigned)*reinterpret_cast<const int *>(plan));  // the tc plan's P
   }
   // [sort_cap] placed candidates, then [sort_cap] ranked (sort_cap = 8 blockDim >= kpow2)
   extern __shared__ unsigned long long s_out[];

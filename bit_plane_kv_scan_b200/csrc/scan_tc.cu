@@ -1066,7 +1066,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
               if (tok0 + rr >= nkeys) cm &= ~(0x1111u << rr);
           }
           // stage each key that passed (rare: one in a few hundred) as its exact
-          // parts in this warp's region (positions from ballots: no atomics)
+          // parts in this warp's region
           if (__any_sync(0xffffffffu, cm != 0u)) {
 #pragma unroll
             for (int h = 0; h < G; ++h) {

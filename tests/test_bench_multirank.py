@@ -128,7 +128,10 @@ def test_reference_arm_uniform_allocation():
 
 def test_profile_traffic_needs_matching_workload():
     src = "bit_plane_kv_scan_b200/csrc/scan_tc.cu"
-    assert bench.profiled_traffic("decode_1m_uniform", src) is None
+    assert bench.profiled_traffic("decode_1m_b92_uniform", src) is None
+    assert bench.profiled_traffic("decode_1m_b136", src) is None  # another budget, other bytes
     assert bench.profiled_traffic("no_such_workload", src) is None
-    t = bench.profiled_traffic("decode_1m", src)
+    t = bench.profiled_traffic("decode_1m_b92", src)
     assert t is None or t > 155_000_000  # at least the algorithmic union bytes when current
+    t = bench.profiled_traffic("decode_1m_b92", "bit_plane_kv_scan_b200/csrc/scan.cu")
+    assert t is None or t > 155_000_000
