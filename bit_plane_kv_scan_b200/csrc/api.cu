@@ -469,4 +469,9 @@ fathom_status fathom_scan_read_report(const void *ws, fathom_scan_report *report
   return ok();
 }
 
+fathom_status fathom_check_device_status(const void *ws, void *stream) {
+  fathom_scan_report r;
+  return fathom_scan_read_report(ws, &r, stream);
+}
+
 }  // extern "C"

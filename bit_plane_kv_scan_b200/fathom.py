@@ -44,7 +44,7 @@ EXPORTED = [
     "fathom_scan_topk",
     "fathom_scan_topk_batched_workspace_size", "fathom_scan_topk_batched",
     "fathom_scan_read_report", "fathom_profile_scan_kernel", "fathom_scan_topk_noalloc",
-    "fathom_scan_read_report_noalloc", "fathom_merge_topk",
+    "fathom_scan_read_report_noalloc", "fathom_check_device_status", "fathom_merge_topk",
     "fathom_sparse_attention",
 ]
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -143,6 +143,8 @@ def lib() -> ctypes.CDLL:
         L.fathom_scan_topk_batched.argtypes = [ctypes.POINTER(BatchedArgs), vp, sz, vp]
         L.fathom_scan_read_report.restype = ci
         L.fathom_scan_read_report.argtypes = [vp, ctypes.POINTER(ScanReport), vp]
+        L.fathom_check_device_status.restype = ci
+        L.fathom_check_device_status.argtypes = [vp, vp]
         L.fathom_profile_scan_kernel.restype = None
         L.fathom_profile_scan_kernel.argtypes = [vp, vp]
         L.fathom_scan_topk_noalloc.restype = ci
@@ -489,3 +491,11 @@ def read_report(workspace: Optional[Workspace] = None, device=None, stream=None)
     _check(lib().fathom_scan_read_report(_ptr(ws.buf[(-ws.buf.data_ptr()) % 256:]),
                                          ctypes.byref(rep), _stream(stream)))
     return rep
+
+
+def check_device_status(workspace: Optional[Workspace] = None, device=None, stream=None) -> None:
+    """Raises FathomError (ERR_DEVICE_CHECK) when the last scan on the
+    workspace recorded a device-side fault; synchronises the stream."""
+    ws = _workspace(workspace, device or "cuda")
+    _check(lib().fathom_check_device_status(_ptr(ws.buf[(-ws.buf.data_ptr()) % 256:]),
+                                            _stream(stream)))

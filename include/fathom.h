@@ -301,6 +301,15 @@ typedef struct fathom_scan_report {
 FATHOM_API fathom_status fathom_scan_read_report(const void *workspace, fathom_scan_report *report,
                                       void *stream);
 
+/* fathom_check_device_status -- FATHOM_OK when the last scan on `workspace`
+ * recorded no device-side fault, else FATHOM_ERR_DEVICE_CHECK with the count
+ * in fathom_last_error().  Faults are bounded mbarrier waits that gave up
+ * and, in the checked build (libfathom_checked.so, FATHOM_DEVICE_CHECKS),
+ * every guarded global or shared access that was out of range and skipped.
+ * Synchronises `stream`; FATHOM_ERR_INVALID_ARGUMENT for a workspace that is
+ * not device memory. */
+FATHOM_API fathom_status fathom_check_device_status(const void *workspace, void *stream);
+
 /* fathom_scan_read_report_noalloc -- the report of the last
  * fathom_scan_topk_noalloc on the current device (its status block lives in
  * the built-in scratch, whose address the caller never sees).  Same fields

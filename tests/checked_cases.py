@@ -36,7 +36,8 @@ def run():
         idx, sc = F.scan_topk(planes, case.qmin.to(dev), case.qscale.to(dev), q, alloc, k, n,
                               flags=flags)
         torch.cuda.synchronize()
-        rep = F.read_report()  # raises on a recorded device fault
+        F.check_device_status()  # raises on a recorded device fault
+        rep = F.read_report()
         assert rep.device_faults == 0
         codes, qd = case.codes.numpy(), case.q.numpy().astype(np.float64)
         want = oracle.allocate_heads(qd, case.sigma.numpy(), B)

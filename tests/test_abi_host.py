@@ -42,6 +42,21 @@ def test_every_declared_symbol_is_exported(L):
     assert sorted(F.EXPORTED) == names
 
 
+def test_checked_build_exports_the_same_symbols():
+    """The debug build (device bounds checks) is a drop-in for libfathom.so."""
+    fbuild.build()
+    assert os.path.exists(fbuild.LIB_CHECKED)
+    C = ctypes.CDLL(fbuild.LIB_CHECKED)
+    for name in declared_functions():
+        assert hasattr(C, name), name
+
+
+def test_check_device_status_rejects_a_host_workspace(L):
+    buf = ctypes.create_string_buffer(256)
+    assert L.fathom_check_device_status(None, None) == F.ERR_INVALID_ARGUMENT
+    assert L.fathom_check_device_status(ctypes.addressof(buf), None) == F.ERR_INVALID_ARGUMENT
+
+
 def test_plane_words(L):
     assert [L.fathom_plane_words(n) for n in (0, 1, 127, 128, 129, 1 << 20)] == \
         [0, 4, 4, 4, 8, 32768]

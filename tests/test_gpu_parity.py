@@ -289,6 +289,7 @@ def test_batched_descriptor_beyond_n_max(cuda_cores):
     rep = F.ScanReport()
     st = L.fathom_scan_read_report(ctypes.c_void_p(buf.data_ptr()), ctypes.byref(rep), None)
     assert st == F.ERR_DEVICE_CHECK and rep.device_faults == 1
+    assert L.fathom_check_device_status(ctypes.c_void_p(buf.data_ptr()), None) == F.ERR_DEVICE_CHECK
     i0, s0 = scan.outs[0]
     assert (_np(i0) == -1).all() and np.isneginf(_np(s0)).all()
     c = cases[1]
