@@ -164,6 +164,47 @@ def scores_at(codes_g, qmin_g, qscale_g, q_h, t_h, idx) -> np.ndarray:
     return out
 
 
+def _group_rows(qmin_g, qscale_g, n: int, token_group: int):
+    qmin_g = np.asarray(qmin_g, dtype=np.float32)
+    qscale_g = np.asarray(qscale_g, dtype=np.float32)
+    groups = (n + token_group - 1) // token_group
+    if token_group <= 0 or qmin_g.ndim != 2 or qmin_g.shape[0] < groups or \
+            qscale_g.shape != qmin_g.shape:
+        raise ValueError("per-group statistics must be [ceil(n / token_group), d]")
+    return qmin_g, qscale_g, groups
+
+
+def scores_from_codes_grouped(codes_g, qmin_g, qscale_g, q_h, t_h, token_group: int) -> np.ndarray:
+    """Scores under per-token-group quantiser statistics (the quantiser variant
+    with one (m, s) per channel and run of token_group tokens; the pages give
+    no group size).  Key i dequantises with row i // token_group of qmin_g and
+    qscale_g ([groups][d]); so each group is scored exactly as a context of its
+    own by scores_from_codes."""
+    codes_g = np.asarray(codes_g)
+    n = codes_g.shape[0]
+    qmin_g, qscale_g, groups = _group_rows(qmin_g, qscale_g, n, token_group)
+    out = np.zeros(n, dtype=np.float64)
+    for j in range(groups):
+        t0, t1 = j * token_group, min(n, (j + 1) * token_group)
+        out[t0:t1] = scores_from_codes(codes_g[t0:t1], qmin_g[j], qscale_g[j], q_h, t_h)
+    return out
+
+
+def scores_at_grouped(codes_g, qmin_g, qscale_g, q_h, t_h, idx, token_group: int) -> np.ndarray:
+    """scores_from_codes_grouped at the listed keys only."""
+    codes_g = np.asarray(codes_g)
+    n = codes_g.shape[0]
+    qmin_g, qscale_g, groups = _group_rows(qmin_g, qscale_g, n, token_group)
+    idx = np.asarray(idx, dtype=np.int64)
+    out = np.zeros(idx.shape[0], dtype=np.float64)
+    for j in range(groups):
+        sel = np.nonzero(idx // token_group == j)[0]
+        if sel.size:
+            t0, t1 = j * token_group, min(n, (j + 1) * token_group)
+            out[sel] = scores_at(codes_g[t0:t1], qmin_g[j], qscale_g[j], q_h, t_h, idx[sel] - t0)
+    return out
+
+
 def scores_from_planes(planes_g, n: int, qmin_g, qscale_g, q_h, t_h) -> np.ndarray:
     planes_g = _c(planes_g, np.uint32)
     d = planes_g.shape[0]

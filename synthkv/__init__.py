@@ -28,6 +28,11 @@ synthetic, with this recipe per (session, KV head):
 The allocator's sigma_c input is the generator's population sigma_c
 (outliers included): it stands for calibrated channel statistics.
 
+Quantiser variant (token_group > 0): the same min-max quantiser applied to
+each run of token_group consecutive tokens on its own, so m and s are
+[h_kv, ceil(n / token_group), d] (the pages give no group size; per-channel
+statistics over the whole context are the default).
+
 Draws use a torch.Generator on the requested device, so a given seed gives
 the same case on the same device type and torch build.  Small cases are drawn
 on the CPU; the 1M-token cases are drawn on the GPU (the CPU draw of 1G
@@ -54,12 +59,13 @@ class KVCase:
     h_kv: int
     h_q: int
     codes: torch.Tensor        # uint8 [h_kv, n, d/2], low nibble = even channel
-    qmin: torch.Tensor         # float32 [h_kv, d]   (m_c)
-    qscale: torch.Tensor       # float32 [h_kv, d]   (s_c)
+    qmin: torch.Tensor         # float32 [h_kv, d] (m_c), or [h_kv, groups, d] per token group
+    qscale: torch.Tensor       # float32 [h_kv, d] (s_c), or [h_kv, groups, d] per token group
     sigma: torch.Tensor        # float32 [h_kv, d]   (population sigma_c)
     q: torch.Tensor            # float32 [h_q, d] holding the exact query values
     q_dtype: str               # "bf16" or "f32": the storage type handed to the library
     keys: Optional[torch.Tensor] = None  # float32 [h_kv, n, d] (kept for small cases)
+    token_group: int = 0       # tokens per quantiser group (0: the whole context)
 
     @property
     def group(self) -> int:
@@ -101,8 +107,11 @@ def _quantise_head(k: torch.Tensor):
 
 def make_case(seed: int, n: int, h_kv: int, h_q: int, d: int = 128,
               q_dtype: str = "bf16", device="cpu", keep_keys: Optional[bool] = None,
-              outliers: int = 4) -> KVCase:
-    """Draw one session: K cache of n tokens x h_kv heads x d channels and h_q queries."""
+              outliers: int = 4, token_group: int = 0) -> KVCase:
+    """Draw one session: K cache of n tokens x h_kv heads x d channels and h_q queries.
+
+    token_group > 0 quantises every run of token_group tokens with its own
+    min-max statistics (the draws are the same as for token_group = 0)."""
     if h_q % h_kv:
         raise ValueError("h_q must be a multiple of h_kv")
     if keep_keys is None:
@@ -121,19 +130,30 @@ def make_case(seed: int, n: int, h_kv: int, h_q: int, d: int = 128,
         sigma[g, out] *= 10.0
 
     codes = torch.empty(h_kv, n, d // 2, dtype=torch.uint8, device=dev)
-    qmin = torch.empty(h_kv, d, dtype=torch.float32, device=dev)
-    qscale = torch.empty(h_kv, d, dtype=torch.float32, device=dev)
+    ng = (n + token_group - 1) // token_group if token_group > 0 else 0
+    shape = (h_kv, ng, d) if token_group > 0 else (h_kv, d)
+    qmin = torch.empty(shape, dtype=torch.float32, device=dev)
+    qscale = torch.empty(shape, dtype=torch.float32, device=dev)
     q = torch.empty(h_q, d, dtype=torch.float32, device=dev)
     keys = torch.empty(h_kv, n, d, dtype=torch.float32, device=dev) if keep_keys else None
 
     for g in range(h_kv):
         k = torch.randn(n, d, generator=gen, device=dev, dtype=torch.float32)
         k.mul_(sigma[g]).add_(mu[g])
-        u, m32, s32 = _quantise_head(k)
-        codes[g] = pack_nibbles(u)
-        del u
-        qmin[g] = m32
-        qscale[g] = s32
+        if token_group > 0:
+            for j in range(ng):
+                t0, t1 = j * token_group, min(n, (j + 1) * token_group)
+                u, m32, s32 = _quantise_head(k[t0:t1])
+                codes[g, t0:t1] = pack_nibbles(u)
+                qmin[g, j] = m32
+                qscale[g, j] = s32
+            del u
+        else:
+            u, m32, s32 = _quantise_head(k)
+            codes[g] = pack_nibbles(u)
+            del u
+            qmin[g] = m32
+            qscale[g] = s32
         for hh in range(G):
             h = g * G + hh
             r = torch.randint(0, n, (4,), generator=gen, device=dev)
@@ -150,7 +170,7 @@ def make_case(seed: int, n: int, h_kv: int, h_q: int, d: int = 128,
         del k
 
     return KVCase(n=n, d=d, h_kv=h_kv, h_q=h_q, codes=codes, qmin=qmin, qscale=qscale,
-                  sigma=sigma, q=q, q_dtype=q_dtype, keys=keys)
+                  sigma=sigma, q=q, q_dtype=q_dtype, keys=keys, token_group=token_group)
 
 
 def make_ragged(seed: int, sessions: int, n_lo: int, n_hi: int, h_kv: int, h_q: int,

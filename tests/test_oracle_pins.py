@@ -415,6 +415,77 @@ def test_scores_at_matches_full_scores(small_gqa):
     np.testing.assert_array_equal(part, full[idx])
 
 
+# ------------------------------------------- per-token-group statistics --
+
+def _grouped_brute_force(u, m, s, q, t, token_group):
+    """Scalar loops straight from the cell-centre reconstruction, each key with
+    its own group's (m, s): u [n][d] codes, m/s [groups][d]."""
+    n, d = u.shape
+    out = np.zeros(n)
+    for i in range(n):
+        g = i // token_group
+        acc = 0.0
+        for c in range(d):
+            tc = int(t[c])
+            v = int(u[i, c]) >> (4 - tc)
+            w = 2.0 ** (4 - tc)
+            acc += q[c] * (float(m[g, c]) + float(s[g, c]) * (w * v + (w - 1.0) / 2.0))
+        out[i] = acc
+    return out
+
+
+def test_grouped_scores_brute_force():
+    """Key i must use group i // token_group's statistics: an off-by-one group,
+    a transposed (group, channel) index or a shared row all fail here."""
+    rng = np.random.default_rng(7)
+    n, d, tg = 300, 8, 128
+    u = rng.integers(0, 16, size=(n, d)).astype(np.uint8)
+    codes = (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+    groups = (n + tg - 1) // tg
+    m = rng.normal(size=(groups, d)).astype(np.float32)
+    s = rng.uniform(0.05, 2.0, size=(groups, d)).astype(np.float32)
+    q = rng.normal(size=d)
+    for t in (np.array([4, 3, 2, 1, 0, 4, 1, 2]), np.full(d, 4), np.zeros(d, dtype=int)):
+        got = oracle.scores_from_codes_grouped(codes, m, s, q, t.astype(np.uint8), tg)
+        want = _grouped_brute_force(u, m, s, q, t, tg)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12 * np.abs(want).max())
+        idx = np.array([0, 127, 128, 255, 256, 299, 5], dtype=np.int64)
+        np.testing.assert_array_equal(
+            oracle.scores_at_grouped(codes, m, s, q, t.astype(np.uint8), idx, tg), got[idx])
+
+
+def test_grouped_scores_reduce_to_per_channel(small_gqa):
+    """Every group holding the context's statistics, or one group spanning the
+    context, gives the per-channel scores."""
+    case = small_gqa
+    q = case.q.numpy().astype(np.float64)
+    t = oracle.allocate(q[2], case.sigma.numpy()[0], 92)
+    codes, m, s = case.codes.numpy()[0], case.qmin.numpy()[0], case.qscale.numpy()[0]
+    full = oracle.scores_from_codes(codes, m, s, q[2], t)
+    for tg in (64, 333, 1000, 4096):
+        groups = (case.n + tg - 1) // tg
+        got = oracle.scores_from_codes_grouped(codes, np.tile(m, (groups, 1)),
+                                               np.tile(s, (groups, 1)), q[2], t, tg)
+        np.testing.assert_array_equal(got, full)
+
+
+def test_grouped_quantiser_fixture_matches_per_range_statistics():
+    """synthkv's grouped variant: each run of token_group keys carries the
+    min/max statistics of its own keys, and its codes reconstruct them."""
+    tg = 512
+    case = synthkv.make_case(seed=12, n=1300, h_kv=1, h_q=1, d=32, q_dtype="f32",
+                             keep_keys=True, token_group=tg)
+    k = case.keys.numpy()[0].astype(np.float64)
+    assert case.qmin.shape == (1, 3, 32)
+    u = _unpack_codes(case.codes.numpy()[0])
+    for j in range(3):
+        kk = k[j * tg:(j + 1) * tg]
+        np.testing.assert_array_equal(case.qmin.numpy()[0, j], kk.min(0).astype(np.float32))
+        rec = case.qmin.numpy()[0, j].astype(np.float64) + \
+            case.qscale.numpy()[0, j].astype(np.float64) * u[j * tg:(j + 1) * tg]
+        assert np.all(np.abs(rec - kk) <= case.qscale.numpy()[0, j] * 0.5 + 1e-5)
+
+
 # ------------------------------------------------------------------- top-k --
 
 def test_topk_brute_force_with_ties():
