@@ -104,10 +104,11 @@ struct WsLayout {
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-WsLayout ws_layout(int S, int64_t n_max, int d, int h_q, int h_kv, int k, uint32_t flags) {
+WsLayout ws_layout(int S, int64_t n_max, int d, int h_q, int h_kv, int k, uint32_t flags,
+                   int n_tgroups = 1) {
   WsLayout L;
   const int64_t heads = (int64_t)S * h_q;
-  const int64_t groups = (int64_t)S * h_kv;
+  const int64_t groups = (int64_t)S * h_kv * n_tgroups;  // one plan each
   L.sample_rank = sample_rank_for(k);
   int64_t cap = 8 * (int64_t)k;
   if (cap < 512 * (int64_t)L.sample_rank) cap = 512 * (int64_t)L.sample_rank;
@@ -302,10 +303,28 @@ fathom_status fathom_sparse_attention(const fathom_attention_args *a, void *stre
   return ok();
 }
 
+// Plans per KV head of a single-session call: one per token group.
+static int tgroups_of(const fathom_scan_args *a) {
+  if (a->token_group <= 0 || a->n <= 0) return 1;
+  return (int)((a->n + a->token_group - 1) / a->token_group);
+}
+
+static fathom_status check_token_group(const fathom_scan_args *a) {
+  REQUIRE(a->token_group >= 0 && a->token_group % FATHOM_TOKEN_GROUP_QUANTUM == 0,
+          "token_group=%lld: need 0 or a positive multiple of %d", (long long)a->token_group,
+          FATHOM_TOKEN_GROUP_QUANTUM);
+  if (a->token_group > 0 && (a->flags & FATHOM_FLAG_CUDA_CORES))
+    return fail(FATHOM_ERR_UNSUPPORTED,
+                "per-token-group statistics are supported by the tensor-core scan only");
+  return FATHOM_OK;
+}
+
 static fathom_status check_scan_args(const fathom_scan_args *a) {
   REQUIRE(a != nullptr, "args is NULL");
   fathom_status st = check_scan_common(a->n, a->d, a->h_q, a->h_kv, a->k, a->q_dtype,
                                        a->planes_location);
+  if (st != FATHOM_OK) return st;
+  st = check_token_group(a);
   if (st != FATHOM_OK) return st;
   REQUIRE_DEV(a->qmin, "qmin");
   REQUIRE_DEV(a->qscale, "qscale");
@@ -329,15 +348,16 @@ static fathom_status check_scan_args(const fathom_scan_args *a) {
 
 size_t fathom_scan_topk_workspace_size(const fathom_scan_args *a) {
   if (a == nullptr || check_scan_common(a->n, a->d, a->h_q, a->h_kv, a->k, a->q_dtype,
-                                        a->planes_location) != FATHOM_OK)
+                                        a->planes_location) != FATHOM_OK ||
+      check_token_group(a) != FATHOM_OK)
     return 0;
-  return ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags).total;
+  return ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags, tgroups_of(a)).total;
 }
 
 fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_bytes, void *stream) {
   fathom_status st = check_scan_args(a);
   if (st != FATHOM_OK) return st;
-  const WsLayout L = ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags);
+  const WsLayout L = ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags, tgroups_of(a));
   REQUIRE_DEV(ws, "workspace");
   REQUIRE(aligned(ws, 256), "workspace must be 256-byte aligned");
   if (ws_bytes < L.total)
@@ -353,6 +373,8 @@ fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_by
   p.one.alloc = a->alloc;
   p.one.n = a->n;
   p.n_max = a->n;
+  p.token_group = a->token_group;
+  p.n_tgroups = tgroups_of(a);
   p.one.out_idx = a->out_idx;
   p.one.out_score = a->out_score;
   p.batched = 0;
@@ -409,6 +431,8 @@ fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, s
   memset(&p, 0, sizeof(p));
   p.sessions = a->sessions;
   p.n_max = a->n_max;
+  p.token_group = 0;
+  p.n_tgroups = 1;
   p.batched = 1;
   p.S = a->num_sessions;
   p.d = a->d;

@@ -113,6 +113,8 @@ struct ScanParams {
   int64_t cap;      // candidate capacity per query head
   int64_t m_max;    // sample slots per query head
   int64_t n_max;    // the workspace's bound on every session's n
+  int64_t token_group;  // keys per quantiser group (0: per channel over the context)
+  int n_tgroups;        // plans per (session, KV head): ceil(n / token_group), or 1
   // workspace
   uint32_t *zero;    // prefix of the workspace the plan kernel clears (status, counts, tau)
   int zero_words;
@@ -120,7 +122,7 @@ struct ScanParams {
   WsStatus *status;
   uint32_t *counts;  // [S * h_q] candidate counts
   uint32_t *tau;     // [S * h_q] threshold keys (0 = keep every key)
-  unsigned char *plans;  // [S * h_kv] plans
+  unsigned char *plans;  // [S * h_kv * n_tgroups] plans
   uint32_t *sample;      // [S * h_q][m_max] sampled keys
   unsigned long long *cand;  // [S * h_q][cap] composite (key << 32 | ~index)
   float *debug_scores;       // single session only

@@ -925,8 +925,10 @@ __device__ unsigned long long block_kth(const unsigned long long *a, int64_t cnt
 // Exact single-block answer for one head: stream all n keys, score each from
 // its allocated prefixes (accumulated in fp64 from the exact products
 // q_c s_c, rounded once to fp32), keep a candidate buffer above a running
-// k-th best, compact it when it fills.  Used when the sampled threshold
-// fails.  Returns the number of buffered candidates (= min(k, n)).
+// k-th best, compact it when it fills.  Under per-token-group statistics the
+// keys are streamed group by group, each with its own (m, s).  Used when the
+// sampled threshold fails.  Returns the number of buffered candidates
+// (= min(k, n)).
 __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned long long *buf,
                                  unsigned long long *s_sort, unsigned *hist, int *s_digit,
                                  unsigned *s_above) {
@@ -940,62 +942,69 @@ __device__ int64_t fallback_head(const ScanParams &p, int s, int hl, unsigned lo
   __shared__ double s_kc[32];
   __shared__ unsigned long long s_nbuf;
   __shared__ unsigned s_fill;
-  double kc = 0.0;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const int t = se.alloc[(int64_t)hl * d + c];
-    const float qv = load_q(se.q, p.q_bf16, (int64_t)hl * d + c);
-    const float m = se.qmin[(int64_t)g * d + c], sc = se.qscale[(int64_t)g * d + c];
-    s_t[c] = (uint8_t)t;
-    s_qs[c] = (double)qv * (double)sc;  // exact
-    const double cell = (double)(1 << (4 - t));
-    kc += (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) kc += __shfl_xor_sync(0xffffffffu, kc, off);
-  if ((threadIdx.x & 31) == 0) s_kc[threadIdx.x >> 5] = kc;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) s_t[c] = se.alloc[(int64_t)hl * d + c];
   if (threadIdx.x == 0) s_nbuf = 0;
-  __syncthreads();
-  double ksum = 0.0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) ksum += s_kc[w];
-  const double K = ksum;
   const uint32_t *gp = se.planes + (int64_t)g * d * 4 * W;
   unsigned long long theta = 0ull;
   const unsigned k = (unsigned)p.k;
-  for (int64_t base = 0; base < n; base += blockDim.x) {
-    const int64_t i = base + threadIdx.x;
-    if (i < n) {
-      double acc = K;
-      for (int c = 0; c < d; ++c) {
-        const int t = s_t[c];
-        if (t == 0) continue;
-        uint32_t y = 0;
-        for (int j = 0; j < t; ++j)
-          y |= ((gp[((int64_t)c * 4 + j) * W + (i >> 5)] >> (i & 31)) & 1u) << (3 - j);
-        acc = fma(s_qs[c], (double)y, acc);
-      }
-      const unsigned long long v = composite((float)acc, (uint32_t)i);
-      if (v > theta) {
-        const unsigned long long at = atomicAdd(&s_nbuf, 1ull);
-        if (in_bounds((int64_t)at < p.cap, p.status)) buf[at] = v;
-      }
+  const int64_t tgk = p.token_group > 0 ? p.token_group : (n > 0 ? n : 1);  // keys per (m, s)
+  int tg = 0;
+  for (int64_t g0 = 0; g0 < n; g0 += tgk, ++tg) {
+    __syncthreads();  // the previous group's s_qs and s_kc are no longer read
+    const int64_t srow = ((int64_t)g * p.n_tgroups + tg) * d;
+    double kc = 0.0;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+      const int t = s_t[c];
+      const float qv = load_q(se.q, p.q_bf16, (int64_t)hl * d + c);
+      const float m = se.qmin[srow + c], sc = se.qscale[srow + c];
+      s_qs[c] = (double)qv * (double)sc;  // exact
+      const double cell = (double)(1 << (4 - t));
+      kc += (double)qv * ((double)m + (double)sc * ((cell - 1.0) * 0.5));
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kc += __shfl_xor_sync(0xffffffffu, kc, off);
+    if ((threadIdx.x & 31) == 0) s_kc[threadIdx.x >> 5] = kc;
     __syncthreads();
-    const int64_t nb = (int64_t)s_nbuf;
-    if (nb > p.cap - (int64_t)blockDim.x) {
-      theta = block_kth(buf, nb, k, hist, s_digit, s_above);
-      if (threadIdx.x == 0) s_fill = 0;
-      __syncthreads();
-      for (int64_t j = threadIdx.x; j < nb; j += blockDim.x)
-        if (buf[j] >= theta) {
-          const unsigned at = atomicAdd(&s_fill, 1u);
-          if (at < k) s_sort[at] = buf[j];
+    double ksum = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) ksum += s_kc[w];
+    const double K = ksum;
+    const int64_t g1 = min(n, g0 + tgk);
+    for (int64_t base = g0; base < g1; base += blockDim.x) {
+      const int64_t i = base + threadIdx.x;
+      if (i < g1) {
+        double acc = K;
+        for (int c = 0; c < d; ++c) {
+          const int t = s_t[c];
+          if (t == 0) continue;
+          uint32_t y = 0;
+          for (int j = 0; j < t; ++j)
+            y |= ((gp[((int64_t)c * 4 + j) * W + (i >> 5)] >> (i & 31)) & 1u) << (3 - j);
+          acc = fma(s_qs[c], (double)y, acc);
         }
+        const unsigned long long v = composite((float)acc, (uint32_t)i);
+        if (v > theta) {
+          const unsigned long long at = atomicAdd(&s_nbuf, 1ull);
+          if (in_bounds((int64_t)at < p.cap, p.status)) buf[at] = v;
+        }
+      }
       __syncthreads();
-      for (int j = threadIdx.x; j < (int)k; j += blockDim.x) buf[j] = s_sort[j];
-      if (threadIdx.x == 0) s_nbuf = k;
-      __syncthreads();
-      // the k kept are the best so far; a later key matters only above the
-      // k-th of them, which is theta
+      const int64_t nb = (int64_t)s_nbuf;
+      if (nb > p.cap - (int64_t)blockDim.x) {
+        theta = block_kth(buf, nb, k, hist, s_digit, s_above);
+        if (threadIdx.x == 0) s_fill = 0;
+        __syncthreads();
+        for (int64_t j = threadIdx.x; j < nb; j += blockDim.x)
+          if (buf[j] >= theta) {
+            const unsigned at = atomicAdd(&s_fill, 1u);
+            if (at < k) s_sort[at] = buf[j];
+          }
+        __syncthreads();
+        for (int j = threadIdx.x; j < (int)k; j += blockDim.x) buf[j] = s_sort[j];
+        if (threadIdx.x == 0) s_nbuf = k;
+        __syncthreads();
+        // the k kept are the best so far; a later key matters only above the
+        // k-th of them, which is theta
+      }
     }
   }
   __syncthreads();
@@ -1021,7 +1030,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(ScanParams p, int 
   // union planes of every (session, KV head), from the plan headers: the
   // block of each KV head's first query head adds its group's
   if (threadIdx.x == 0 && blockIdx.x % p.G == 0) {
-    const unsigned char *plan = p.plans + (size_t)(blockIdx.x / p.G) * p.plan_stride;
+    const unsigned char *plan =
+        p.plans + (size_t)(blockIdx.x / p.G) * p.n_tgroups * p.plan_stride;  // token group 0's
     atomicAdd(&p.status->union_planes,
               (p.flags & FATHOM_FLAG_CUDA_CORES)
                   ? (unsigned)reinterpret_cast<const PlanHeader *>(plan)->union_planes

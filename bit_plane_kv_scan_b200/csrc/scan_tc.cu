@@ -378,7 +378,8 @@ __device__ __forceinline__ float tc_pow2_neg(int e) { return __int_as_float((127
 
 // ------------------------------------------------------------ plan kernel --
 
-// One block of 256 threads per (session, KV head); thread c is channel c.
+// One block of 256 threads per plan: (session, KV head, token group), the
+// token group only under per-token-group statistics; thread c is channel c.
 __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   grid_dependency_wait();
   allow_dependent_launch();
@@ -386,14 +387,17 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   // kernels after this one)
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_words; i += gridDim.x * blockDim.x)
     p.zero[i] = 0u;
-  const int gid = blockIdx.x;
+  const int pid = blockIdx.x;
+  const int gid = pid / p.n_tgroups;  // (session, KV head)
+  const int tg = pid - gid * p.n_tgroups;
   const int s = gid / p.h_kv;
   const int g = gid - s * p.h_kv;
   const fathom_session &se = session_of(p, s);
   const int d = p.d, G = p.G;
   const int c = threadIdx.x;
   const TcPlanLayout L = tc_plan_layout(d);
-  unsigned char *plan = p.plans + (size_t)gid * L.bytes;
+  unsigned char *plan = p.plans + (size_t)pid * L.bytes;
+  const int64_t srow = ((int64_t)g * p.n_tgroups + tg) * d;  // this plan's (m, s) row
   TcPlanHeader *hdr = reinterpret_cast<TcPlanHeader *>(plan);
   uint16_t *rows = reinterpret_cast<uint16_t *>(plan + L.off_rows);
   int8_t *bmat = reinterpret_cast<int8_t *>(plan + L.off_b);
@@ -410,8 +414,8 @@ __global__ void __launch_bounds__(256) tc_plan_kernel(ScanParams p) {
   double kpart[4] = {0.0, 0.0, 0.0, 0.0};  // its share of C_h
   int tstar = 0;
   if (c < d) {
-    const double m = se.qmin[(int64_t)g * d + c];
-    const double sc = se.qscale[(int64_t)g * d + c];
+    const double m = se.qmin[srow + c];
+    const double sc = se.qscale[srow + c];
     // fixed trip count, so that t, w and kpart stay in registers
 #pragma unroll
     for (int hh = 0; hh < 4; ++hh) {
@@ -538,6 +542,19 @@ __device__ __forceinline__ int64_t tc_tiles_per_group(int64_t n, const ScanParam
   return (plane_words(n) + kTcTileWords - 1) / kTcTileWords;
 }
 
+// Tiles per token group under per-token-group statistics (0 without them).
+// A filtering tile covers 1024 keys; a sample tile covers 65536 (it reads the
+// first 256-key sector of four 64-sector strides), and a token group is a
+// multiple of 65536 keys, so every tile lies in one token group.
+template <int MODE>
+__device__ __forceinline__ int tc_tiles_per_tgroup(const ScanParams &p) {
+  if (p.token_group <= 0) return 0;
+  const int64_t span = MODE == kModeSample
+                           ? (int64_t)kTcSampleSectorsPerTile * kSampleStride * kSectorWords * 32
+                           : (int64_t)kTcTileWords * 32;
+  return (int)(p.token_group / span);
+}
+
 struct TcLoc {
   int s, g, ti, per;
   int64_t n, W;
@@ -564,8 +581,10 @@ __device__ __forceinline__ TcLoc tc_locate(const ScanParams &p, const int *s_tpr
   return L;
 }
 
-// A block whose tiles span two (session, KV head) groups drains its pipeline
-// between them.  The filtering pass splits the tiles over the blocks on a
+// A block whose tiles span two plans ((session, KV head) groups, or token
+// groups) drains its pipeline between them.  The cost line charges the drain
+// at (session, KV head) boundaries only: token groups are 64 or more tiles
+// long, so a run crosses at most one or two of them.  The filtering pass splits the tiles over the blocks on a
 // cost line on which every group is preceded by that overhead, so that a
 // block that crosses a group boundary takes correspondingly fewer tiles.
 // Costs are in half tiles.
@@ -738,18 +757,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_scan_kernel(ScanParams p) {
   // same counts: they index the stages, slots, buffers and phases)
   uint32_t u0 = 0, tt0 = 0;
 
-  // ---- segments: runs of tiles that share one (session, KV head) ---------
+  // ---- segments: runs of tiles that share one plan -----------------------
   int t = t_begin;
   while (t < t_end) {
     __syncthreads();
     if (s_fault) break;
     const TcLoc L0 = tc_locate<MODE>(p, s_tprefix, t);
-    const int seg_end = min(t_end, t - L0.ti + L0.per);
+    // a segment is the run's tiles that share one plan (worked out by one
+    // thread: measured faster than every thread doing it)
+    if (tid == 0) {
+      const int tpg = tc_tiles_per_tgroup<MODE>(p);
+      const int tgx = tpg > 0 ? L0.ti / tpg : 0;
+      const int plan_end = tpg > 0 ? min(L0.per, (tgx + 1) * tpg) : L0.per;
+      s_tmp[2] = min(t_end, t - L0.ti + plan_end);
+      s_tmp[3] = tgx;
+    }
+    __syncthreads();
+    const int seg_end = s_tmp[2];
+    const int tg = s_tmp[3];
     const int ntiles = seg_end - t;
     const int ti0 = L0.ti;
     const int gid = L0.s * p.h_kv + L0.g;
     {
-      const unsigned char *gplan = p.plans + (size_t)gid * PL.bytes;
+      const unsigned char *gplan = p.plans + ((size_t)gid * p.n_tgroups + tg) * PL.bytes;
       const int nk = reinterpret_cast<const TcPlanHeader *>(gplan)->nks;
       const int used = PL.off_b + nk * kTcBStepBytes;
       for (int i = tid; i < used / 16; i += kTcThreads)
@@ -1184,7 +1214,8 @@ static cudaError_t launch_tc_gm(const ScanParams &p, int sms, cudaStream_t strea
 }
 
 cudaError_t launch_tc_plan(const ScanParams &p, cudaStream_t stream) {
-  return launch_dependent(tc_plan_kernel, dim3(p.S * p.h_kv), dim3(256), 0, stream, p);
+  return launch_dependent(tc_plan_kernel, dim3(p.S * p.h_kv * p.n_tgroups), dim3(256), 0, stream,
+                          p);
 }
 
 cudaError_t launch_tc_scan(const ScanParams &p, int mode, int sms, cudaStream_t stream) {

@@ -48,6 +48,7 @@ EXPORTED = [
     "fathom_sparse_attention",
 ]
 NOALLOC_SCRATCH_BYTES = 16 << 20
+TOKEN_GROUP_QUANTUM = 65536
 MAX_MERGE_PARTS = 64
 
 
@@ -66,6 +67,7 @@ class ScanArgs(ctypes.Structure):
         ("d", ctypes.c_int), ("h_q", ctypes.c_int), ("h_kv", ctypes.c_int), ("k", ctypes.c_int),
         ("out_idx", ctypes.c_void_p), ("out_score", ctypes.c_void_p),
         ("debug_scores", ctypes.c_void_p), ("flags", ctypes.c_uint32),
+        ("token_group", ctypes.c_int64),
     ]
 
 
@@ -313,7 +315,8 @@ def _workspace(ws: Optional[Workspace], device) -> Workspace:
 
 
 def scan_args(planes, qmin, qscale, q, alloc, k: int, n: int, out_idx, out_score,
-              debug_scores=None, flags: int = 0, host_mapped: bool = False) -> ScanArgs:
+              debug_scores=None, flags: int = 0, host_mapped: bool = False,
+              token_group: int = 0) -> ScanArgs:
     h_q, d = q.shape
     h_kv = qmin.shape[0]
     return ScanArgs(planes=planes.data_ptr(),
@@ -323,22 +326,26 @@ def scan_args(planes, qmin, qscale, q, alloc, k: int, n: int, out_idx, out_score
                     h_kv=h_kv, k=int(k), out_idx=out_idx.data_ptr(),
                     out_score=out_score.data_ptr(),
                     debug_scores=None if debug_scores is None else debug_scores.data_ptr(),
-                    flags=int(flags))
+                    flags=int(flags), token_group=int(token_group))
 
 
 def scan_topk(planes: torch.Tensor, qmin: torch.Tensor, qscale: torch.Tensor, q: torch.Tensor,
               alloc: torch.Tensor, k: int, n: int, *, host_mapped: bool = False,
               debug_scores: bool = False, flags: int = 0, workspace: Optional[Workspace] = None,
-              stream=None, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None):
+              stream=None, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+              token_group: int = 0):
     """Top-k keys per query head.  Returns (idx int32 [h_q,k], score f32 [h_q,k]) and,
-    with debug_scores=True, also every score f32 [h_q, n]."""
+    with debug_scores=True, also every score f32 [h_q, n].  token_group > 0 (a
+    multiple of TOKEN_GROUP_QUANTUM) takes qmin/qscale as [h_kv, groups, d]
+    statistics per run of token_group keys."""
     dev = q.device
     h_q = q.shape[0]
     if out is None:
         out = (torch.empty((h_q, k), dtype=torch.int32, device=dev),
                torch.empty((h_q, k), dtype=torch.float32, device=dev))
     dbg = torch.empty((h_q, n), dtype=torch.float32, device=dev) if debug_scores else None
-    args = scan_args(planes, qmin, qscale, q, alloc, k, n, out[0], out[1], dbg, flags, host_mapped)
+    args = scan_args(planes, qmin, qscale, q, alloc, k, n, out[0], out[1], dbg, flags, host_mapped,
+                     token_group)
     L = lib()
     need = L.fathom_scan_topk_workspace_size(ctypes.byref(args))
     if need == 0:

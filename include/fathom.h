@@ -208,7 +208,18 @@ typedef struct fathom_scan_args {
   float *out_score;        /* [h_q][k] out */
   float *debug_scores;     /* optional [h_q][n] out: every score (tests); NULL normally */
   uint32_t flags;          /* FATHOM_FLAG_* test knobs, 0 normally */
+  int64_t token_group;     /* 0: qmin/qscale are one (m, s) per channel over the whole
+                            * context (the default reading).  Else the quantiser variant
+                            * with statistics per run of token_group keys: a positive
+                            * multiple of FATHOM_TOKEN_GROUP_QUANTUM, qmin/qscale
+                            * [h_kv][ceil(n / token_group)][d], key i dequantised with row
+                            * i / token_group.  The tensor-core scan only:
+                            * FATHOM_ERR_UNSUPPORTED with FATHOM_FLAG_CUDA_CORES. */
 } fathom_scan_args;
+
+/* Token groups hold whole sample tiles (the sample pass reads one 256-key
+ * sector in 64 and four of those per 1024-key tile): 65536 keys. */
+#define FATHOM_TOKEN_GROUP_QUANTUM 65536
 
 /* Bytes of workspace fathom_scan_topk needs for these arguments (0 on bad
  * arguments).  The workspace is device memory, 256-byte aligned, owned by the

@@ -52,6 +52,31 @@ def run():
             check_topk(idx.cpu().numpy()[h], sc.cpu().numpy()[h], ref, k,
                        what="checked n=%d G=%d B=%d flags=%d head %d" % (n, G, B, flags, h), **tol)
         print("ok n=%d G=%d B=%d k=%d flags=%d" % (n, G, B, k, flags))
+    # per-token-group statistics: plans per token group, segments split at
+    # group boundaries, and the exact fallback walking the groups
+    for n, tg, k, flags in ((140001, 65536, 64, 0), (140001, 65536, 64, F.FLAG_FORCE_FALLBACK)):
+        case = synthkv.make_case(seed=977, n=n, h_kv=2, h_q=8, d=128, q_dtype="bf16",
+                                 token_group=tg)
+        q = case.q_storage().to(dev)
+        alloc = F.allocate(q, case.sigma.to(dev), 92)
+        planes = F.pack_planes(case.codes.to(dev))
+        idx, sc = F.scan_topk(planes, case.qmin.to(dev), case.qscale.to(dev), q, alloc, k, n,
+                              flags=flags, token_group=tg)
+        torch.cuda.synchronize()
+        F.check_device_status()
+        codes, qd = case.codes.numpy(), case.q.numpy().astype(np.float64)
+        want = oracle.allocate_heads(qd, case.sigma.numpy(), 92)
+        for h in range(8):
+            g = h // 4
+            m, s = case.qmin.numpy()[g], case.qscale.numpy()[g]
+            ref = oracle.scores_from_codes_grouped(codes[g], m, s, qd[h], want[h], tg)
+            if flags & F.FLAG_FORCE_FALLBACK:
+                tol = dict(floor=max(score_scale(qd[h], a, b) for a, b in zip(m, s)) / 8.0)
+            else:
+                tol = dict(abs_tol=max(fixed_point_bound(qd[h], b, want[h]) for b in s))
+            check_topk(idx.cpu().numpy()[h], sc.cpu().numpy()[h], ref, k,
+                       what="checked token groups flags=%d head %d" % (flags, h), **tol)
+        print("ok token_group=%d n=%d flags=%d" % (tg, n, flags))
     # the batched launch over ragged sessions
     sessions = [synthkv.make_case(seed=950 + i, n=n, h_kv=2, h_q=8, d=128, q_dtype="bf16")
                 for i, n in enumerate((9000, 20001, 3333))]

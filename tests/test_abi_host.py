@@ -156,6 +156,27 @@ def test_scan_workspace_size_and_limits(L):
     assert big >= 32 * 8 * (1 << 20)
 
 
+def test_token_group_arguments(L):
+    """Per-token-group statistics: a positive multiple of the quantum, tensor-core
+    scan only; the workspace grows by one plan per extra token group."""
+    for tg in (-65536, 1000, 65537, 3 * 65536 + 1):
+        a = _args(token_group=tg)
+        assert L.fathom_scan_topk_workspace_size(ctypes.byref(a)) == 0
+        assert L.fathom_scan_topk(ctypes.byref(a), None, 0, None) == F.ERR_INVALID_ARGUMENT
+        assert b"token_group" in L.fathom_last_error()
+    a = _args(token_group=65536, flags=F.FLAG_CUDA_CORES)
+    assert L.fathom_scan_topk_workspace_size(ctypes.byref(a)) == 0
+    assert L.fathom_scan_topk(ctypes.byref(a), None, 0, None) == F.ERR_UNSUPPORTED
+    # past the token-group checks, the null pointers are what is rejected
+    a = _args(token_group=65536)
+    assert L.fathom_scan_topk(ctypes.byref(a), None, 0, None) == F.ERR_INVALID_ARGUMENT
+    assert b"qmin" in L.fathom_last_error()
+    base = L.fathom_scan_topk_workspace_size(ctypes.byref(_args()))
+    for tg, groups in ((65536, 16), (1 << 20, 1), (1 << 21, 1), (3 * 65536, 6)):
+        size = L.fathom_scan_topk_workspace_size(ctypes.byref(_args(token_group=tg)))
+        assert size >= base and (size > base) == (groups > 1), (tg, size, base)
+
+
 def test_scan_rejects_before_launch(L):
     assert L.fathom_scan_topk(None, None, 0, None) == F.ERR_INVALID_ARGUMENT
     assert L.fathom_scan_topk(ctypes.byref(_args(h_q=24)), None, 0, None) == F.ERR_UNSUPPORTED

@@ -693,6 +693,65 @@ def test_append_token_by_token():
     np.testing.assert_array_equal(_planes_np(planes), oracle.pack_planes(_np(case.codes)))
 
 
+# ------------------------------------------- per-token-group statistics --
+
+def _group_tol(flags, q_h, qmin_gg, qscale_gg, t_h):
+    """_tol with the worst token group's bound (each group has its own Delta_h
+    and score scale)."""
+    if flags & (F.FLAG_CUDA_CORES | F.FLAG_FORCE_FALLBACK):
+        return dict(floor=max(score_scale(q_h, m, s) for m, s in zip(qmin_gg, qscale_gg)) / 8.0)
+    return dict(abs_tol=max(fixed_point_bound(q_h, s, t_h) for s in qscale_gg))
+
+
+@pytest.mark.parametrize("n,tg,k,flags", [(200003, 65536, 256, 0), (131072, 131072, 100, 0),
+                                          (70000, 65536, 1024, 0), (150001, 65536, 64, 2),
+                                          (140000, 65536, 300, 1), (65536, 65536 * 4, 50, 0)])
+def test_token_group_statistics(n, tg, k, flags):
+    """The quantiser variant with (m, s) per run of tg keys: dense scores and the
+    top-k of every head against the oracle's grouped scores (ragged last group,
+    one group spanning the context, forced fallback, no sampling)."""
+    case = synthkv.make_case(seed=70 + n % 97, n=n, h_kv=2, h_q=8, d=128, q_dtype="bf16",
+                             token_group=tg)
+    dev = torch.device("cuda")
+    q = case.q_storage().to(dev)
+    alloc = F.allocate(q, case.sigma.to(dev), 92)
+    planes = F.pack_planes(case.codes.to(dev))
+    idx, sc, dbg = F.scan_topk(planes, case.qmin.to(dev), case.qscale.to(dev), q, alloc, k, n,
+                               flags=flags, debug_scores=True, token_group=tg)
+    torch.cuda.synchronize()
+    assert F.read_report().device_faults == 0
+    codes, qmin, qscale = _np(case.codes), _np(case.qmin), _np(case.qscale)
+    qd = _np(case.q).astype(np.float64)
+    want = oracle.allocate_heads(qd, _np(case.sigma), 92)
+    np.testing.assert_array_equal(_np(alloc), want)
+    for h in range(8):
+        g = h // 4
+        ref = oracle.scores_from_codes_grouped(codes[g], qmin[g], qscale[g], qd[h], want[h], tg)
+        scale = max(score_scale(qd[h], m, s) for m, s in zip(qmin[g], qscale[g]))
+        check_dense(_np(dbg)[h], ref, scale, "tg=%d head %d" % (tg, h))
+        check_topk(_np(idx)[h], _np(sc)[h], ref, k, what="tg=%d flags=%d head %d" % (tg, flags, h),
+                   **_group_tol(flags, qd[h], qmin[g], qscale[g], want[h]))
+
+
+def test_token_groups_with_shared_statistics_change_nothing():
+    """Every token group holding the context's (m, s): the same top-k, bit for
+    bit, as the per-channel scan (the plans are equal; only the segments split)."""
+    n, tg, k = 300000, 65536, 500
+    case = synthkv.make_case(seed=88, n=n, h_kv=2, h_q=8, d=128, q_dtype="bf16")
+    dev = torch.device("cuda")
+    q = case.q_storage().to(dev)
+    alloc = F.allocate(q, case.sigma.to(dev), 92)
+    planes = F.pack_planes(case.codes.to(dev))
+    qmin, qscale = case.qmin.to(dev), case.qscale.to(dev)
+    groups = (n + tg - 1) // tg
+    qmin_g = qmin[:, None, :].expand(2, groups, 128).contiguous()
+    qscale_g = qscale[:, None, :].expand(2, groups, 128).contiguous()
+    i0, s0 = F.scan_topk(planes, qmin, qscale, q, alloc, k, n)
+    i1, s1 = F.scan_topk(planes, qmin_g, qscale_g, q, alloc, k, n, token_group=tg)
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1) and torch.equal(s0, s1)
+
+
 # ---------------------------------------------------- token-range sharding --
 
 @pytest.mark.parametrize("cuts,k", [((0, 3000, 9000), 50), ((0, 1, 4096, 4097, 20000), 300),
