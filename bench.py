@@ -67,6 +67,9 @@ def parse(argv=None):
     ap.add_argument("--uniform", action="store_true",
                     help="allocate the budget query-independently (the same depth in every "
                          "channel, fathom_allocate_uniform) instead of by water-filling")
+    ap.add_argument("--token-group", type=int, default=0,
+                    help="quantiser statistics per run of this many keys (a multiple of 65536; "
+                         "0 = per channel over the context)")
     ap.add_argument("--attention", action="store_true",
                     help="also time the sparse attention over each head's top-k (the step after "
                          "the scan; random bf16 K/V rows of the workload's shape), outside the step")
@@ -264,9 +267,11 @@ def profiled_traffic(workload, kernel_source):
             return int(fields["traffic_bytes_per_launch"])
     return None
 
-def workload_desc(cfg, budget, k, uniform=False):
+def workload_desc(cfg, budget, k, uniform=False, token_group=0):
     how = (", uniform allocation (the same depth in every channel for every query head)"
            if uniform else "")
+    if token_group:
+        how += ", quantiser statistics per %d-key token group" % token_group
     if cfg["name"] == "ragged_32_sessions":
         return ("ragged_32_sessions: 32 sessions, n ~ U[%d, %d] keys each, %d KV heads x d=%d, "
                 "%d %s query heads (GQA %d), B=%d bits/key%s, top-k=%d, one batched launch set" % (
@@ -291,7 +296,7 @@ def union_plane_bytes(alloc, n, h_kv, words):
 
 # ------------------------------------------------------------ CPU oracle --
 
-def oracle_sample(case_np, budget, k, heads, uniform=False):
+def oracle_sample(case_np, budget, k, heads, uniform=False, token_group=0):
     """Oracle allocation + scores + top-k for the listed query heads; returns seconds."""
     import oracle
     codes, qmin, qscale, q, sigma = case_np
@@ -304,7 +309,10 @@ def oracle_sample(case_np, budget, k, heads, uniform=False):
             t = oracle.allocate_uniform(1, d, budget)[0]
         else:
             t = oracle.allocate(q[h], sigma[g], budget)
-        s = oracle.scores_from_codes(codes[g], qmin[g], qscale[g], q[h], t)
+        if token_group:
+            s = oracle.scores_from_codes_grouped(codes[g], qmin[g], qscale[g], q[h], t, token_group)
+        else:
+            s = oracle.scores_from_codes(codes[g], qmin[g], qscale[g], q[h], t)
         oracle.topk(s, k)
     return time.perf_counter() - t0
 
@@ -331,11 +339,13 @@ def run_reference(args):
                                    cfg["h_q"], cfg["d"], cfg["q_dtype"], device=dev)[0]
     else:
         case = synthkv.make_case(cfg["seed"], cfg["n"], cfg["h_kv"], cfg["h_q"], cfg["d"],
-                                 cfg["q_dtype"], device=dev, keep_keys=False)
+                                 cfg["q_dtype"], device=dev, keep_keys=False,
+                                 token_group=args.token_group)
     cn = case_numpy(case)
+    tg = args.token_group if cfg["name"] != "ragged_32_sessions" else 0
     for i in range(args.warmup):
-        oracle_sample(cn, args.budget, k, [i % cfg["h_q"]], args.uniform)
-    secs = [oracle_sample(cn, args.budget, k, [(args.warmup + i) % cfg["h_q"]], args.uniform)
+        oracle_sample(cn, args.budget, k, [i % cfg["h_q"]], args.uniform, tg)
+    secs = [oracle_sample(cn, args.budget, k, [(args.warmup + i) % cfg["h_q"]], args.uniform, tg)
             for i in range(args.steps)]
     t = float(np.mean(secs))
     value = case.n / t / 1e9
@@ -346,7 +356,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, synthkv)",
-        "config": {"workload": workload_desc(cfg, args.budget, k, args.uniform),
+        "config": {"workload": workload_desc(cfg, args.budget, k, args.uniform, tg),
                    "budget_bits": args.budget,
                    "k": k, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -403,6 +413,9 @@ def run_native(args):
     flags = F.FLAG_CUDA_CORES if args.cuda_cores else 0
     ragged = cfg["name"] == "ragged_32_sessions"
     host = cfg["name"] == "host_resident_1m"
+    tg = args.token_group
+    if tg and ragged:
+        raise SystemExit("--token-group applies to the single-session workloads")
     ws = F.Workspace(device)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
@@ -412,7 +425,7 @@ def run_native(args):
                                     cfg["n_hi"], h_kv, h_q, d, cfg["q_dtype"], device=device)
     else:
         cases = [synthkv.make_case(cfg["seed"] + rank, cfg["n"], h_kv, h_q, d, cfg["q_dtype"],
-                                   device=device, keep_keys=False)]
+                                   device=device, keep_keys=False, token_group=tg)]
     S = len(cases)
     q_all = torch.cat([c.q_storage() for c in cases]).contiguous()
     sigma_all = torch.cat([c.sigma for c in cases]).contiguous()
@@ -456,7 +469,8 @@ def run_native(args):
             def step():
                 allocate(q_src)
                 F.scan_topk(planes[0], c.qmin, c.qscale, q_src, alloc_all, k, c.n,
-                            host_mapped=host, flags=flags, workspace=ws, out=outs[0])
+                            host_mapped=host, flags=flags, workspace=ws, out=outs[0],
+                            token_group=tg)
         return step
 
     step = make_step(q_all)
@@ -615,10 +629,10 @@ def run_native(args):
         oracle.build()
         c = cases[0]
         c.codes = synthkv.make_case(cfg["seed"], cfg["n"], h_kv, h_q, d, cfg["q_dtype"],
-                                    device=device, keep_keys=False).codes
+                                    device=device, keep_keys=False, token_group=tg).codes
         cn = case_numpy(c)
         heads = list(range(min(8, h_q)))
-        secs = oracle_sample(cn, B, k, heads, args.uniform)
+        secs = oracle_sample(cn, B, k, heads, args.uniform, tg)
         cpu = {"value": len(heads) * c.n / secs / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "query heads 0-%d of this step: allocation, fp64 scores of all %d "
                          "keys, brute-force top-%d; single thread, %.1f s"
@@ -627,7 +641,8 @@ def run_native(args):
     if rank == 0:
         traffic = None
         if not ragged and not host:
-            traffic = profiled_traffic("%s_b%d%s" % (cfg["name"], B, "_uniform" if args.uniform else ""),
+            traffic = profiled_traffic("%s_b%d%s%s" % (cfg["name"], B, "_uniform" if args.uniform else "",
+                                                        "_tg%d" % tg if tg else ""),
                                        "bit_plane_kv_scan_b200/csrc/scan.cu"
                                        if flags else "bit_plane_kv_scan_b200/csrc/scan_tc.cu")
         res = {
@@ -636,7 +651,7 @@ def run_native(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded, synthkv: Qwen3-8B-shaped GQA keys with outlier "
                     "channels, 4-bit min-max codes)",
-            "config": {"workload": workload_desc(cfg, B, k, args.uniform), "sessions_per_rank": S,
+            "config": {"workload": workload_desc(cfg, B, k, args.uniform, tg), "sessions_per_rank": S,
                        "keys_per_rank": n_total, "h_kv": h_kv, "h_q": h_q, "d": d,
                        "budget_bits": B, "k": k, "scan_kernel": "cuda-core" if flags else "tcgen05",
                        "allocation": "uniform" if args.uniform else "water-filling",
