@@ -14,8 +14,9 @@
 // runs on 8 SMs per head.  Warp w of the head's 64 takes the selected rows
 // w * U .. w * U + U - 1, then the next 64 U, ...; each lane holds d / 32
 // consecutive dimensions of q, of the running output and of every row it
-// loads.  A warp first issues the loads (K and V, bf16) of its U rows (U = 8
-// up to d = 128, else 4), then folds them into an online softmax in base 2
+// loads.  A warp first issues the loads (K and V) of its U rows (U = 8 up to
+// d = 128, else 4), reduces their U dot products across the warp together,
+// then folds them into an online softmax in base 2 with one rescale per pass
 // (q pre-scaled by scale * log2 e).  Each CTA merges its 8 warps' partial
 // (max, sum, output) in shared memory; CTA 0 of the cluster merges the 8 CTA
 // partials through distributed shared memory and writes the result.
@@ -39,7 +40,8 @@ constexpr int kAttnSplit = 8;  // CTAs per query head: one cluster
 constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;            // per CTA
 constexpr int kAttnHeadWarps = kAttnSplit * kAttnWarps;  // per head
-// rows a warp has in flight
+// rows a warp has in flight (a pass): their loads are issued together, and
+// their scores reduced and folded into the online softmax together
 __host__ __device__ constexpr int attn_rows(int dpl) { return dpl <= 4 ? 8 : 4; }
 
 struct AttnParams {
@@ -147,46 +149,88 @@ __global__ void __cluster_dims__(kAttnSplit, 1, 1) __launch_bounds__(kAttnThread
 #pragma unroll
   for (int i = 0; i < DPL; ++i) o[i] = 0.0f;
 
-  for (int r0 = (rank * kAttnWarps + warp) * kAttnRows; r0 < a.k;
-       r0 += kAttnHeadWarps * kAttnRows) {
-    int row[kAttnRows];  // n < 2^31
+  // A pass: kAttnRows rows of this warp, their loads issued together.  Two
+  // passes are in flight: the loads of the next pass are issued before the
+  // current one is folded in, so their latency overlaps its arithmetic.
+  struct Pass {
+    int row[kAttnRows];  // -1: no selected row (n < 2^31)
     uint32_t kw[kAttnRows][CODES ? 1 : NW], vw[kAttnRows][NW];
+  };
+  auto load_pass = [&](int r0, Pass &ps) {
 #pragma unroll
     for (int u = 0; u < kAttnRows; ++u) {
       const int r = r0 + u;
       const int32_t x = r < a.k ? __ldg(ix + r) : -1;
-      row[u] = (x >= 0 && (int64_t)x < a.n) ? x : -1;
-      if (row[u] >= 0) {
+      ps.row[u] = (x >= 0 && (int64_t)x < a.n) ? x : -1;
+      if (ps.row[u] >= 0) {
         if constexpr (CODES)
-          kw[u][0] = load_codes_part<DPL>(Cg + (int64_t)row[u] * (D / 2), c0);
+          ps.kw[u][0] = load_codes_part<DPL>(Cg + (int64_t)ps.row[u] * (D / 2), c0);
         else
-          load_row_part<DPL>(Kg + (int64_t)row[u] * D, kw[u]);
-        load_row_part<DPL>(Vg + (int64_t)row[u] * D, vw[u]);
+          load_row_part<DPL>(Kg + (int64_t)ps.row[u] * D, ps.kw[u]);
+        load_row_part<DPL>(Vg + (int64_t)ps.row[u] * D, ps.vw[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < (CODES ? 1 : NW); ++i) ps.kw[u][i] = 0u;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) ps.vw[u][i] = 0u;
       }
     }
+  };
+  auto fold_pass = [&](const Pass &ps) {
+    // the pass's dot products: lane partials, then all kAttnRows warp sums at
+    // once (independent shuffles), so the rows share the reduction latency
+    float sc[kAttnRows];
 #pragma unroll
     for (int u = 0; u < kAttnRows; ++u) {
-      if (row[u] < 0) continue;  // the same for every lane of the warp
       float s = 0.0f;
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
         float kv;
         if constexpr (CODES)
-          kv = fmaf(ks[i], (float)((kw[u][0] >> (4 * i)) & 15u), km[i]);
+          kv = fmaf(ks[i], (float)((ps.kw[u][0] >> (4 * i)) & 15u), km[i]);
         else
-          kv = part_value(kw[u], i);
+          kv = part_value(ps.kw[u], i);
         s = fmaf(qv[i], kv, s);
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      const float mn = fmaxf(m, s);
-      const float corr = exp2f(m - mn);  // 0 for the first row (m = -inf)
-      const float p = exp2f(s - mn);
-      l = fmaf(l, corr, p);
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) o[i] = fmaf(o[i], corr, p * part_value(vw[u], i));
-      m = mn;
+      sc[u] = s;
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int u = 0; u < kAttnRows; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], off);
+    // one rescale per pass: the pass's largest score joins the running max
+    float mb = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kAttnRows; ++u)
+      if (ps.row[u] >= 0) mb = fmaxf(mb, sc[u]);  // the same for every lane of the warp
+    if (mb == -INFINITY) return;                  // no selected row in this pass
+    const float mn = fmaxf(m, mb);
+    const float corr = exp2f(m - mn);  // 0 while m = -inf
+    l *= corr;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) o[i] *= corr;
+#pragma unroll
+    for (int u = 0; u < kAttnRows; ++u) {
+      if (ps.row[u] < 0) continue;
+      const float pr = exp2f(sc[u] - mn);
+      l += pr;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) o[i] = fmaf(pr, part_value(ps.vw[u], i), o[i]);
+    }
+    m = mn;
+  };
+  const int rstep = kAttnHeadWarps * kAttnRows;
+  int r0 = (rank * kAttnWarps + warp) * kAttnRows;
+  Pass pa, pb;
+  if (r0 < a.k) load_pass(r0, pa);
+  while (r0 < a.k) {
+    if (r0 + rstep < a.k) load_pass(r0 + rstep, pb);
+    fold_pass(pa);
+    r0 += rstep;
+    if (r0 >= a.k) break;
+    if (r0 + rstep < a.k) load_pass(r0 + rstep, pa);
+    fold_pass(pb);
+    r0 += rstep;
   }
 
   if (lane == 0) {
