@@ -5,8 +5,8 @@ This module only draws inputs.  It holds none of the scan's arithmetic
 the CUDA library consume what it returns.
 
 What it draws (Fathom, "Fathom Makes KV-Cache Scans Query-Adaptive...",
-method paragraphs; arXiv 2609.17652 abstract): a 4-bit K cache "a quantized
-serving stack already holds", shaped like Qwen3-8B GQA layers (8 KV heads of
+method paragraphs; arXiv 2609.17652 abstract): the 4-bit K cache that a
+quantised serving stack keeps anyway, shaped like Qwen3-8B GQA layers (8 KV heads of
 d = 128 channels, 32 query heads), with contexts up to 1M tokens.  The pages
 use real models and sessions that are not available here, so every input is
 synthetic, with this recipe per (session, KV head):
