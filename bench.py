@@ -70,6 +70,9 @@ def parse(argv=None):
     ap.add_argument("--token-group", type=int, default=0,
                     help="quantiser statistics per run of this many keys (a multiple of 65536; "
                          "0 = per channel over the context)")
+    ap.add_argument("--append", action="store_true",
+                    help="also time fathom_append_planes: one decoded token into the store, "
+                         "in place, and a 128-token append that lengthens the rows")
     ap.add_argument("--attention", action="store_true",
                     help="also time the sparse attention over each head's top-k (the step after "
                          "the scan; random bf16 K/V rows of the workload's shape), outside the step")
@@ -563,6 +566,46 @@ def run_native(args):
     h2d = q_host.numel() * q_host.element_size()
     d2h = S * h_q * k * 8
 
+    append = None
+    if args.append and not ragged and not host:
+        # a decode step's append: the store of the first n - 256 tokens takes the
+        # next tokens one at a time (in place: the row length holds), then 128
+        # at once across a row-length boundary (a copy into the longer layout)
+        n1 = cases[0].n
+        codes = synthkv.make_case(cfg["seed"] + rank, n1, h_kv, h_q, d, cfg["q_dtype"],
+                                  device=device, keep_keys=False, token_group=tg).codes
+        n0 = n1 - 256
+        store = F.pack_planes(codes[:, :n0].contiguous())
+        one = [codes[:, n0 + i:n0 + i + 1].contiguous() for i in range(64)]
+        torch.cuda.synchronize()
+        ab = [torch.cuda.Event(enable_timing=True) for _ in range(64)]
+        ae = [torch.cuda.Event(enable_timing=True) for _ in range(64)]
+        for i in range(64):
+            ab[i].record(stream)
+            store = F.append_planes(store, n0 + i, one[i])
+            ae[i].record(stream)
+        torch.cuda.synchronize()
+        t_one = float(np.median([x.elapsed_time(y) for x, y in zip(ab[3:], ae[3:])]))
+        n2 = n0 + 64
+        n2r = ((n2 + 127) // 128) * 128  # fill to the row boundary, then cross it
+        store = F.append_planes(store, n2, codes[:, n2:n2r].contiguous())
+        blk = codes[:, n2r:n2r + 128].contiguous()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        grown = F.append_planes(store, n2r, blk)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_grow = e0.elapsed_time(e1)
+        moved = 2 * F.lib().fathom_planes_bytes(n2r, d, h_kv)  # read and written once
+        hbm_peak, hbm_kind = load_peaks()
+        append = {"kernels": ["append_bits_kernel", "append_copy_kernel"],
+                  "one_token_in_place_us": t_one * 1e3,
+                  "grow_128_tokens_us": t_grow * 1e3,
+                  "grow_bytes": moved, "grow_achieved_gbs": moved / (t_grow * 1e-3) / 1e9,
+                  "grow_frac": moved / (t_grow * 1e-3) / 1e9 / hbm_peak, "peak_kind": hbm_kind}
+        del store, grown, codes, one, blk
+
     attention = None
     if args.attention and not ragged:
         # the step after the scan, timed on its own: each head's attention over
@@ -673,6 +716,8 @@ def run_native(args):
             res["cpu_baseline"] = cpu
         if attention is not None:
             res["attention"] = attention
+        if append is not None:
+            res["append"] = append
         print(json.dumps(res))
     if world > 1:
         import torch.distributed as dist
