@@ -197,8 +197,8 @@ FATHOM_API fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits
 typedef struct fathom_scan_args {
   const uint32_t *planes;  /* [h_kv][d][4][W] (device, or host-mapped pinned) */
   int planes_location;     /* fathom_planes_location */
-  const float *qmin;       /* [h_kv][d] m_c, float */
-  const float *qscale;     /* [h_kv][d] s_c, float */
+  const float *qmin;       /* [h_kv][d] m_c, float ([h_kv][groups][d] with token_group) */
+  const float *qscale;     /* [h_kv][d] s_c, float ([h_kv][groups][d] with token_group) */
   const void *q;           /* [h_q][d], q_dtype */
   int q_dtype;             /* fathom_dtype */
   const uint8_t *alloc;    /* [h_q][d] from fathom_allocate */
