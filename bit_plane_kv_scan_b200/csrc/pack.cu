@@ -13,6 +13,8 @@
 // encodes.  The words are staged in shared memory and written out as
 // 128-byte row segments.  Integer and bit-exact; each byte of the store is
 // read and written once (HBM-bound).
+#include <type_traits>
+
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -116,13 +118,22 @@ static cudaError_t launch_pack_d(const uint8_t *codes, int64_t n, int h_kv, uint
 
 // Out-of-place step: word w < W_in of every row comes from the old store,
 // the rest of the new row is zero (padding, or about to receive new bits).
+// Row lengths are multiples of 4 words, so with 16-byte aligned stores the
+// copy moves whole 16-byte pieces (V = 4 words); else one word at a time.
+template <int V>
 __global__ void append_copy_kernel(const uint32_t *__restrict__ in, int64_t W_in,
                                    uint32_t *__restrict__ out, int64_t W_out, int64_t rows) {
-  const int64_t total = rows * W_out;
+  using Piece = typename std::conditional<V == 4, uint4, uint32_t>::type;
+  const Piece *src = reinterpret_cast<const Piece *>(in);
+  Piece *dst = reinterpret_cast<Piece *>(out);
+  const int64_t q_in = W_in / V, q_out = W_out / V;
+  const int64_t total = rows * q_out;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / W_out, w = i - r * W_out;
-    out[i] = w < W_in ? in[r * W_in + w] : 0u;
+    const int64_t r = i / q_out, w = i - r * q_out;
+    Piece v{};  // zero past the old row
+    if (w < q_in) v = src[r * q_in + w];
+    dst[i] = v;
   }
 }
 
@@ -158,9 +169,14 @@ cudaError_t launch_append(const uint8_t *codes, int64_t n, int64_t m, int d, int
   const int64_t W_in = plane_words(n), W_out = plane_words(n + m);
   const int64_t rows = (int64_t)h_kv * d * 4;
   if (planes_out != planes_in && rows * W_out > 0) {
-    const int64_t total = rows * W_out;
+    const bool wide = ((uintptr_t)planes_in % 16 == 0) && ((uintptr_t)planes_out % 16 == 0) &&
+                      W_in % 4 == 0 && W_out % 4 == 0;
+    const int64_t total = rows * W_out / (wide ? 4 : 1);
     const int blocks = (int)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
-    append_copy_kernel<<<blocks, 256, 0, stream>>>(planes_in, W_in, planes_out, W_out, rows);
+    if (wide)
+      append_copy_kernel<4><<<blocks, 256, 0, stream>>>(planes_in, W_in, planes_out, W_out, rows);
+    else
+      append_copy_kernel<1><<<blocks, 256, 0, stream>>>(planes_in, W_in, planes_out, W_out, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
