@@ -23,7 +23,15 @@
  *                        spread evenly over the channels (the fixed-depth
  *                        read that the adaptive allocation is compared with);
  *   fathom_sparse_attention    after the scan: each query head's attention
- *                        over only its selected keys.
+ *                        over only its selected keys;
+ *   fathom_merge_topk          token-range sharding: the top-k of the ranges'
+ *                        top-k lists;
+ *   fathom_scan_topk_noalloc   fathom_scan_topk on built-in scratch, for
+ *                        callers that cannot allocate;
+ *   fathom_scan_read_report, fathom_check_device_status    what the last
+ *                        scan on a workspace recorded (faults, fallbacks).
+ * fathom_scan_args.token_group selects the quantiser variant with (m, s) per
+ * run of token_group keys instead of per channel over the whole context.
  *
  * Conventions shared by every call
  *   - The caller owns every buffer.  The library never allocates or frees;
@@ -34,7 +42,7 @@
  *     prefixes across the host link.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     stream-ordered and asynchronous: none synchronises the host except
- *     fathom_scan_read_report.  Kernels are launched with programmatic
+ *     the report and status reads.  Kernels are launched with programmatic
  *     stream serialisation: one may be scheduled while the stream's previous
  *     kernel finishes, but waits for that kernel to complete before it reads
  *     or writes anything; ordering with the caller's own work is unchanged.
