@@ -18,7 +18,10 @@
 //   s_h = C_h + Delta_h 2^-e (65536 U + L)
 // (e below).  The epilogue decides a key against the head's threshold on U
 // alone, with a bound on |L| folded into an integer threshold per head, and
-// forms the fp32 score only for the keys that pass.
+// forms the fp32 score only for the keys that pass.  Under per-token-group
+// quantiser statistics m_c and s_c (so W, C_h and Delta_h) are those of the
+// key's token group: each token group has its own plan, and a run of tiles is
+// cut into segments at token-group boundaries.
 //
 // Layout (B200 design).  A tile is 1024 keys of one KV head: 32 plane words
 // per plane row.  Tensor-memory lane 32 q + l (quarter q, lane l) of M-block
@@ -44,8 +47,8 @@
 //    is staged in the warp's own shared-memory region as its exact integer
 //    parts (U, L, index); when a region might not hold another tile's keys,
 //    and at the end of a run, the warp scores its staged keys in fp64, tests
-//    them exactly and writes them to the workspace with one global atomic per
-//    32 keys (no barrier between epilogue warps);
+//    them exactly and writes them to the workspace, one global atomic per
+//    head reserving room for all of them (no barrier between epilogue warps);
 //  * build warps 8-15: warp (quarter q, parity) turns the T values of the
 //    K-steps of its parity into cells and stores them in the K-step's A slot
 //    with tcgen05.st;
