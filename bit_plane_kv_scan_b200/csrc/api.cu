@@ -8,6 +8,8 @@
 
 #include <cmath>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fathom_internal.cuh"
 
 namespace fathom {
@@ -171,6 +173,14 @@ namespace fathom {
 void set_error_message(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 }  // namespace fathom
 
+// An NVTX range over one ABI call, so that a trace (nsys, ncu's NVTX
+// filters) shows each call's launches under its name.  Without a tool
+// attached the push and pop do nothing.
+struct CallRange {
+  explicit CallRange(const char *name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+};
+
 extern "C" {
 
 const char *fathom_last_error(void) { return g_err; }
@@ -189,6 +199,7 @@ size_t fathom_planes_bytes(int64_t n, int d, int h_kv) {
 
 fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int d, int h_kv, uint32_t *planes,
                                  void *stream) {
+  const CallRange range("fathom_pack_planes");
   fathom_status st = check_shape(d, h_kv, h_kv);
   if (st != FATHOM_OK) return st;
   REQUIRE(n >= 0 && n < ((int64_t)1 << 31), "n=%lld out of range [0, 2^31)", (long long)n);
@@ -203,6 +214,7 @@ fathom_status fathom_pack_planes(const uint8_t *codes, int64_t n, int d, int h_k
 
 fathom_status fathom_append_planes(const uint8_t *codes, int64_t n, int64_t m, int d, int h_kv,
                                    const uint32_t *planes_in, uint32_t *planes_out, void *stream) {
+  const CallRange range("fathom_append_planes");
   fathom_status st = check_shape(d, h_kv, h_kv);
   if (st != FATHOM_OK) return st;
   REQUIRE(n >= 0 && m >= 0 && n + m < ((int64_t)1 << 31), "n=%lld m=%lld out of range",
@@ -229,6 +241,7 @@ fathom_status fathom_append_planes(const uint8_t *codes, int64_t n, int64_t m, i
 
 fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, const float *sigma, int h_q,
                               int h_kv, int d, int budget_bits, uint8_t *alloc, void *stream) {
+  const CallRange range("fathom_allocate");
   fathom_status st = check_shape(d, h_q, h_kv);
   if (st != FATHOM_OK) return st;
   REQUIRE(q_dtype == FATHOM_F32 || q_dtype == FATHOM_BF16, "q_dtype=%d unknown", (int)q_dtype);
@@ -245,6 +258,7 @@ fathom_status fathom_allocate(const void *q, fathom_dtype q_dtype, const float *
 
 fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits, uint8_t *alloc,
                                       void *stream) {
+  const CallRange range("fathom_allocate_uniform");
   fathom_status st = check_shape(d, h_q, 1);
   if (st != FATHOM_OK) return st;
   REQUIRE((int64_t)h_q * d < ((int64_t)1 << 30), "h_q=%d too large", h_q);
@@ -257,6 +271,7 @@ fathom_status fathom_allocate_uniform(int h_q, int d, int budget_bits, uint8_t *
 }
 
 fathom_status fathom_sparse_attention(const fathom_attention_args *a, void *stream) {
+  const CallRange range("fathom_sparse_attention");
   REQUIRE(a != nullptr, "args is NULL");
   fathom_status st = check_shape(a->d, a->h_q, a->h_kv);
   if (st != FATHOM_OK) return st;
@@ -355,6 +370,7 @@ size_t fathom_scan_topk_workspace_size(const fathom_scan_args *a) {
 }
 
 fathom_status fathom_scan_topk(const fathom_scan_args *a, void *ws, size_t ws_bytes, void *stream) {
+  const CallRange range("fathom_scan_topk");
   fathom_status st = check_scan_args(a);
   if (st != FATHOM_OK) return st;
   const WsLayout L = ws_layout(1, a->n, a->d, a->h_q, a->h_kv, a->k, a->flags, tgroups_of(a));
@@ -419,6 +435,7 @@ size_t fathom_scan_topk_batched_workspace_size(const fathom_batched_args *a) {
 
 fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, size_t ws_bytes,
                                        void *stream) {
+  const CallRange range("fathom_scan_topk_batched");
   fathom_status st = check_batched_args(a);
   if (st != FATHOM_OK) return st;
   const WsLayout L = ws_layout(a->num_sessions, a->n_max, a->d, a->h_q, a->h_kv, a->k, a->flags);
@@ -456,6 +473,7 @@ fathom_status fathom_scan_topk_batched(const fathom_batched_args *a, void *ws, s
 fathom_status fathom_merge_topk(const int32_t *in_idx, const float *in_score, int parts,
                                 const int64_t *offsets, int h_q, int k_in, int k, int32_t *out_idx,
                                 float *out_score, void *stream) {
+  const CallRange range("fathom_merge_topk");
   REQUIRE(parts >= 1 && parts <= FATHOM_MAX_MERGE_PARTS, "parts=%d out of range [1, %d]", parts,
           FATHOM_MAX_MERGE_PARTS);
   REQUIRE(h_q >= 1, "h_q=%d: need >= 1", h_q);
