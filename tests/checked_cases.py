@@ -28,8 +28,12 @@ def run():
              (3000, 4, 0, 50, 0), (3000, 4, 512, 50, 0), (40000, 4, 136, 64, F.FLAG_CUDA_CORES),
              (5000, 2, 92, 33, F.FLAG_CUDA_CORES), (40000, 4, 92, 64, F.FLAG_FORCE_FALLBACK),
              (20000, 4, 92, 64, F.FLAG_NO_SAMPLING)]
-    for n, G, B, k, flags in cases:
-        case = synthkv.make_case(seed=900 + n + G, n=n, h_kv=2, h_q=2 * G, d=128, q_dtype="bf16")
+    # tiny contexts and the narrowest channel count as well (n = 33, 64, 4096 at d = 32)
+    cases = [(n, G, B, k, flags, 128) for n, G, B, k, flags in cases] + \
+        [(33, 1, 17, 5, 0, 32), (64, 2, 92, 10, 0, 32), (4096, 4, 64, 50, 0, 32),
+         (64, 2, 92, 10, F.FLAG_CUDA_CORES, 32)]
+    for n, G, B, k, flags, d in cases:
+        case = synthkv.make_case(seed=900 + n + G, n=n, h_kv=2, h_q=2 * G, d=d, q_dtype="bf16")
         q = case.q_storage().to(dev)
         alloc = F.allocate(q, case.sigma.to(dev), B)
         planes = F.pack_planes(case.codes.to(dev))
