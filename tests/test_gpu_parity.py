@@ -316,6 +316,13 @@ def test_k_larger_than_n_and_empty():
 
 
 @pytest.mark.parametrize("cuda_cores", [False, True])
+def test_largest_k(cuda_cores):
+    """k = FATHOM_MAX_K (8192), the merge's largest output and sort."""
+    case = synthkv.make_case(seed=17, n=100000, h_kv=1, h_q=4, d=128, q_dtype="bf16")
+    _full_check(case, 92, 8192, flags=F.FLAG_CUDA_CORES if cuda_cores else 0, what="k=8192")
+
+
+@pytest.mark.parametrize("cuda_cores", [False, True])
 def test_report_counts_and_workspace_reuse(cuda_cores):
     """The report's union-plane count is the sum over KV heads of every
     channel's largest prefix in its query-head group (the bytes the scan
