@@ -740,6 +740,32 @@ def test_token_group_statistics(n, tg, k, flags):
                    **_group_tol(flags, qd[h], qmin[g], qscale[g], want[h]))
 
 
+@pytest.mark.parametrize("d", [64, 256])
+def test_token_groups_host_mapped_planes(d):
+    """Token groups with the planes in pinned host memory: the same answer as
+    from device memory, and the oracle's top-k."""
+    n, tg, k = 140000, 65536, 100
+    case = synthkv.make_case(seed=91, n=n, h_kv=1, h_q=4, d=d, q_dtype="bf16", token_group=tg)
+    dev = torch.device("cuda")
+    q = case.q_storage().to(dev)
+    alloc = F.allocate(q, case.sigma.to(dev), 92)
+    planes = F.pack_planes(case.codes.to(dev))
+    hp = torch.empty(planes.shape, dtype=planes.dtype, pin_memory=True)
+    hp.copy_(planes)
+    qmin, qscale = case.qmin.to(dev), case.qscale.to(dev)
+    i0, s0 = F.scan_topk(planes, qmin, qscale, q, alloc, k, n, token_group=tg)
+    i1, s1 = F.scan_topk(hp, qmin, qscale, q, alloc, k, n, token_group=tg, host_mapped=True)
+    torch.cuda.synchronize()
+    assert torch.equal(i0, i1) and torch.equal(s0, s1)
+    codes, m, s = _np(case.codes), _np(case.qmin), _np(case.qscale)
+    qd = _np(case.q).astype(np.float64)
+    want = oracle.allocate_heads(qd, _np(case.sigma), 92)
+    for h in range(4):
+        ref = oracle.scores_from_codes_grouped(codes[0], m[0], s[0], qd[h], want[h], tg)
+        check_topk(_np(i1)[h], _np(s1)[h], ref, k, what="host tg d=%d head %d" % (d, h),
+                   **_group_tol(0, qd[h], m[0], s[0], want[h]))
+
+
 def test_token_groups_with_shared_statistics_change_nothing():
     """Every token group holding the context's (m, s): the same top-k, bit for
     bit, as the per-channel scan (the plans are equal; only the segments split)."""
