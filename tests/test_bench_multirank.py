@@ -126,6 +126,19 @@ def test_reference_arm_uniform_allocation():
     assert out["config"]["budget_bits"] == 136
 
 
+def test_reference_arm_token_groups():
+    """The reference arm times the grouped oracle when --token-group is given."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--config", "tiny_4k",
+                        "--token-group", "65536"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    out = json.loads([ln for ln in r.stdout.splitlines() if ln.strip()][-1])
+    assert "65536-key token group" in out["config"]["workload"]
+    assert out["value"] > 0
+
+
 def test_profile_traffic_needs_matching_workload():
     src = "bit_plane_kv_scan_b200/csrc/scan_tc.cu"
     assert bench.profiled_traffic("decode_1m_b92_uniform", src) is None
